@@ -1,0 +1,253 @@
+"""Seeded synthetic FlashHead indices and queries.
+
+This module only builds inputs: embedding matrices E, the equal-size cluster-to-token table C2T,
+the centroids C (and their INT4 packing), hidden vectors h and target ids.  It performs none of
+the head's own arithmetic (scoring, selection, gathering, logits, sampling, Monte Carlo), so both
+the CUDA path and the CPU oracle can take their inputs from here.
+
+Recipe (the pages give no data; these shapes follow the heads the FlashHead pages evaluate —
+Llama-3.2-1B with hidden size 2048 and a 128,256-token vocabulary, c = 8016 clusters and p = 512
+probes as the default configuration, plus Gemma-3-1B and Qwen-3-0.6B shapes):
+
+* c unit centroids uniform on the sphere S^{d-1}.
+* b = v/c tokens per centroid: token = centroid + N(0, sigma^2 I) noise, L2-normalised, then scaled
+  by a norm drawn from U(0.8, 1.2).  A fraction ``heavy_frac`` of the token ids (chosen by a seeded
+  permutation) has its norm multiplied by ``heavy_mult`` to mimic frequent tokens.
+* Token ids are a seeded random permutation of the generation order; cluster k's row of C2T lists
+  the ids of the tokens generated from centroid k, sorted ascending, so every cluster holds exactly
+  b tokens (the equal-size constraint of FlashHead notes, Module 1) and C2T flattened is a
+  permutation of 0..v-1.
+* The stored centroid C[k] is the L2-normalised mean of the *stored* rows of cluster k (the centroid
+  update of FlashHead notes, Eq. 5), computed in float64 and rounded to the storage dtype.  This is
+  the offline index construction of the synthetic workload; no k-means iterations are run.
+* Queries h ~ N(0, I/d) * scale, rounded to the storage dtype.
+
+BF16 values are stored as uint16 bit patterns rounded to nearest even from float32.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import numpy as np
+
+# ----------------------------------------------------------------------------- bf16 helpers
+
+
+def bf16_from_f32(x: np.ndarray) -> np.ndarray:
+    """Round float32 values to bfloat16 (nearest, ties to even); returns uint16 bit patterns.
+
+    Inputs are finite by construction here; NaN handling is not needed."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return rounded.astype(np.uint16)
+
+
+def f32_from_bf16(u: np.ndarray) -> np.ndarray:
+    """Exact widening of bfloat16 bit patterns to float32."""
+    u = np.ascontiguousarray(u, dtype=np.uint16)
+    return (u.astype(np.uint32) << 16).view(np.float32)
+
+
+def stored_to_f64(a: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact float64 value of a stored array (float32 values or bf16 bit patterns)."""
+    if dtype == "f32":
+        return np.asarray(a, dtype=np.float32).astype(np.float64)
+    return f32_from_bf16(a).astype(np.float64)
+
+
+def store(x: np.ndarray, dtype: str) -> np.ndarray:
+    """Round float values to the storage dtype ("f32" -> float32, "bf16" -> uint16 patterns)."""
+    if dtype == "f32":
+        return np.ascontiguousarray(x, dtype=np.float32)
+    return bf16_from_f32(np.asarray(x, dtype=np.float32))
+
+
+# ----------------------------------------------------------------------------- configurations
+
+
+@dataclasses.dataclass(frozen=True)
+class HeadConfig:
+    """Shapes and generator parameters of one synthetic head."""
+
+    name: str
+    v: int
+    d: int
+    c: int
+    p: int
+    dtype: str                 # "f32" or "bf16"
+    noise: float               # sigma * sqrt(d) of the token noise
+    heavy_frac: float          # fraction of tokens with norm * heavy_mult
+    heavy_mult: float
+    h_scale: float             # h ~ N(0, I/d) * h_scale
+    data_seed: int
+    query_seed: int
+    tau: float = 1.0
+    int4: bool = False
+
+    @property
+    def b(self) -> int:
+        return self.v // self.c
+
+
+CONFIGS = {
+    # tiny greedy case: fp32, v=4096, d=256, 64 clusters of 64, 8 probes
+    "tiny": HeadConfig("tiny", v=4096, d=256, c=64, p=8, dtype="f32", noise=0.3,
+                       heavy_frac=0.0, heavy_mult=1.0, h_scale=1.0,
+                       data_seed=1000, query_seed=1001),
+    # Llama-3.2-1B-shaped head (greedy and sampling, tau = 0.8 for sampling)
+    "llama": HeadConfig("llama", v=128256, d=2048, c=8016, p=512, dtype="bf16", noise=0.5,
+                        heavy_frac=0.02, heavy_mult=3.0, h_scale=8.0,
+                        data_seed=2000, query_seed=2001, tau=0.8),
+    # Gemma-3-1B-shaped head with INT4 Stage-1 centroids
+    "gemma": HeadConfig("gemma", v=262144, d=1152, c=16384, p=1024, dtype="bf16", noise=0.5,
+                        heavy_frac=0.02, heavy_mult=3.0, h_scale=8.0,
+                        data_seed=4000, query_seed=4001, int4=True),
+    # Qwen-3-0.6B-shaped head for the Monte Carlo marginal, tau = 1.0
+    "qwen": HeadConfig("qwen", v=151936, d=1024, c=9496, p=512, dtype="bf16", noise=0.5,
+                       heavy_frac=0.02, heavy_mult=3.0, h_scale=8.0,
+                       data_seed=5000, query_seed=5001, tau=1.0),
+}
+
+SAMPLE_SEED = 0xF1A54EAD      # Philox seed of the sampling workload
+MC_SEED = 5000                 # Philox seed of the Monte Carlo workload
+MC_TARGET_SEED = 5002
+
+
+def scaled(cfg: HeadConfig, v: int, c: int, d: int | None = None, p: int | None = None,
+           name: str | None = None) -> HeadConfig:
+    """A smaller head with the same generator recipe (used for fast checks)."""
+    return dataclasses.replace(cfg, v=v, c=c, d=d if d is not None else cfg.d,
+                               p=p if p is not None else cfg.p,
+                               name=name or f"{cfg.name}-v{v}-c{c}")
+
+
+# ----------------------------------------------------------------------------- index
+
+
+@dataclasses.dataclass
+class Index:
+    cfg: HeadConfig
+    E: np.ndarray          # v x d, float32 or uint16 (bf16 patterns)
+    C: np.ndarray          # c x d, same dtype
+    C2T: np.ndarray        # c x b, int32
+    C_q4: np.ndarray | None = None      # c x d/2 uint8
+    C_scales: np.ndarray | None = None  # c x d/32 uint16 (bf16 patterns)
+
+    @property
+    def v(self):
+        return self.cfg.v
+
+    @property
+    def d(self):
+        return self.cfg.d
+
+    @property
+    def c(self):
+        return self.cfg.c
+
+    @property
+    def b(self):
+        return self.cfg.b
+
+
+def make_index(cfg: HeadConfig, chunk_clusters: int = 2048) -> Index:
+    """Build E, C, C2T (and the INT4 packing of C when cfg.int4) for one configuration."""
+    v, d, c = cfg.v, cfg.d, cfg.c
+    if v % c:
+        raise ValueError("v must be a multiple of c (equal-size clusters)")
+    b = v // c
+    rng = np.random.Generator(np.random.PCG64(cfg.data_seed))
+
+    # 1. unit centroids uniform on the sphere
+    cent = rng.standard_normal((c, d), dtype=np.float32)
+    cent /= np.linalg.norm(cent, axis=1, keepdims=True)
+
+    # 2. token ids: generation index g = k*b + j receives id perm[g]
+    perm = rng.permutation(v).astype(np.int64)
+    # 3. norms and the heavy-token subset (chosen among token ids)
+    norms = rng.uniform(0.8, 1.2, size=v).astype(np.float32)   # indexed by token id
+    n_heavy = int(math.floor(cfg.heavy_frac * v))
+    if n_heavy:
+        heavy_ids = rng.permutation(v)[:n_heavy]
+        norms[heavy_ids] *= np.float32(cfg.heavy_mult)
+
+    sigma = np.float32(cfg.noise / math.sqrt(d))
+    E = np.empty((v, d), dtype=np.float32 if cfg.dtype == "f32" else np.uint16)
+    for k0 in range(0, c, chunk_clusters):
+        k1 = min(c, k0 + chunk_clusters)
+        n = (k1 - k0) * b
+        tok = np.repeat(cent[k0:k1], b, axis=0)
+        tok += rng.standard_normal((n, d), dtype=np.float32) * sigma
+        tok /= np.linalg.norm(tok, axis=1, keepdims=True)
+        ids = perm[k0 * b:k1 * b]
+        tok *= norms[ids][:, None]
+        E[ids] = store(tok, cfg.dtype)
+
+    C2T = np.sort(perm.reshape(c, b), axis=1).astype(np.int32)
+
+    # 4. centroids: normalised mean of the stored rows of each cluster, in float64
+    C = np.empty((c, d), dtype=E.dtype)
+    for k0 in range(0, c, chunk_clusters):
+        k1 = min(c, k0 + chunk_clusters)
+        rows = stored_to_f64(E[C2T[k0:k1].reshape(-1)], cfg.dtype).reshape(k1 - k0, b, d)
+        mean = rows.mean(axis=1)
+        mean /= np.linalg.norm(mean, axis=1, keepdims=True)
+        C[k0:k1] = store(mean.astype(np.float32) if cfg.dtype == "bf16" else mean, cfg.dtype)
+
+    idx = Index(cfg, E, C, C2T)
+    if cfg.int4:
+        idx.C_q4, idx.C_scales = quantize_int4_g32(stored_to_f64(C, cfg.dtype))
+    return idx
+
+
+def quantize_int4_g32(x: np.ndarray):
+    """Symmetric 4-bit quantisation with one BF16 scale per group of 32 columns.
+
+    scale = bf16(float32(max|x| / 7)); q = clamp(round_half_even(x / scale), -8, 7), q = 0 where
+    scale == 0.  Packing: two values per byte, the low nibble holds the even column, two's complement.
+    Returns (packed uint8 [rows, d/2], scales uint16 bf16 patterns [rows, d/32])."""
+    rows, d = x.shape
+    if d % 32:
+        raise ValueError("d must be a multiple of 32 for INT4 groups")
+    g = x.reshape(rows, d // 32, 32)
+    amax = np.abs(g).max(axis=2)
+    scales_bits = bf16_from_f32((amax / 7.0).astype(np.float32))
+    scale = f32_from_bf16(scales_bits).astype(np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(scale[:, :, None] > 0, np.rint(g / scale[:, :, None]), 0.0)
+    q = np.clip(q, -8, 7).astype(np.int8).reshape(rows, d)
+    nib = (q.astype(np.int16) & 0xF).astype(np.uint8)
+    packed = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    return np.ascontiguousarray(packed), np.ascontiguousarray(scales_bits)
+
+
+def make_queries(cfg: HeadConfig, n: int, seed: int | None = None) -> np.ndarray:
+    """n hidden vectors h ~ N(0, I/d) * h_scale, rounded to the storage dtype."""
+    rng = np.random.Generator(np.random.PCG64(cfg.query_seed if seed is None else seed))
+    h = rng.standard_normal((n, cfg.d)) / math.sqrt(cfg.d) * cfg.h_scale
+    return store(h.astype(np.float32), cfg.dtype)
+
+
+def make_targets(v: int, n: int, t: int, seed: int = MC_TARGET_SEED) -> np.ndarray:
+    """n x t token ids drawn uniformly from [0, v)."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.integers(0, v, size=(n, t)).astype(np.int32)
+
+
+def random_index(v: int, d: int, c: int, seed: int, dtype: str = "f32") -> Index:
+    """A small unstructured index: E ~ N(0, 1/d) rows, random equal-size C2T, C = unit means.
+    Used for edge cases where clustered structure is not wanted."""
+    b = v // c
+    rng = np.random.Generator(np.random.PCG64(seed))
+    E = store(rng.standard_normal((v, d)).astype(np.float32) / np.float32(math.sqrt(d)), dtype)
+    C2T = np.sort(rng.permutation(v).reshape(c, b), axis=1).astype(np.int32)
+    rows = stored_to_f64(E[C2T.reshape(-1)], dtype).reshape(c, b, d).mean(axis=1)
+    rows /= np.linalg.norm(rows, axis=1, keepdims=True)
+    C = store(rows.astype(np.float32), dtype)
+    cfg = HeadConfig(f"random-{v}-{d}-{c}", v=v, d=d, c=c, p=min(c, 4), dtype=dtype, noise=0.0,
+                     heavy_frac=0.0, heavy_mult=1.0, h_scale=1.0, data_seed=seed,
+                     query_seed=seed + 1)
+    return Index(cfg, E, C, C2T)

@@ -42,8 +42,8 @@
  *   - Random numbers.  Sampling uses Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
  *     numbers: as easy as 1, 2, 3", SC'11) with key = (seed low 32 bits, seed high 32 bits) and
  *     counter = (elem >> 2, row, step low 32 bits, (stream << 24) | (step high 32 bits & 0xFFFFFF)),
- *     taking output word (elem & 3).  A draw x becomes u = ((x >> 8) + 0.5)·2^-24 ∈ (0,1) and the
- *     Gumbel variate G = -log(-log u).  Streams: FH_RNG_STAGE1 (Stage-1 keys, elem = cluster id),
+ *     taking output word (elem & 3).  A draw x becomes u = ((x >> 9) + 0.5)·2^-23 ∈ (0,1), which is
+ *     exact in fp32, and the Gumbel variate G = -log(-log u).  Streams: FH_RNG_STAGE1 (Stage-1 keys, elem = cluster id),
  *     FH_RNG_STAGE2 (Stage-2 and dense-head keys, elem = token id), FH_RNG_MC (Monte Carlo draws,
  *     elem = cluster id, step = draw index).  row = the query's index within the batch.
  */

@@ -26,7 +26,7 @@
  *   - the returned probe set is in ascending cluster id, candidates in slot order r*b + j;
  *   - sampling without replacement is realised as Gumbel-top-p, token sampling as Gumbel-max;
  *   - random numbers are Philox4x32-10 words with the counter layout of orc_draw_u32, mapped to
- *     u = ((x >> 8) + 0.5) * 2^-24 and G = -log(-log u);
+ *     u = ((x >> 9) + 0.5) * 2^-23 (exact in fp32 as well) and G = -log(-log u);
  *   - p(t|h,S) = 0 for a token outside the candidates of S; the standard error is the sample
  *     standard deviation (N-1 denominator) over sqrt(N).
  *
@@ -108,9 +108,10 @@ void orc_philox_words(uint64_t seed, uint64_t step, uint32_t row, uint32_t strea
   for (int64_t e = 0; e < n; ++e) out[e] = orc_draw_u32(seed, step, row, stream, (uint64_t)e);
 }
 
-/* u = ((x >> 8) + 0.5) * 2^-24 lies strictly inside (0, 1); G = -log(-log u) is a standard Gumbel
-   variate.  Both logarithms in double. */
-double orc_uniform(uint32_t x) { return ((double)(x >> 8) + 0.5) * (1.0 / 16777216.0); }
+/* u = ((x >> 9) + 0.5) * 2^-23 lies strictly inside (0, 1) and has at most 24 significant bits, so
+   an fp32 implementation can form it exactly too; G = -log(-log u) is a standard Gumbel variate.
+   Both logarithms in double. */
+double orc_uniform(uint32_t x) { return ((double)(x >> 9) + 0.5) * (1.0 / 8388608.0); }
 
 double orc_gumbel(uint32_t x) { return -log(-log(orc_uniform(x))); }
 

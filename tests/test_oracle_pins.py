@@ -68,12 +68,15 @@ def test_counter_layout(orc):
 
 
 def test_uniform_endpoints(orc):
-    assert orc.uniform(0) == 0.5 * 2.0 ** -24
-    assert orc.uniform(0xFFFFFFFF) == (2.0 ** 24 - 0.5) * 2.0 ** -24
+    assert orc.uniform(0) == 0.5 * 2.0 ** -23
+    assert orc.uniform(0xFFFFFFFF) == (2.0 ** 23 - 0.5) * 2.0 ** -23
+    # every value is exactly representable in fp32 (at most 24 significant bits)
+    for x in (0, 1 << 9, 0x7FFFFFFF, 0xFFFFFE00, 0xFFFFFFFF):
+        assert float(np.float32(orc.uniform(x))) == orc.uniform(x)
     assert 0.0 < orc.uniform(0) < orc.uniform(0xFFFFFFFF) < 1.0
     # G = -log(-log u) at the middle of the range
     x = 0x80000000
-    u = ((x >> 8) + 0.5) / 2 ** 24
+    u = ((x >> 9) + 0.5) / 2 ** 23
     assert orc.gumbel(x) == pytest.approx(-math.log(-math.log(u)), rel=0, abs=1e-15)
 
 
@@ -82,7 +85,7 @@ def test_gumbel_distribution(orc):
     n = 200_000
     words = orc.philox_words(12345, 3, 1, 0, n)
     g = np.array([orc.gumbel(int(x)) for x in words[:20000]])
-    u = (((words.astype(np.float64) // 256) + 0.5) / 2 ** 24)
+    u = (((words.astype(np.float64) // 512) + 0.5) / 2 ** 23)
     gall = -np.log(-np.log(u))
     np.testing.assert_allclose(g, gall[:20000], rtol=0, atol=1e-15)
     se_mean = math.pi / math.sqrt(6) / math.sqrt(n)

@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the FlashHead head on B200.
+
+Headline: the Llama-3.2-1B-shaped head (v=128256, d=2048, c=8016, p=512), greedy, batch 1,
+synthetic BF16 inputs resident in HBM; value = tokens/s (= calls/s at batch 1), with µs/call and the
+achieved HBM GB/s against the measured copy bandwidth.  L2 is flushed (256 MiB device write)
+before every timed call; each call is timed with CUDA events on the stream it runs on.
+
+The sweep (on by default) times the other rows of the path at their own shapes: batches 4/16/64,
+the in-run dense head, sampling, the Gemma-shaped INT4 Stage 1 and the Qwen-shaped Monte Carlo
+marginal.  `--impl reference` times the CPU oracle (fp64, host cores) on the same workload.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under torch.distributed.run,
+one independent replica per GPU (the head does not shard), time = max over ranks.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from clustered_retrieval_classification_b200 import costmodel, synth  # noqa: E402
+
+# A40 head latency the pages print for this workload (FlashHead summary, Table 3: TPOT^H 0.40 ms for
+# Llama-3.2-1B with c=8016, p=512, batch 1) -> 2500 tokens/s.  Context from other hardware.
+PAGES_TOKENS_PER_S = 1.0 / 0.40e-3
+
+# DRAM traffic per launch from the committed ncu captures (profiles/), valid only for the kernel
+# sources they were taken on (sha1 of the csrc files); null otherwise.
+TRAFFIC = {}
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha1()
+    d = os.path.join(ROOT, "clustered_retrieval_classification_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:12]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """Samples the SM clock and clock-event reasons through NVML every few ms (read-only)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= int(get_r(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in self.REASONS.items() if self.reasons & b],
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- timing
+
+
+class Timer:
+    def __init__(self, dist, flush):
+        self.dist, self.flush = dist, flush
+
+    def barrier(self):
+        if self.dist:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    def run(self, step_fn, K, W, sampler=None):
+        """W untimed steps, then K timed steps; L2 flushed before each step, outside the events.
+        Returns the per-step device times in ms (this rank)."""
+        for k in range(W):
+            self.flush()
+            step_fn(k)
+        self.barrier()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+        ctx = sampler if sampler is not None else _Null()
+        with ctx:
+            for k in range(K):
+                self.flush()
+                ev[k][0].record()
+                step_fn(W + k)
+                ev[k][1].record()
+            self.barrier()
+        return [a.elapsed_time(b) for a, b in ev]
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        pass
+
+
+def max_over_ranks(x: float, dist) -> float:
+    if not dist:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, dist) -> float:
+    if not dist:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- workloads
+
+
+def load_llama(F, cluster_major=True):
+    cfg = synth.CONFIGS["llama"]
+    idx = synth.make_index(cfg)
+    I = F.index_from_host(idx.E, idx.C, idx.C2T, "bf16", cluster_major=cluster_major)
+    return cfg, idx, I
+
+
+def unique_clusters(F, I, H, p, B, n_batches=8):
+    """Mean number of distinct clusters probed per batch (for the Stage-2 byte count)."""
+    us = []
+    for j in range(n_batches):
+        Hb = H[j * B:(j + 1) * B]
+        if Hb.shape[0] < B:
+            break
+        sel = torch.empty((B, p), dtype=torch.int32, device="cuda")
+        F.head_greedy(I, Hb, p, debug=dict(sel=sel))
+        us.append(int(torch.unique(sel).numel()))
+    return float(np.mean(us))
+
+
+def bench_head(F, T, I, Hd, cfg, B, K, W, mode="greedy", sampler=None, tau=0.8, int4=False):
+    p = cfg.p
+    pool = Hd.shape[0]
+    ws = I.workspace(F.FH_OP_SAMPLE if mode == "sample" else F.FH_OP_GREEDY, B, p)
+    out = torch.empty(B, dtype=torch.int32, device="cuda")
+
+    def step(k):
+        off = (k * B) % (pool - B + 1)
+        Hb = Hd[off:off + B]
+        if mode == "sample":
+            F.head_sample(I, Hb, p, tau, synth.SAMPLE_SEED, k, out=out, ws=ws)
+        else:
+            F.head_greedy(I, Hb, p, out=out, ws=ws)
+    ms = T.run(step, K, W, sampler)
+    return ms
+
+
+def bench_dense(F, T, I, Hd, B, K, W):
+    pool = Hd.shape[0]
+    ws = I.workspace(F.FH_OP_DENSE, B)
+    out = torch.empty(B, dtype=torch.int32, device="cuda")
+
+    def step(k):
+        off = (k * B) % (pool - B + 1)
+        F.dense_head(I, Hd[off:off + B], out=out, ws=ws)
+    return T.run(step, K, W)
+
+
+def gbs(bytes_, ms):
+    return bytes_ / (ms * 1e-3) / 1e9
+
+
+def summarize(ms_list):
+    return {"us_mean": 1e3 * statistics.fmean(ms_list), "us_median": 1e3 * statistics.median(ms_list),
+            "us_min": 1e3 * min(ms_list)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+
+def oracle_baseline(idx, H, p, budget_s=12.0):
+    import oracle
+    t0 = time.perf_counter()
+    oracle.head(idx, H[:1], p)
+    t1 = time.perf_counter() - t0
+    n = int(max(1, min(H.shape[0] - 1, budget_s / max(t1, 1e-6))))
+    t0 = time.perf_counter()
+    oracle.head(idx, H[1:1 + n], p)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} queries of the Llama-shaped greedy head (v=128256, d=2048, c=8016, "
+                      f"p=512), fp64 oracle, one batched call, {dt:.1f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: each step = one batch of the headline workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    cfg = synth.CONFIGS["llama"]
+    idx = synth.make_index(cfg)
+    H = synth.make_queries(cfg, max(512, args.batch * (args.steps + args.warmup) + 1))
+    B = args.batch
+    for k in range(args.warmup):
+        oracle.head(idx, H[k * B:(k + 1) * B], cfg.p)
+    t = []
+    for k in range(args.steps):
+        o = (args.warmup + k) * B
+        t0 = time.perf_counter()
+        oracle.head(idx, H[o:o + B], cfg.p)
+        t.append(time.perf_counter() - t0)
+    total = sum(t)
+    value = B * args.steps / total
+    line = {"impl": "reference", "metric": "head tokens/s at batch 1 (µs/call and HBM GB/s alongside)",
+            "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"llama-3.2-1b-shaped FlashHead greedy v=128256 d=2048 c=8016 "
+                                   f"p=512 batch {B}", "impl": "fp64 CPU oracle"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"{args.steps} timed steps of batch {B}"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = world > 1
+    torch.cuda.set_device(local)
+    if dist:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+
+    from clustered_retrieval_classification_b200 import flashhead as F
+    F.load()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    T = Timer(dist, lambda: flush_buf.fill_(1))
+    peak, peak_kind = measured_peaks()
+
+    cfg, idx, I = load_llama(F)
+    B = args.batch
+    Hh = synth.make_queries(cfg, 1024, seed=cfg.query_seed + 17 * rank)
+    Hd = F.device_array(Hh, "bf16")
+    sampler = ClockSampler(local)
+    ms = bench_head(F, T, I, Hd, cfg, B, args.steps, args.warmup, sampler=sampler)
+    ms_mean = statistics.fmean(ms)
+    total_ms = max_over_ranks(sum(ms), dist)
+    tokens = sum_over_ranks(B * args.steps, dist)
+    value = tokens / (total_ms * 1e-3)
+    U = cfg.p if B == 1 else unique_clusters(F, I, Hd, cfg.p, B)
+    bytes_call = costmodel.head_bytes(cfg.v, cfg.d, cfg.c, cfg.p, B, int(round(U)), 2)
+    achieved = gbs(bytes_call, ms_mean)
+
+    # stage-1 kernel alone (same kernel as inside the call)
+    s_out = torch.empty((B, cfg.c), dtype=torch.float32, device="cuda")
+    ws1 = I.workspace(F.FH_OP_DENSE, B)
+    ms_s1 = T.run(lambda k: F.stage1_scores(I, Hd[k % 512:k % 512 + B], out=s_out, ws=ws1),
+                  min(args.steps, 200), args.warmup)
+    s1_bytes = costmodel.stage1_bytes(cfg.c, cfg.d, 2) + B * cfg.d * 2 + B * cfg.c * 4
+
+    # end to end through the public API with pinned host buffers
+    h_host = torch.from_numpy(Hh.view(np.int16)).view(torch.bfloat16).pin_memory()
+    tok_host = torch.empty(B, dtype=torch.int32).pin_memory()
+    h_dev = torch.empty((B, cfg.d), dtype=torch.bfloat16, device="cuda")
+    tok_dev = torch.empty(B, dtype=torch.int32, device="cuda")
+    ws = I.workspace(F.FH_OP_GREEDY, B, cfg.p)
+
+    def e2e_step(k):
+        off = (k * B) % (1024 - B + 1)
+        h_dev.copy_(h_host[off:off + B], non_blocking=True)
+        F.head_greedy(I, h_dev, cfg.p, out=tok_dev, ws=ws)
+        tok_host.copy_(tok_dev, non_blocking=True)
+    ms_e2e = T.run(e2e_step, args.steps, args.warmup)
+    e2e_total = max_over_ranks(sum(ms_e2e), dist)
+    e2e_value = tokens / (e2e_total * 1e-3)
+
+    line = {
+        "metric": "head tokens/s at batch 1 (µs/call and HBM GB/s alongside)",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+        "us_per_call": 1e3 * ms_mean, "us_per_call_median": 1e3 * statistics.median(ms),
+        "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": value / PAGES_TOKENS_PER_S / world,
+        "vs_baseline_note": "per GPU vs the pages' A40 TPOT^H 0.40 ms (Table 3); other hardware",
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": f"llama-3.2-1b-shaped FlashHead greedy: v={cfg.v} d={cfg.d} "
+                               f"c={cfg.c} b={cfg.b} p={cfg.p} batch {B}",
+                   "batch": B, "parallelism": f"replicas x{world}" if dist else "single GPU",
+                   "l2": "flushed before every timed call (256 MiB device write, outside the events)",
+                   "inputs": "resident in HBM; a pool of 1024 distinct h, one per call"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": TRAFFIC.get(("head", B, csrc_hash())),
+                     "kernel": "fused head call: stage-1 GEMV + stage-2 (selection, C2T gather, "
+                               "dot, arg-max), PDL-chained",
+                     "algorithmic_bytes": bytes_call, "unique_clusters": U},
+        "stage1_roofline": {"achieved": gbs(s1_bytes, statistics.fmean(ms_s1)), "peak": peak,
+                            "frac": gbs(s1_bytes, statistics.fmean(ms_s1)) / peak,
+                            "us": 1e3 * statistics.fmean(ms_s1), "bytes": s1_bytes},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * cfg.d * 2,
+                "d2h_bytes_per_step": B * 4, "us_per_call": 1e3 * statistics.fmean(ms_e2e)},
+        "gpu_launches": 2 * args.steps if B == 1 else 3 * args.steps,
+        "clocks": sampler.summary(),
+    }
+
+    if not args.no_sweep and rank == 0:
+        line["sweep"] = sweep(F, T, I, cfg, idx, Hd, Hh, args, peak)
+    if not args.no_cpu and rank == 0:
+        line["cpu_baseline"] = oracle_baseline(idx, Hh, cfg.p)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def sweep(F, T, I, cfg, idx, Hd, Hh, args, peak):
+    K = min(args.steps, 100)
+    W = args.warmup
+    out = {}
+    # batches of the greedy head, and the in-run dense head
+    for B in (1, 4, 16, 64):
+        ms = bench_head(F, T, I, Hd, cfg, B, K, W)
+        U = cfg.p if B == 1 else unique_clusters(F, I, Hd, cfg.p, B)
+        by = costmodel.head_bytes(cfg.v, cfg.d, cfg.c, cfg.p, B, int(round(U)), 2)
+        s = summarize(ms)
+        g = gbs(by, statistics.fmean(ms))
+        out[f"greedy_b{B}"] = dict(s, tokens_per_s=B / (statistics.fmean(ms) * 1e-3), bytes=by,
+                                   unique_clusters=U, gbs=g, frac=g / peak)
+    for B in (1, 64):
+        ms = bench_dense(F, T, I, Hd, B, min(K, 30), W)
+        by = costmodel.dense_bytes(cfg.v, cfg.d, B, 2)
+        g = gbs(by, statistics.fmean(ms))
+        out[f"dense_b{B}"] = dict(summarize(ms), tokens_per_s=B / (statistics.fmean(ms) * 1e-3),
+                                  bytes=by, gbs=g, frac=g / peak)
+    for B in (1, 64):
+        ms = bench_head(F, T, I, Hd, cfg, B, K, W, mode="sample")
+        out[f"sample_b{B}"] = dict(summarize(ms), tokens_per_s=B / (statistics.fmean(ms) * 1e-3))
+    # top-1 agreement FlashHead vs dense on 256 queries (a statistic; no page number to match)
+    g = F.head_greedy(I, Hd[:64], cfg.p).cpu().numpy()
+    d = F.dense_head(I, Hd[:64]).cpu().numpy()
+    out["agreement_flashhead_vs_dense_top1"] = float(np.mean(g == d))
+    del I
+    torch.cuda.empty_cache()
+    # Gemma-shaped INT4 Stage 1
+    gcfg = synth.CONFIGS["gemma"]
+    gidx = synth.make_index(gcfg)
+    GI = F.index_from_host(gidx.E, gidx.C, gidx.C2T, "bf16", gidx.C_q4, gidx.C_scales, int4=True)
+    GB = F.index_from_host(gidx.E, gidx.C, gidx.C2T, "bf16")
+    GH = F.device_array(synth.make_queries(gcfg, 1024), "bf16")
+    for B in (1, 8, 32):
+        ms = bench_head(F, T, GI, GH, gcfg, B, K, W)
+        U = gcfg.p if B == 1 else unique_clusters(F, GI, GH, gcfg.p, B)
+        by = costmodel.head_bytes(gcfg.v, gcfg.d, gcfg.c, gcfg.p, B, int(round(U)), 2, int4=True)
+        gg = gbs(by, statistics.fmean(ms))
+        out[f"int4_b{B}"] = dict(summarize(ms), tokens_per_s=B / (statistics.fmean(ms) * 1e-3),
+                                 bytes=by, unique_clusters=U, gbs=gg, frac=gg / peak)
+    a = F.head_greedy(GI, GH[:64], gcfg.p).cpu().numpy()
+    b = F.head_greedy(GB, GH[:64], gcfg.p).cpu().numpy()
+    out["int4_agreement_with_bf16_stage1"] = float(np.mean(a == b))
+    del GI, GB
+    torch.cuda.empty_cache()
+    # Qwen-shaped Monte Carlo marginal: 16 h x 8 targets, N = 10000 draws each
+    qcfg = synth.CONFIGS["qwen"]
+    qidx = synth.make_index(qcfg)
+    QI = F.index_from_host(qidx.E, qidx.C, qidx.C2T, "bf16", cluster_major=False)
+    QH = F.device_array(synth.make_queries(qcfg, 16), "bf16")
+    tg = F.device_array(synth.make_targets(qcfg.v, 16, 8), "i32")
+    N = 10000
+    ws = QI.workspace(F.FH_OP_MC, 16, qcfg.p, 8, N)
+    ms = T.run(lambda k: F.mc_token_prob(QI, QH, tg, qcfg.p, 1.0, N, synth.MC_SEED, ws=ws), 3, 1)
+    mean, se = F.mc_token_prob(QI, QH, tg, qcfg.p, 1.0, N, synth.MC_SEED, ws=ws)
+    t = statistics.fmean(ms) * 1e-3
+    out["mc_qwen"] = {"ms_per_call": t * 1e3, "draws_per_s": 16 * N / t,
+                      "keys_per_s": 16 * N * qcfg.c / t, "max_se": float(se.max().item()),
+                      "B": 16, "T": 8, "N": N}
+    return out
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,894 @@
+// fh_kernels.cu — CUDA-core streaming kernels of the FlashHead head (sm_100a).
+//
+// Every kernel that reads rows of C or E streams them through shared memory with bulk copies
+// (cp.async.bulk on the TMA engine): each warp owns a private ring of K row slots, one mbarrier per
+// slot, and keeps K rows in flight while it computes the dot product of the previous one with the
+// query vector(s) held in shared memory.  Rows are the unit of work, so a C2T-indexed gather costs
+// the same as a contiguous stream: every row is 4 KiB of contiguous HBM at the Llama-shaped head.
+//
+// Kernels:
+//   k_stage1<E,QB>   s = C·h for QB queries per block; optional Gumbel-key epilogue   (Stage 1)
+//   k_stage1_int4<M> the same from INT4 centroids with BF16 group scales               (Stage 1, INT4)
+//   k_select<KPT>    top-p per query                                                    (selection)
+//   k_rows<E,MODE,KPT> candidates (fused selection or given sets) or all rows (dense):
+//                    dot, arg-max / Gumbel-max, partial results, last-block reduction   (Stage 2, dense)
+//   k_gather, k_cand_logits, k_gumbel_keys, k_philox                                    (single steps)
+//   k_validate_c2t, k_build_perm                                                        (index load)
+//   k_mc_*                                                                              (Monte Carlo)
+#include "fh_kernels.cuh"
+#include "fh_device.cuh"
+#include "fh_select.cuh"
+
+namespace fh {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kSelThreads = 512;
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Lane-partial dot product of a staged row (shared address row_s) with a staged query vector
+// (shared address h_s); nch = row bytes / 16.
+template <int ELEM>
+__device__ __forceinline__ float row_dot_partial(uint32_t row_s, uint32_t h_s, int nch, int lane) {
+  float acc = 0.0f;
+#pragma unroll 4
+  for (int ch = lane; ch < nch; ch += 32) {
+    const uint4 a = lds_v4(row_s + ch * 16);
+    const uint4 h = lds_v4(h_s + ch * 16);
+    acc = (ELEM == kBF16) ? dot8_bf16(a, h, acc) : dot4_f32(a, h, acc);
+  }
+  return acc;
+}
+
+// Copy `bytes` (multiple of 16) from global to shared memory with 16-byte loads by the whole block.
+__device__ __forceinline__ void block_copy_g2s(void* dst, const void* src, int bytes) {
+  for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(dst)[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
+}
+
+// The per-warp streaming loop.  Rows first, first+W, first+2W, ... below `hi` are brought into the
+// warp's ring (K slots of row_bytes) and handed to body(row, shared address) in order.  src(row)
+// gives the global address of a row.  Returns false if a wait timed out (status already set).
+template <typename Src, typename Body>
+__device__ __forceinline__ bool warp_stream_rows(int64_t first, int64_t hi, int W, int lane,
+                                                 uint8_t* ring, uint64_t* bars, int K,
+                                                 uint32_t row_bytes, const Src& src,
+                                                 const Body& body, uint32_t* status) {
+  if (first >= hi) return true;
+  const int64_t nw = (hi - first + W - 1) / W;
+  if (lane == 0) {
+    for (int n = 0; n < K && n < nw; ++n) {
+      mbar_arrive_expect_tx(&bars[n], row_bytes);
+      bulk_g2s(ring + (size_t)n * row_bytes, src(first + (int64_t)W * n), row_bytes, &bars[n]);
+    }
+  }
+  for (int64_t n = 0; n < nw; ++n) {
+    const int slot = (int)(n % K);
+    const uint32_t parity = (uint32_t)((n / K) & 1);
+    if (!mbar_wait(&bars[slot], parity, status)) {
+      // Give the copies still in flight a bounded chance to land before the block exits.
+      for (int64_t m = n + 1; m < nw && m < n + K; ++m)
+        mbar_wait(&bars[m % K], (uint32_t)((m / K) & 1), nullptr, 50000000ull);
+      return false;
+    }
+    body(first + (int64_t)W * n, smem_addr(ring + (size_t)slot * row_bytes));
+    __syncwarp();
+    if (lane == 0 && n + K < nw) {
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(&bars[slot], row_bytes);
+      bulk_g2s(ring + (size_t)slot * row_bytes, src(first + (int64_t)W * (n + K)), row_bytes,
+               &bars[slot]);
+    }
+  }
+  return true;
+}
+
+// ============================================================================ Stage 1 (dense C)
+
+template <int ELEM, int QB>
+__global__ void __launch_bounds__(kThreads) k_stage1(const Stage1Params prm, int K) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid < prm.n_tickets) prm.tickets_to_clear[tid] = 0u;
+
+  const uint32_t row_bytes = (uint32_t)(prm.d * (ELEM == kBF16 ? 2 : 4));
+  const int nch = (int)(row_bytes / 16);
+  const int q0 = blockIdx.y * QB;
+  const int nq = min(QB, prm.B - q0);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+  uint8_t* hs = smem + 1024;
+  uint8_t* ring = hs + (size_t)QB * row_bytes;
+
+  if (tid < kWarps * K) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
+  for (int q = 0; q < nq; ++q)
+    block_copy_g2s(hs + (size_t)q * row_bytes,
+                   static_cast<const uint8_t*>(prm.H) + (size_t)(q0 + q) * row_bytes, row_bytes);
+  __syncthreads();
+
+  const int64_t lo = prm.c * blockIdx.x / gridDim.x;
+  const int64_t hi = prm.c * (blockIdx.x + 1) / gridDim.x;
+  const uint8_t* C = static_cast<const uint8_t*>(prm.C);
+  const uint32_t hs_addr = smem_addr(hs);
+  auto src = [&](int64_t k) { return C + (size_t)k * row_bytes; };
+  auto body = [&](int64_t k, uint32_t row_s) {
+#pragma unroll
+    for (int q = 0; q < QB; ++q) {
+      if (q < nq) {
+        const float s = warp_sum(row_dot_partial<ELEM>(row_s, hs_addr + q * row_bytes, nch, lane));
+        if (lane == 0) {
+          float out = s;
+          if (prm.sample)
+            out = s / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)(q0 + q),
+                                                            prm.rng_stream, (uint32_t)k));
+          prm.out[(size_t)(q0 + q) * prm.c + k] = out;
+        }
+      }
+    }
+  };
+  warp_stream_rows(lo + warp, hi, kWarps, lane, ring + (size_t)warp * K * row_bytes, bars + warp * K,
+                   K, row_bytes, src, body, prm.status);
+}
+
+// ============================================================================ Stage 1 (INT4 C)
+// One query per blockIdx.y.  Lane l handles the 16-byte chunks l, l+32, ... of a row (one chunk =
+// one 32-column group), so its slice of h lives in registers as fp32.  A nibble n decodes to
+// q = (n ^ 8) - 8 through the float pattern 0x4B000000 | (n ^ 8) = 2^23 + (n ^ 8), exactly.
+
+__device__ __forceinline__ float int4_group_dot(const uint4 w, const float* hg) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+  float acc = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t even = (words[i] & 0x0F0F0F0Fu) ^ 0x08080808u;         // columns 8i + 0,2,4,6
+    const uint32_t odd = ((words[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // columns 8i + 1,3,5,7
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float qe = __uint_as_float(__byte_perm(even, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
+      const float qo = __uint_as_float(__byte_perm(odd, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
+      acc = fmaf(qe, hg[8 * i + 2 * j], acc);
+      acc = fmaf(qo, hg[8 * i + 2 * j + 1], acc);
+    }
+  }
+  return acc;
+}
+
+template <int MCH>
+__global__ void __launch_bounds__(kThreads) k_stage1_int4(const Stage1Params prm, int K,
+                                                          int rows_max) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid < prm.n_tickets) prm.tickets_to_clear[tid] = 0u;
+
+  const int q = blockIdx.y;
+  const int64_t d = prm.d;
+  const uint32_t row_bytes = (uint32_t)(d / 2);
+  const int nch = (int)(d / 32);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+  uint16_t* sc_s = reinterpret_cast<uint16_t*>(smem + 1024);
+  uint8_t* ring = smem + 1024 + (((size_t)rows_max * nch * 2 + 127) / 128) * 128;
+
+  const int64_t lo = prm.c * blockIdx.x / gridDim.x;
+  const int64_t hi = prm.c * (blockIdx.x + 1) / gridDim.x;
+  if (tid < kWarps * K) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
+  // the block's scales, row-major (hi-lo) x nch
+  for (int64_t i = tid; i < (hi - lo) * nch; i += kThreads) sc_s[i] = prm.scales[lo * nch + i];
+  // this lane's slice of h
+  float hreg[MCH][32];
+  const uint16_t* H = static_cast<const uint16_t*>(prm.H) + (size_t)q * d;
+#pragma unroll
+  for (int m = 0; m < MCH; ++m) {
+    const int ch = lane + 32 * m;
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+      hreg[m][e] = (ch < nch) ? __uint_as_float((uint32_t)H[32 * ch + e] << 16) : 0.0f;
+  }
+  __syncthreads();
+
+  auto src = [&](int64_t k) { return prm.q4 + (size_t)k * row_bytes; };
+  auto body = [&](int64_t k, uint32_t row_s) {
+    float part = 0.0f;
+#pragma unroll
+    for (int m = 0; m < MCH; ++m) {
+      const int ch = lane + 32 * m;
+      if (ch < nch) {
+        const uint4 w = lds_v4(row_s + ch * 16);
+        const float scale = __uint_as_float((uint32_t)sc_s[(k - lo) * nch + ch] << 16);
+        part = fmaf(scale, int4_group_dot(w, hreg[m]), part);
+      }
+    }
+    const float s = warp_sum(part);
+    if (lane == 0) {
+      float out = s;
+      if (prm.sample)
+        out = s / prm.tau +
+              gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, prm.rng_stream, (uint32_t)k));
+      prm.out[(size_t)q * prm.c + k] = out;
+    }
+  };
+  warp_stream_rows(lo + warp, hi, kWarps, lane, ring + (size_t)warp * K * row_bytes, bars + warp * K,
+                   K, row_bytes, src, body, prm.status);
+}
+
+// ============================================================================ single steps
+
+__global__ void k_gumbel_keys(const float* s, float* keys, int B, int64_t c, float tau, uint64_t seed,
+                              uint64_t step, uint32_t rng_stream) {
+  const int64_t n = (int64_t)B * c;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int q = (int)(i / c);
+    const uint32_t k = (uint32_t)(i % c);
+    keys[i] = s[i] / tau + gumbel_from_u32(philox_word(seed, step, (uint32_t)q, rng_stream, k));
+  }
+}
+
+__global__ void k_philox(uint64_t seed, uint64_t step, uint32_t row, uint32_t rng_stream, int64_t n,
+                         uint32_t* out) {
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x)
+    out[e] = philox_word(seed, step, row, rng_stream, (uint32_t)e);
+}
+
+__global__ void k_gather(const int32_t* C2T, int64_t b, const int32_t* sel, int B, int p,
+                         int32_t* cand) {
+  const int64_t P = (int64_t)p * b;
+  const int64_t n = (int64_t)B * P;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t q = i / P, slot = i % P;
+    cand[i] = C2T[(int64_t)sel[q * p + slot / b] * b + slot % b];
+  }
+}
+
+// One warp per candidate: z = E[tok]·h_q with 16-byte loads straight from global memory.
+template <int ELEM>
+__global__ void k_cand_logits(const void* E, int64_t d, const void* H, int B, const int32_t* cand,
+                              int64_t P, float* out_z) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t row_bytes = d * (ELEM == kBF16 ? 2 : 4);
+  const int nch = (int)(row_bytes / 16);
+  for (int64_t i = warp; i < (int64_t)B * P; i += nwarps) {
+    const int64_t q = i / P;
+    const uint8_t* row = static_cast<const uint8_t*>(E) + (size_t)cand[i] * row_bytes;
+    const uint8_t* h = static_cast<const uint8_t*>(H) + (size_t)q * row_bytes;
+    float acc = 0.0f;
+    for (int ch = lane; ch < nch; ch += 32) {
+      const uint4 a = ld_stream_v4(row + ch * 16);
+      const uint4 b = __ldg(reinterpret_cast<const uint4*>(h) + ch);
+      acc = (ELEM == kBF16) ? dot8_bf16(a, b, acc) : dot4_f32(a, b, acc);
+    }
+    acc = warp_sum(acc);
+    if (lane == 0) out_z[i] = acc;
+  }
+}
+
+// ============================================================================ selection kernel
+
+template <int KPT>
+__global__ void __launch_bounds__(kSelThreads) k_select(const float* keys, int32_t* sel, int64_t c,
+                                                        int p) {
+  __shared__ SelectSmem<kSelThreads> sm;
+  const int q = blockIdx.x;
+  const float* row = keys + (size_t)q * c;
+  float x[KPT];
+  const int base = threadIdx.x * KPT;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) x[j] = (base + j < c) ? row[base + j] : 0.0f;
+  block_select_topp<kSelThreads, KPT>(x, (int)c, p, sm, sel + (size_t)q * p);
+}
+
+// ============================================================================ rows + arg-max
+// MODE_FUSED: candidates of query blockIdx.y; the block first selects S itself from the Stage-1 keys.
+// MODE_SEL:   candidates of query blockIdx.y from the given probe sets.
+// MODE_DENSE: all v rows of E.
+enum { MODE_FUSED = 0, MODE_SEL = 1, MODE_DENSE = 2 };
+
+struct RowsSmemLayout {
+  uint32_t bars, hs, ring, selsm, sel, tok, total;
+};
+
+__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline RowsSmemLayout rows_layout(uint32_t row_bytes, int K, int p,
+                                                      int rows_max, int mode) {
+  RowsSmemLayout L;
+  L.bars = 0;
+  L.hs = 1024;
+  L.ring = align_up(L.hs + row_bytes, 128);
+  L.selsm = align_up(L.ring + (uint32_t)kWarps * K * row_bytes, 128);
+  L.sel = align_up(L.selsm + (mode == MODE_FUSED ? (uint32_t)sizeof(SelectSmem<kThreads>) : 0u), 16);
+  L.tok = align_up(L.sel + (mode == MODE_DENSE ? 0u : (uint32_t)p * 4u), 16);
+  L.total = align_up(L.tok + (mode == MODE_DENSE ? 0u : (uint32_t)rows_max * 4u), 128);
+  return L;
+}
+
+template <int ELEM, int MODE, int KPT>
+__global__ void __launch_bounds__(kThreads) k_rows(const Stage2Params prm, int K, int rows_max) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = blockIdx.y;
+  const uint32_t row_bytes = (uint32_t)(prm.d * (ELEM == kBF16 ? 2 : 4));
+  const int nch = (int)(row_bytes / 16);
+  const RowsSmemLayout L = rows_layout(row_bytes, K, prm.p, rows_max, MODE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint8_t* hs = smem + L.hs;
+  uint8_t* ring = smem + L.ring;
+  int* sel_s = reinterpret_cast<int*>(smem + L.sel);
+  int32_t* tok_s = reinterpret_cast<int32_t*>(smem + L.tok);
+  __shared__ unsigned long long warp_best[kWarps];
+  __shared__ bool is_last;
+
+  // ---- prologue (independent of the previous kernel)
+  if (tid < kWarps * K) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
+  block_copy_g2s(hs, static_cast<const uint8_t*>(prm.H) + (size_t)q * row_bytes, row_bytes);
+  pdl_wait_prior();
+
+  // ---- probe set S of this query
+  const int64_t b = prm.b;
+  if (MODE == MODE_FUSED) {
+    SelectSmem<kThreads>& ssm = *reinterpret_cast<SelectSmem<kThreads>*>(smem + L.selsm);
+    const float* krow = prm.keys + (size_t)q * prm.c;
+    float x[KPT];
+    const int base = tid * KPT;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) x[j] = (base + j < prm.c) ? krow[base + j] : 0.0f;
+    block_select_topp<kThreads, KPT>(x, (int)prm.c, prm.p, ssm, sel_s);
+    if (prm.dbg_sel && blockIdx.x == 0)
+      for (int r = tid; r < prm.p; r += kThreads) prm.dbg_sel[(size_t)q * prm.p + r] = sel_s[r];
+  } else if (MODE == MODE_SEL) {
+    for (int r = tid; r < prm.p; r += kThreads) sel_s[r] = prm.sel[(size_t)q * prm.p + r];
+  }
+  __syncthreads();
+
+  const int64_t rows = (MODE == MODE_DENSE) ? prm.v : (int64_t)prm.p * b;
+  const int64_t lo = rows * blockIdx.x / gridDim.x;
+  const int64_t hi = rows * (blockIdx.x + 1) / gridDim.x;
+  const uint8_t* E = static_cast<const uint8_t*>(prm.E);
+  const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
+  const bool perm = (MODE != MODE_DENSE) && Ep != nullptr;
+
+  // token ids of this block's rows (candidates only)
+  auto load_toks = [&]() {
+    for (int64_t i = lo + tid; i < hi; i += kThreads)
+      tok_s[i - lo] = prm.C2T[(int64_t)sel_s[i / b] * b + i % b];
+  };
+  auto src = [&](int64_t i) -> const uint8_t* {
+    if (MODE == MODE_DENSE) return E + (size_t)i * row_bytes;
+    if (perm) return Ep + (size_t)((int64_t)sel_s[i / b] * b + i % b) * row_bytes;
+    return E + (size_t)tok_s[i - lo] * row_bytes;
+  };
+  // The first K rows of each warp are issued before the token ids are known when the cluster-major
+  // copy gives their addresses directly.
+  const int64_t first = lo + warp;
+  int64_t nw = (first < hi) ? (hi - first + kWarps - 1) / kWarps : 0;
+  if (MODE != MODE_DENSE) {
+    if (perm && lane == 0)
+      for (int n = 0; n < K && n < nw; ++n) {
+        mbar_arrive_expect_tx(&bars[warp * K + n], row_bytes);
+        bulk_g2s(ring + ((size_t)warp * K + n) * row_bytes, src(first + (int64_t)kWarps * n),
+                 row_bytes, &bars[warp * K + n]);
+      }
+    load_toks();
+    __syncthreads();
+    if (!perm && lane == 0)
+      for (int n = 0; n < K && n < nw; ++n) {
+        mbar_arrive_expect_tx(&bars[warp * K + n], row_bytes);
+        bulk_g2s(ring + ((size_t)warp * K + n) * row_bytes, src(first + (int64_t)kWarps * n),
+                 row_bytes, &bars[warp * K + n]);
+      }
+  } else if (lane == 0) {
+    for (int n = 0; n < K && n < nw; ++n) {
+      mbar_arrive_expect_tx(&bars[warp * K + n], row_bytes);
+      bulk_g2s(ring + ((size_t)warp * K + n) * row_bytes, src(first + (int64_t)kWarps * n),
+               row_bytes, &bars[warp * K + n]);
+    }
+  }
+
+  // ---- stream the rows: dot, decision key, running arg-max
+  const uint32_t hs_addr = smem_addr(hs);
+  const int64_t P = (MODE == MODE_DENSE) ? prm.v : (int64_t)prm.p * b;
+  unsigned long long best = 0ull;
+  uint8_t* ring_w = ring + (size_t)warp * K * row_bytes;
+  uint64_t* bars_w = bars + warp * K;
+  for (int64_t n = 0; n < nw; ++n) {
+    const int slot = (int)(n % K);
+    if (!mbar_wait(&bars_w[slot], (uint32_t)((n / K) & 1), prm.status)) {
+      for (int64_t m = n + 1; m < nw && m < n + K; ++m)
+        mbar_wait(&bars_w[m % K], (uint32_t)((m / K) & 1), nullptr, 50000000ull);
+      nw = n;
+      break;
+    }
+    const int64_t i = first + (int64_t)kWarps * n;
+    const float z =
+        warp_sum(row_dot_partial<ELEM>(smem_addr(ring_w + (size_t)slot * row_bytes), hs_addr, nch, lane));
+    __syncwarp();
+    if (lane == 0) {
+      if (n + K < nw) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bars_w[slot], row_bytes);
+        bulk_g2s(ring_w + (size_t)slot * row_bytes, src(first + (int64_t)kWarps * (n + K)), row_bytes,
+                 &bars_w[slot]);
+      }
+      const uint32_t tok = (MODE == MODE_DENSE) ? (uint32_t)i : (uint32_t)tok_s[i - lo];
+      float val = z;
+      if (prm.sample)
+        val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, 1u, tok));
+      const unsigned long long pk = pack_best(val, tok);
+      best = pk > best ? pk : best;
+      if (prm.dbg_logit) prm.dbg_logit[(size_t)q * P + i] = z;
+      if (prm.dbg_tok) prm.dbg_tok[(size_t)q * P + i] = (int32_t)tok;
+    }
+  }
+
+  // ---- block arg-max, then the last block of this query reduces all partial results
+  if (lane == 0) warp_best[warp] = best;
+  __syncthreads();
+  if (tid == 0) {
+    unsigned long long bb = 0ull;
+    for (int w = 0; w < kWarps; ++w) bb = warp_best[w] > bb ? warp_best[w] : bb;
+    prm.part[(size_t)q * gridDim.x + blockIdx.x] = bb;
+    __threadfence();
+    const uint32_t t = atomicAdd(&prm.tickets[q], 1u);
+    is_last = (t == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (is_last) {
+    __threadfence();
+    unsigned long long bb = 0ull;
+    for (uint32_t g = lane; g < gridDim.x; g += 32) {
+      const unsigned long long v = __ldcg(&prm.part[(size_t)q * gridDim.x + g]);
+      bb = v > bb ? v : bb;
+    }
+    if (warp == 0) {
+      bb = warp_max_u64(bb);
+      if (lane == 0) {
+        if (prm.out_tok) prm.out_tok[q] = (int32_t)best_id(bb);
+        prm.tickets[q] = 0u;
+      }
+    }
+  }
+}
+
+// Dense head: the same kernel over all rows; logits optionally written out.
+template <int ELEM>
+__global__ void __launch_bounds__(kThreads) k_dense(const DenseParams prm, int K) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q = blockIdx.y;
+  const uint32_t row_bytes = (uint32_t)(prm.d * (ELEM == kBF16 ? 2 : 4));
+  const int nch = (int)(row_bytes / 16);
+  const RowsSmemLayout L = rows_layout(row_bytes, K, 0, 0, MODE_DENSE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint8_t* hs = smem + L.hs;
+  uint8_t* ring = smem + L.ring;
+  __shared__ unsigned long long warp_best[kWarps];
+  __shared__ bool is_last;
+  if (tid < kWarps * K) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
+  block_copy_g2s(hs, static_cast<const uint8_t*>(prm.H) + (size_t)q * row_bytes, row_bytes);
+  __syncthreads();
+
+  const int64_t lo = prm.v * blockIdx.x / gridDim.x;
+  const int64_t hi = prm.v * (blockIdx.x + 1) / gridDim.x;
+  const uint8_t* E = static_cast<const uint8_t*>(prm.E);
+  const uint32_t hs_addr = smem_addr(hs);
+  unsigned long long best = 0ull;
+  auto src = [&](int64_t t) { return E + (size_t)t * row_bytes; };
+  auto body = [&](int64_t t, uint32_t row_s) {
+    const float z = warp_sum(row_dot_partial<ELEM>(row_s, hs_addr, nch, lane));
+    if (lane == 0) {
+      float val = z;
+      if (prm.sample)
+        val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, 1u, (uint32_t)t));
+      const unsigned long long pk = pack_best(val, (uint32_t)t);
+      best = pk > best ? pk : best;
+      if (prm.out_logits) prm.out_logits[(size_t)q * prm.v + t] = z;
+    }
+  };
+  warp_stream_rows(lo + warp, hi, kWarps, lane, ring + (size_t)warp * K * row_bytes, bars + warp * K,
+                   K, row_bytes, src, body, prm.status);
+
+  if (lane == 0) warp_best[warp] = best;
+  __syncthreads();
+  if (tid == 0) {
+    unsigned long long bb = 0ull;
+    for (int w = 0; w < kWarps; ++w) bb = warp_best[w] > bb ? warp_best[w] : bb;
+    prm.part[(size_t)q * gridDim.x + blockIdx.x] = bb;
+    __threadfence();
+    const uint32_t t = atomicAdd(&prm.tickets[q], 1u);
+    is_last = (t == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (is_last && warp == 0) {
+    __threadfence();
+    unsigned long long bb = 0ull;
+    for (uint32_t g = lane; g < gridDim.x; g += 32) {
+      const unsigned long long v = __ldcg(&prm.part[(size_t)q * gridDim.x + g]);
+      bb = v > bb ? v : bb;
+    }
+    bb = warp_max_u64(bb);
+    if (lane == 0) {
+      if (prm.out_tok) prm.out_tok[q] = (int32_t)best_id(bb);
+      prm.tickets[q] = 0u;
+    }
+  }
+}
+
+// ============================================================================ index load
+
+__global__ void k_validate_c2t(const int32_t* C2T, int64_t v, uint32_t* bitmap, uint32_t* status) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < v;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t t = C2T[i];
+    if (t < 0 || (int64_t)t >= v) {
+      set_status(status, kStatusIndex);
+      continue;
+    }
+    const uint32_t bit = 1u << (t & 31);
+    const uint32_t old = atomicOr(&bitmap[t >> 5], bit);
+    if (old & bit) set_status(status, kStatusIndex);
+  }
+}
+
+__global__ void k_build_perm(const uint8_t* E, const int32_t* C2T, int64_t v, int64_t row_bytes,
+                             uint8_t* E_perm) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t r = warp; r < v; r += nwarps) {
+    const uint4* s = reinterpret_cast<const uint4*>(E + (size_t)C2T[r] * row_bytes);
+    uint4* d = reinterpret_cast<uint4*>(E_perm + (size_t)r * row_bytes);
+    for (int64_t ch = lane; ch < row_bytes / 16; ch += 32) d[ch] = s[ch];
+  }
+}
+
+// ============================================================================ Monte Carlo
+// FlashHead notes, Module 4 and Eq. 7.  The candidates of a draw are whole clusters, so the softmax
+// denominator over cand(S_i) equals Σ_{k∈S_i} Z_k with Z_k = Σ_{u∈cluster k} exp(z_u/τ - zmax):
+// the S-independent part is computed once per query and each draw only selects and sums.
+
+__global__ void k_mc_cluster_of(const int32_t* C2T, int64_t v, int64_t b, int32_t* cluster_of) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < v;
+       i += (int64_t)gridDim.x * blockDim.x)
+    cluster_of[C2T[i]] = (int32_t)(i / b);
+}
+
+__global__ void k_mc_zmax(const float* z, int64_t v, float tau, float* zmax) {
+  __shared__ float red[32];
+  const int q = blockIdx.x;
+  float m = -INFINITY;
+  for (int64_t t = threadIdx.x; t < v; t += blockDim.x) m = fmaxf(m, z[(size_t)q * v + t] / tau);
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = (threadIdx.x < blockDim.x / 32) ? red[threadIdx.x] : -INFINITY;
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, off));
+    if (threadIdx.x == 0) zmax[q] = m;
+  }
+}
+
+__global__ void k_mc_partition(const float* z, const int32_t* C2T, int64_t v, int64_t c, int64_t b,
+                               float tau, const float* zmax, double* Z, int B) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)B * c;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t q = i / c, k = i % c;
+    const double m = (double)zmax[q];
+    double acc = 0.0;
+    for (int64_t j = 0; j < b; ++j)
+      acc += exp((double)z[(size_t)q * v + C2T[k * b + j]] / (double)tau - m);
+    Z[i] = acc;
+  }
+}
+
+constexpr int kMcThreads = 256;
+
+template <int KPT>
+__global__ void __launch_bounds__(kMcThreads) k_mc_draws(const McParams prm) {
+  __shared__ SelectSmem<kMcThreads> sm;
+  __shared__ double red[kMcThreads / 32];
+  __shared__ double denom_s;
+  __shared__ int32_t tcl[64];     // cluster of each target
+  __shared__ double tnum[64];     // exp(z_t/τ - zmax)
+  __shared__ uint8_t tsel[64];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int q = blockIdx.y;
+  const int64_t c = prm.c;
+  const int base = tid * KPT;
+  const double m = (double)prm.zmax[q];
+  for (int j = tid; j < prm.T; j += kMcThreads) {
+    const int32_t t = prm.targets[(size_t)q * prm.T + j];
+    if (t < 0 || (int64_t)t >= prm.v) {  // out-of-range target: reported, probability 0
+      set_status(prm.status, kStatusIndex);
+      tcl[j] = -1;
+      tnum[j] = 0.0;
+      continue;
+    }
+    tcl[j] = prm.cluster_of[t];
+    tnum[j] = exp((double)prm.z[(size_t)q * prm.v + t] / (double)prm.tau - m);
+  }
+  float sdiv[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j)
+    sdiv[j] = (base + j < c) ? prm.s[(size_t)q * c + base + j] / prm.tau : 0.0f;
+  __syncthreads();
+
+  const int64_t lo = prm.N * blockIdx.x / gridDim.x;
+  const int64_t hi = prm.N * (blockIdx.x + 1) / gridDim.x;
+  for (int64_t i = lo; i < hi; ++i) {
+    float x[KPT];
+#pragma unroll
+    for (int g = 0; g < KPT / 4; ++g) {
+      const uint4 w = philox_block(prm.seed, (uint64_t)i, (uint32_t)q, 2u, (uint32_t)((base >> 2) + g));
+      x[4 * g + 0] = sdiv[4 * g + 0] + gumbel_from_u32(w.x);
+      x[4 * g + 1] = sdiv[4 * g + 1] + gumbel_from_u32(w.y);
+      x[4 * g + 2] = sdiv[4 * g + 2] + gumbel_from_u32(w.z);
+      x[4 * g + 3] = sdiv[4 * g + 3] + gumbel_from_u32(w.w);
+    }
+    const uint64_t mine = block_select_topp<kMcThreads, KPT>(x, (int)c, prm.p, sm, nullptr);
+    double acc = 0.0;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j)
+      if (mine >> j & 1ull) acc += prm.Z[(size_t)q * c + base + j];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+    if (lane == 0) red[wid] = acc;
+    for (int j = 0; j < prm.T; ++j) {
+      const int k = tcl[j];
+      if (k >= base && k < base + KPT) tsel[j] = (mine >> (k - base)) & 1ull ? 1 : 0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double dsum = 0.0;
+      for (int w = 0; w < kMcThreads / 32; ++w) dsum += red[w];
+      denom_s = dsum;
+    }
+    __syncthreads();
+    for (int j = tid; j < prm.T; j += kMcThreads)
+      prm.per_draw[((size_t)q * prm.N + i) * prm.T + j] = tsel[j] ? tnum[j] / denom_s : 0.0;
+    __syncthreads();
+  }
+}
+
+__global__ void k_mc_reduce(const double* per_draw, int64_t N, int T, int B, double* mean,
+                            double* se) {
+  const int lane = threadIdx.x & 31;
+  const int w = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  if (w >= B * T) return;
+  const int q = w / T, j = w % T;
+  double s = 0.0;
+  for (int64_t i = lane; i < N; i += 32) s += per_draw[((size_t)q * N + i) * T + j];
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
+  const double mu = s / (double)N;
+  double ss = 0.0;
+  for (int64_t i = lane; i < N; i += 32) {
+    const double dl = per_draw[((size_t)q * N + i) * T + j] - mu;
+    ss += dl * dl;
+  }
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+  if (lane == 0) {
+    mean[w] = mu;
+    se[w] = (N > 1) ? sqrt(ss / (double)(N - 1)) / sqrt((double)N) : 0.0;
+  }
+}
+
+// ============================================================================ launchers
+
+static int ring_slots(uint32_t row_bytes, uint32_t budget) {
+  int k = (int)(budget / ((uint32_t)kWarps * row_bytes));
+  return k < 1 ? 1 : (k > 8 ? 8 : k);
+}
+
+template <typename Kern>
+static cudaError_t set_smem(Kern kern, size_t bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_sms,
+                          cudaStream_t st, bool pdl_primary) {
+  (void)pdl_primary;
+  if (int4) {
+    const uint32_t row_bytes = (uint32_t)(prm.d / 2);
+    const int K = ring_slots(row_bytes, 32 * 1024);
+    const int G = num_sms;
+    const int rows_max = (int)((prm.c + G - 1) / G);
+    const int nch = (int)(prm.d / 32);
+    const size_t smem = 1024 + (((size_t)rows_max * nch * 2 + 127) / 128) * 128 +
+                        (size_t)kWarps * K * row_bytes;
+    dim3 grid(G, prm.B);
+    cudaError_t e;
+    if (nch <= 32) {
+      if ((e = set_smem(k_stage1_int4<1>, smem)) != cudaSuccess) return e;
+      k_stage1_int4<1><<<grid, kThreads, smem, st>>>(prm, K, rows_max);
+    } else if (nch <= 64) {
+      if ((e = set_smem(k_stage1_int4<2>, smem)) != cudaSuccess) return e;
+      k_stage1_int4<2><<<grid, kThreads, smem, st>>>(prm, K, rows_max);
+    } else {
+      if ((e = set_smem(k_stage1_int4<4>, smem)) != cudaSuccess) return e;
+      k_stage1_int4<4><<<grid, kThreads, smem, st>>>(prm, K, rows_max);
+    }
+    return cudaGetLastError();
+  }
+  const uint32_t row_bytes = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
+  const int K = ring_slots(row_bytes, 64 * 1024);
+  const int QB = prm.B == 1 ? 1 : 4;
+  const size_t smem = 1024 + (size_t)QB * row_bytes + (size_t)kWarps * K * row_bytes;
+  dim3 grid(num_sms, (prm.B + QB - 1) / QB);
+  cudaError_t e;
+#define FH_S1(EL, Q)                                                          \
+  do {                                                                        \
+    if ((e = set_smem(k_stage1<EL, Q>, smem)) != cudaSuccess) return e;       \
+    k_stage1<EL, Q><<<grid, kThreads, smem, st>>>(prm, K);                    \
+  } while (0)
+  if (elem == kBF16) {
+    if (QB == 1) FH_S1(kBF16, 1); else FH_S1(kBF16, 4);
+  } else {
+    if (QB == 1) FH_S1(kF32, 1); else FH_S1(kF32, 4);
+  }
+#undef FH_S1
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gumbel_keys(const float* s, float* keys, int B, int64_t c, float tau,
+                               uint64_t seed, uint64_t step, uint32_t rng_stream, cudaStream_t st) {
+  const int64_t n = (int64_t)B * c;
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  k_gumbel_keys<<<blocks, 256, 0, st>>>(s, keys, B, c, tau, seed, step, rng_stream);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p, cudaStream_t st) {
+  const int64_t kpt = (c + kSelThreads - 1) / kSelThreads;
+#define FH_SEL(KP) k_select<KP><<<B, kSelThreads, 0, st>>>(keys, sel, c, p)
+  if (kpt <= 4) FH_SEL(4);
+  else if (kpt <= 8) FH_SEL(8);
+  else if (kpt <= 16) FH_SEL(16);
+  else if (kpt <= 32) FH_SEL(32);
+  else FH_SEL(64);
+#undef FH_SEL
+  return cudaGetLastError();
+}
+
+int stage2_blocks(int64_t rows, int B, int num_sms) {
+  int64_t g = (B == 1) ? num_sms : (2 * (int64_t)num_sms + B - 1) / B;
+  const int64_t max_g = (rows + 7) / 8;  // at least ~8 rows per block
+  if (g > max_g) g = max_g;
+  return (int)(g < 1 ? 1 : g);
+}
+
+cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st,
+                          bool pdl_secondary) {
+  const uint32_t row_bytes = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
+  const int K = ring_slots(row_bytes, 128 * 1024);
+  const int64_t P = (int64_t)prm.p * prm.b;
+  const int G = stage2_blocks(P, prm.B, num_sms);
+  const int rows_max = (int)((P + G - 1) / G);
+  const int mode = prm.keys ? MODE_FUSED : MODE_SEL;
+  const RowsSmemLayout L = rows_layout(row_bytes, K, prm.p, rows_max, mode);
+  const size_t smem = L.total;
+  const int64_t kpt = (prm.c + kThreads - 1) / kThreads;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G, prm.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_secondary ? 1 : 0;
+  cudaError_t e;
+#define FH_ROWS(EL, MO, KP)                                                        \
+  do {                                                                             \
+    if ((e = set_smem(k_rows<EL, MO, KP>, smem)) != cudaSuccess) return e;         \
+    e = cudaLaunchKernelEx(&cfg, k_rows<EL, MO, KP>, prm, K, rows_max);            \
+  } while (0)
+#define FH_ROWS_E(EL)                                     \
+  do {                                                    \
+    if (mode == MODE_SEL) FH_ROWS(EL, MODE_SEL, 1);       \
+    else if (kpt <= 8) FH_ROWS(EL, MODE_FUSED, 8);        \
+    else if (kpt <= 16) FH_ROWS(EL, MODE_FUSED, 16);      \
+    else if (kpt <= 32) FH_ROWS(EL, MODE_FUSED, 32);      \
+    else FH_ROWS(EL, MODE_FUSED, 64);                     \
+  } while (0)
+  if (elem == kBF16) FH_ROWS_E(kBF16); else FH_ROWS_E(kF32);
+#undef FH_ROWS_E
+#undef FH_ROWS
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dense(const DenseParams& prm, int elem, int num_sms, cudaStream_t st) {
+  const uint32_t row_bytes = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
+  const int K = ring_slots(row_bytes, 128 * 1024);
+  const int G = stage2_blocks(prm.v, prm.B, num_sms);
+  const RowsSmemLayout L = rows_layout(row_bytes, K, 0, 0, MODE_DENSE);
+  const size_t smem = L.total;
+  cudaError_t e;
+  if (elem == kBF16) {
+    if ((e = set_smem(k_dense<kBF16>, smem)) != cudaSuccess) return e;
+    k_dense<kBF16><<<dim3(G, prm.B), kThreads, smem, st>>>(prm, K);
+  } else {
+    if ((e = set_smem(k_dense<kF32>, smem)) != cudaSuccess) return e;
+    k_dense<kF32><<<dim3(G, prm.B), kThreads, smem, st>>>(prm, K);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const int32_t* C2T, int64_t b, const int32_t* sel, int B, int p,
+                          int32_t* cand, cudaStream_t st) {
+  const int64_t n = (int64_t)B * p * b;
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  k_gather<<<blocks, 256, 0, st>>>(C2T, b, sel, B, p, cand);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cand_logits(const void* E, int elem, int64_t d, const void* H, int B,
+                               const int32_t* cand, int64_t P, float* out_z, cudaStream_t st) {
+  const int64_t warps = (int64_t)B * P;
+  const int blocks = (int)((warps * 32 + 255) / 256 < 8192 ? (warps * 32 + 255) / 256 : 8192);
+  if (elem == kBF16) k_cand_logits<kBF16><<<blocks, 256, 0, st>>>(E, d, H, B, cand, P, out_z);
+  else k_cand_logits<kF32><<<blocks, 256, 0, st>>>(E, d, H, B, cand, P, out_z);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_philox(uint64_t seed, uint64_t step, uint32_t row, uint32_t rng_stream, int64_t n,
+                          uint32_t* out, cudaStream_t st) {
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  k_philox<<<blocks, 256, 0, st>>>(seed, step, row, rng_stream, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_validate_c2t(const int32_t* C2T, int64_t v, uint32_t* bitmap, uint32_t* status,
+                                cudaStream_t st) {
+  const int blocks = (int)((v + 255) / 256 < 4096 ? (v + 255) / 256 : 4096);
+  k_validate_c2t<<<blocks, 256, 0, st>>>(C2T, v, bitmap, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_perm(const void* E, const int32_t* C2T, int64_t v, int64_t d, int elem,
+                              void* E_perm, cudaStream_t st) {
+  const int64_t row_bytes = d * (elem == kBF16 ? 2 : 4);
+  k_build_perm<<<1184, 256, 0, st>>>(static_cast<const uint8_t*>(E), C2T, v, row_bytes,
+                                     static_cast<uint8_t*>(E_perm));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mc(const McParams& prm, int num_sms, cudaStream_t st) {
+  cudaError_t e;
+  k_mc_cluster_of<<<1024, 256, 0, st>>>(prm.C2T, prm.v, prm.b, const_cast<int32_t*>(prm.cluster_of));
+  k_mc_zmax<<<prm.B, 1024, 0, st>>>(prm.z, prm.v, prm.tau, prm.zmax);
+  k_mc_partition<<<1024, 256, 0, st>>>(prm.z, prm.C2T, prm.v, prm.c, prm.b, prm.tau, prm.zmax, prm.Z,
+                                       prm.B);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t kpt = (prm.c + kMcThreads - 1) / kMcThreads;
+  int64_t gd = (4 * (int64_t)num_sms + prm.B - 1) / prm.B;
+  if (gd > prm.N) gd = prm.N;
+  dim3 grid((unsigned)gd, prm.B);
+#define FH_MC(KP) k_mc_draws<KP><<<grid, kMcThreads, 0, st>>>(prm)
+  if (kpt <= 4) FH_MC(4);
+  else if (kpt <= 8) FH_MC(8);
+  else if (kpt <= 16) FH_MC(16);
+  else if (kpt <= 32) FH_MC(32);
+  else if (kpt <= 40) FH_MC(40);
+  else FH_MC(64);
+#undef FH_MC
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int warps = prm.B * prm.T;
+  k_mc_reduce<<<(warps * 32 + 255) / 256, 256, 0, st>>>(prm.per_draw, prm.N, prm.T, prm.B,
+                                                       prm.out_mean, prm.out_se);
+  return cudaGetLastError();
+}
+
+}  // namespace fh

@@ -1,0 +1,114 @@
+// fh_kernels.cuh — launch parameters of the FlashHead kernels and their host-side launchers.
+// The launchers are defined in fh_kernels.cu; the C ABI in fh_api.cu validates arguments, lays out
+// the caller's workspace and calls them.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fh {
+
+enum ElemKind : int { kF32 = 0, kBF16 = 1 };
+
+// Stage 1: s[q][k] = C[k]·h_q (or the Gumbel key s/τ + G when sample != 0).
+struct Stage1Params {
+  const void* C;               // c x d (dense) — or null for INT4
+  const uint8_t* q4;           // c x d/2 (INT4)
+  const uint16_t* scales;      // c x d/32 (INT4)
+  const void* H;               // B x d
+  float* out;                  // B x c
+  int64_t c, d;
+  int B;
+  int sample;
+  float tau;
+  uint64_t seed, step;
+  uint32_t rng_stream;
+  uint32_t* status;
+  uint32_t* tickets_to_clear;  // reset to 0 by block (0,0) for the kernels that follow
+  int n_tickets;
+};
+
+// Stage 2 over the candidates of each query, with the token decision fused in.
+struct Stage2Params {
+  const void* E;               // v x d (row source when E_perm is null)
+  const void* E_perm;          // v x d cluster-major copy, or null
+  const int32_t* C2T;          // c x b
+  const void* H;               // B x d
+  const float* keys;           // B x c Stage-1 keys (fused selection) — or null
+  const int32_t* sel;          // B x p probe sets (when keys is null)
+  int64_t v, d, c, b;
+  int B, p;
+  int sample;
+  float tau;
+  uint64_t seed, step;
+  unsigned long long* part;    // gridDim.x x B partial arg-maxima
+  uint32_t* tickets;           // B counters
+  int32_t* out_tok;            // B
+  int32_t* dbg_sel;            // B x p or null
+  int32_t* dbg_tok;            // B x P or null
+  float* dbg_logit;            // B x P or null
+  uint32_t* status;
+};
+
+// Dense head over all v rows of E for each query.
+struct DenseParams {
+  const void* E;
+  const void* H;
+  int64_t v, d;
+  int B;
+  int sample;
+  float tau;
+  uint64_t seed, step;
+  unsigned long long* part;    // gridDim.x x B
+  uint32_t* tickets;           // B
+  int32_t* out_tok;            // B (may be null)
+  float* out_logits;           // B x v or null
+  uint32_t* status;
+};
+
+// Monte Carlo marginal (per query: N draws of Gumbel-top-p over the Stage-1 scores).
+struct McParams {
+  const float* s;              // B x c Stage-1 scores
+  const float* z;              // B x v logits
+  const int32_t* C2T;          // c x b
+  const int32_t* cluster_of;   // v: token → cluster
+  const int32_t* targets;      // B x T
+  float* zmax;                 // B: max_t z_t/τ
+  double* Z;                   // B x c: Σ_{u in cluster} exp(z_u/τ - zmax)
+  double* per_draw;            // B x N x T
+  double* out_mean;            // B x T
+  double* out_se;              // B x T
+  int64_t v, c, b, N;
+  int B, T, p;
+  float tau;
+  uint64_t seed;
+  uint32_t* status;
+};
+
+// ---- launchers (return cudaGetLastError() of the launch) ----
+cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_sms,
+                          cudaStream_t st, bool pdl_primary);
+cudaError_t launch_gumbel_keys(const float* s, float* keys, int B, int64_t c, float tau,
+                               uint64_t seed, uint64_t step, uint32_t rng_stream,
+                               cudaStream_t st);
+cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p,
+                          cudaStream_t st);
+cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st,
+                          bool pdl_secondary);
+cudaError_t launch_dense(const DenseParams& prm, int elem, int num_sms, cudaStream_t st);
+cudaError_t launch_gather(const int32_t* C2T, int64_t b, const int32_t* sel, int B, int p,
+                          int32_t* cand, cudaStream_t st);
+cudaError_t launch_cand_logits(const void* E, int elem, int64_t d, const void* H, int B,
+                               const int32_t* cand, int64_t P, float* out_z, cudaStream_t st);
+cudaError_t launch_philox(uint64_t seed, uint64_t step, uint32_t row, uint32_t rng_stream,
+                          int64_t n, uint32_t* out, cudaStream_t st);
+cudaError_t launch_validate_c2t(const int32_t* C2T, int64_t v, uint32_t* bitmap,
+                                uint32_t* status, cudaStream_t st);
+cudaError_t launch_build_perm(const void* E, const int32_t* C2T, int64_t v, int64_t d, int elem,
+                              void* E_perm, cudaStream_t st);
+cudaError_t launch_mc(const McParams& prm, int num_sms, cudaStream_t st);
+
+// Number of Stage-2 blocks used per query for `rows` candidate rows.
+int stage2_blocks(int64_t rows, int B, int num_sms);
+
+}  // namespace fh

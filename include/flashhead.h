@@ -43,9 +43,10 @@
  *     numbers: as easy as 1, 2, 3", SC'11) with key = (seed low 32 bits, seed high 32 bits) and
  *     counter = (elem >> 2, row, step low 32 bits, (stream << 24) | (step high 32 bits & 0xFFFFFF)),
  *     taking output word (elem & 3).  A draw x becomes u = ((x >> 9) + 0.5)·2^-23 ∈ (0,1), which is
- *     exact in fp32, and the Gumbel variate G = -log(-log u).  Streams: FH_RNG_STAGE1 (Stage-1 keys, elem = cluster id),
- *     FH_RNG_STAGE2 (Stage-2 and dense-head keys, elem = token id), FH_RNG_MC (Monte Carlo draws,
- *     elem = cluster id, step = draw index).  row = the query's index within the batch.
+ *     exact in fp32, and the Gumbel variate G = -log(-log u).  Streams: FH_RNG_STAGE1 (Stage-1
+ *     keys, elem = cluster id), FH_RNG_STAGE2 (Stage-2 and dense-head keys, elem = token id),
+ *     FH_RNG_MC (Monte Carlo draws, elem = cluster id, step = draw index).  row = the query's
+ *     index within the batch.
  */
 #ifndef FLASHHEAD_H
 #define FLASHHEAD_H
@@ -82,7 +83,7 @@ typedef enum { FH_OP_GREEDY = 0, FH_OP_SAMPLE = 1, FH_OP_MC = 2, FH_OP_DENSE = 3
 enum { FH_RNG_STAGE1 = 0, FH_RNG_STAGE2 = 1, FH_RNG_MC = 2 };
 
 /* Limits of this build. */
-enum { FH_MAX_BATCH = 64, FH_MAX_C = 65536, FH_MAX_D = 8192 };
+enum { FH_MAX_BATCH = 64, FH_MAX_C = 32768, FH_MAX_D = 8192 };
 
 typedef void* fh_stream;            /* cudaStream_t */
 typedef struct fh_index fh_index;   /* opaque host-side handle */
@@ -107,7 +108,7 @@ typedef struct {
 /* Optional device outputs of one fused head call, for checking the intermediate results.
    Any field may be NULL.  sel: B x p cluster ids of S, ascending.  cand_tok: B x (p*b) token ids
    in slot order (slot r*b + j holds C2T[S[r]][j]).  cand_logit: B x (p*b) fp32 logits z of those
-   tokens (greedy) — for sampling, z/τ + G' of those tokens. */
+   tokens (the raw logits in both greedy and sampling mode). */
 typedef struct {
   int32_t* sel;
   int32_t* cand_tok;

@@ -1,0 +1,357 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle on the same seeded inputs.
+
+Sizes span several blocks per kernel with ragged tails; the full Llama-shaped head is checked on
+sampled queries in the launch configuration the benchmark times (batch 1, fused selection)."""
+
+import numpy as np
+import pytest
+import torch
+
+from clustered_retrieval_classification_b200 import synth
+from parity import LOGIT_TOL, MARGIN, check_sets, check_tokens
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def widen(a, dtype):
+    return synth.stored_to_f64(a, dtype)
+
+
+def dev(a, kind):
+    from clustered_retrieval_classification_b200 import flashhead as F
+    return F.device_array(a, kind, DEV)
+
+
+def load(fh, idx, int4=False, cluster_major=True):
+    return fh.index_from_host(idx.E, idx.C, idx.C2T, idx.cfg.dtype, idx.C_q4, idx.C_scales,
+                              int4=int4, cluster_major=cluster_major)
+
+
+# ----------------------------------------------------------------------------- fixtures
+
+MID = synth.scaled(synth.CONFIGS["llama"], v=32064, c=2004, d=512, p=128, name="llama-mid")
+MID_INT4 = synth.dataclasses.replace(synth.scaled(synth.CONFIGS["gemma"], v=32768, c=2048, d=1152,
+                                                  p=128), name="gemma-mid")
+
+
+@pytest.fixture(scope="module")
+def tiny():
+    cfg = synth.CONFIGS["tiny"]
+    return synth.make_index(cfg), synth.make_queries(cfg, 256)
+
+
+@pytest.fixture(scope="module")
+def mid():
+    return synth.make_index(MID), synth.make_queries(MID, 24)
+
+
+@pytest.fixture(scope="module")
+def mid_int4():
+    return synth.make_index(MID_INT4), synth.make_queries(MID_INT4, 8)
+
+
+# ----------------------------------------------------------------------------- Philox / Gumbel
+
+
+@pytest.mark.parametrize("seed,step,row,stream", [(0, 0, 0, 0), (0xF1A54EAD, 12345, 3, 1),
+                                                  (2 ** 64 - 1, 2 ** 40 + 7, 63, 2)])
+def test_philox_bit_exact(fh, orc, seed, step, row, stream):
+    n = 100_003
+    g = fh.philox_u32(seed, step, row, stream, n).cpu().numpy().view(np.uint32)
+    o = orc.philox_words(seed, step, row, stream, n)
+    assert np.array_equal(g, o)
+
+
+def test_gumbel_keys(fh, orc):
+    rng = np.random.default_rng(1)
+    s = (rng.standard_normal((3, 5000)) * 0.3).astype(np.float32)
+    for tau in (0.8, 1.0):
+        g = fh.gumbel_keys(dev(s, "f32"), tau, seed=99, step=7).cpu().numpy()
+        o = orc.gumbel_keys(s.astype(np.float64), tau, 99, 7, 0)
+        np.testing.assert_allclose(g, o, rtol=2e-6, atol=2e-5)
+
+
+# ----------------------------------------------------------------------------- selection
+
+
+def _select_cases():
+    rng = np.random.default_rng(2)
+    cases = []
+    for c, p in [(1, 1), (7, 3), (64, 8), (100, 100), (2004, 128), (8016, 512), (8016, 1),
+                 (9496, 512), (16384, 1024), (32768, 4000)]:
+        cases.append((f"normal-{c}-{p}", rng.standard_normal((2, c)).astype(np.float32), p))
+    cases.append(("ties", rng.integers(-3, 4, size=(3, 5000)).astype(np.float32), 700))
+    cases.append(("all-equal", np.full((2, 3000), 0.25, np.float32), 1000))
+    z = np.zeros((2, 999), np.float32)
+    z[:, ::2] = -0.0
+    cases.append(("signed-zero", z, 500))
+    big = rng.standard_normal((2, 4000)).astype(np.float32)
+    big[:, 0], big[:, 1] = 3e38, -3e38
+    cases.append(("huge-range", big, 300))
+    dense_bin = np.round(rng.standard_normal((2, 8016)) * 0.001, 6).astype(np.float32)
+    dense_bin[:, :10] = 50.0
+    cases.append(("crowded-bin", dense_bin, 2000))
+    return cases
+
+
+@pytest.mark.parametrize("name,keys,p", _select_cases(), ids=lambda x: x if isinstance(x, str) else "")
+def test_select_bit_exact(fh, orc, name, keys, p):
+    g = fh.select_topp(dev(keys, "f32"), p).cpu().numpy()
+    o, _ = orc.select_topp(keys.astype(np.float64), p)
+    assert np.array_equal(g, o), name
+
+
+# ----------------------------------------------------------------------------- single steps
+
+
+def test_stage1_scores(fh, orc, tiny, mid):
+    for idx, H in (tiny, mid):
+        cfg = idx.cfg
+        I = load(fh, idx)
+        Hq = H[:5]
+        g = fh.stage1_scores(I, dev(Hq, cfg.dtype)).cpu().numpy()
+        o = orc.stage1_scores(idx.C, cfg.dtype, Hq, cfg.c, cfg.d)
+        assert np.abs(g - o).max() <= LOGIT_TOL
+
+
+def test_stage1_scores_int4(fh, orc, mid_int4):
+    idx, H = mid_int4
+    I = load(fh, idx, int4=True)
+    g = fh.stage1_scores(I, dev(H[:3], "bf16")).cpu().numpy()
+    o = orc.stage1_scores(None, "bf16", H[:3], idx.c, idx.d, q4=idx.C_q4, scales=idx.C_scales)
+    assert np.abs(g - o).max() <= LOGIT_TOL
+
+
+def test_gather_and_candidate_logits(fh, orc, mid):
+    idx, H = mid
+    cfg = idx.cfg
+    I = load(fh, idx)
+    rng = np.random.default_rng(5)
+    sel = np.sort(np.stack([rng.choice(cfg.c, cfg.p, replace=False) for _ in range(3)]), axis=1)
+    sel = sel.astype(np.int32)
+    g = fh.gather_candidates(I, dev(sel, "i32")).cpu().numpy()
+    o = orc.gather(idx.C2T, sel)
+    assert np.array_equal(g, o)
+    z = fh.candidate_logits(I, dev(H[:3], cfg.dtype), dev(o, "i32")).cpu().numpy()
+    assert np.abs(z - orc.logits(idx.E, cfg.dtype, H[:3], o)).max() <= LOGIT_TOL
+
+
+# ----------------------------------------------------------------------------- fused head
+
+
+def _run_head(fh, I, Hd, p, sample, tau, seed, step, P, B):
+    dbg = dict(sel=torch.empty((B, p), dtype=torch.int32, device=DEV),
+               cand_tok=torch.empty((B, P), dtype=torch.int32, device=DEV),
+               cand_logit=torch.empty((B, P), dtype=torch.float32, device=DEV))
+    if sample:
+        tok = fh.head_sample(I, Hd, p, tau, seed, step, debug=dbg)
+    else:
+        tok = fh.head_greedy(I, Hd, p, debug=dbg)
+    torch.cuda.synchronize()
+    return tok.cpu().numpy(), {k: v.cpu().numpy() for k, v in dbg.items()}
+
+
+def _check_head(fh, orc, idx, H, p, sample=False, tau=1.0, seed=0, step=0, batch=None,
+                cluster_major=True, int4=False):
+    cfg = idx.cfg
+    I = load(fh, idx, int4=int4, cluster_major=cluster_major)
+    B = batch or H.shape[0]
+    Hq = H[:B]
+    P = p * cfg.b
+    tok, dbg = _run_head(fh, I, dev(Hq, cfg.dtype), p, sample, tau, seed, step, P, B)
+    o = orc.head(idx, Hq, p, sample=sample, tau=tau, seed=seed, step=step, use_int4=int4)
+    s = orc.stage1_scores(idx.C if not int4 else None, cfg.dtype, Hq, cfg.c, cfg.d,
+                          q4=idx.C_q4 if int4 else None, scales=idx.C_scales if int4 else None)
+    keys = orc.gumbel_keys(s, tau, seed, step, 0) if sample else s
+    n_set = check_sets(dbg["sel"], o["sel"], keys, o["set_margin"])
+    same = [set(dbg["sel"][q]) == set(o["sel"][q]) for q in range(B)]
+    for q in range(B):
+        if same[q]:
+            assert np.array_equal(dbg["cand_tok"][q], o["cand"][q])
+            assert np.abs(dbg["cand_logit"][q] - o["z"][q]).max() <= LOGIT_TOL
+
+    def valid(q, t):
+        cand = dbg["cand_tok"][q:q + 1]
+        z = orc.logits(idx.E, cfg.dtype, Hq[q:q + 1], cand)[0]
+        if sample:
+            g = np.array([orc.gumbel(orc.draw_u32(seed, step, q, 1, int(u))) for u in cand[0]])
+            z = z / tau + g
+        return z.max(), z[list(cand[0]).index(t)]
+
+    n_tok = check_tokens(tok, o["tok"], o["tok_margin"], same, valid)
+    return n_set, n_tok
+
+
+def test_greedy_tiny_fp32_batch1(fh, orc, tiny):
+    idx, H = tiny
+    for q in range(0, 64, 3):
+        _check_head(fh, orc, idx, H[q:q + 1], idx.cfg.p)
+
+
+def test_greedy_tiny_batched(fh, orc, tiny):
+    idx, H = tiny
+    _check_head(fh, orc, idx, H[:64], idx.cfg.p)
+    _check_head(fh, orc, idx, H[:5], idx.cfg.p)
+
+
+@pytest.mark.parametrize("cluster_major", [True, False])
+def test_greedy_mid_batch1(fh, orc, mid, cluster_major):
+    idx, H = mid
+    for q in range(6):
+        _check_head(fh, orc, idx, H[q:q + 1], idx.cfg.p, cluster_major=cluster_major)
+
+
+@pytest.mark.parametrize("B", [3, 16])
+def test_greedy_mid_batched(fh, orc, mid, B):
+    idx, H = mid
+    _check_head(fh, orc, idx, H, idx.cfg.p, batch=B)
+
+
+@pytest.mark.parametrize("p", [1, 2004])
+def test_greedy_mid_edge_p(fh, orc, mid, p):
+    idx, H = mid
+    _check_head(fh, orc, idx, H[:1], p)
+    _check_head(fh, orc, idx, H[:2], p)
+
+
+def test_sample_mid(fh, orc, mid):
+    idx, H = mid
+    for step in range(4):
+        _check_head(fh, orc, idx, H[step:step + 1], idx.cfg.p, sample=True, tau=0.8,
+                    seed=synth.SAMPLE_SEED, step=step)
+    _check_head(fh, orc, idx, H[:6], idx.cfg.p, sample=True, tau=0.8, seed=synth.SAMPLE_SEED,
+                step=99)
+
+
+def test_int4_mid(fh, orc, mid_int4):
+    idx, H = mid_int4
+    _check_head(fh, orc, idx, H[:1], idx.cfg.p, int4=True)
+    _check_head(fh, orc, idx, H[:4], idx.cfg.p, int4=True)
+
+
+def test_p_equals_c_matches_dense(fh, mid):
+    """With p = c the candidates are the vocabulary: the greedy head must return the dense argmax and
+    the sampling head the dense sample (same Stage-2 noise keyed by token id)."""
+    idx, H = mid
+    I = load(fh, idx)
+    Hd = dev(H[:4], "bf16")
+    for B in (1, 4):
+        g = fh.head_greedy(I, Hd[:B], idx.c).cpu().numpy()
+        d = fh.dense_head(I, Hd[:B]).cpu().numpy()
+        assert np.array_equal(g, d)
+        gs = fh.head_sample(I, Hd[:B], idx.c, 0.8, 5, 3).cpu().numpy()
+        ds = fh.dense_head(I, Hd[:B], sample=True, tau=0.8, seed=5, step=3).cpu().numpy()
+        assert np.array_equal(gs, ds)
+
+
+# ----------------------------------------------------------------------------- dense head
+
+
+@pytest.mark.parametrize("sample", [False, True])
+def test_dense_head(fh, orc, mid, sample):
+    idx, H = mid
+    cfg = idx.cfg
+    I = load(fh, idx)
+    B = 3
+    logits = torch.empty((B, cfg.v), dtype=torch.float32, device=DEV)
+    tok = fh.dense_head(I, dev(H[:B], "bf16"), sample=sample, tau=0.8, seed=11, step=2,
+                        logits=logits).cpu().numpy()
+    o = orc.dense(idx, H[:B], sample=sample, tau=0.8, seed=11, step=2, want_z=True)
+    assert np.abs(logits.cpu().numpy() - o["z"]).max() <= LOGIT_TOL
+    for q in range(B):
+        if tok[q] != o["tok"][q]:
+            assert o["tok_margin"][q] <= MARGIN
+
+
+# ----------------------------------------------------------------------------- Monte Carlo
+
+
+def test_mc_matches_oracle(fh, orc):
+    cfg = synth.scaled(synth.CONFIGS["qwen"], v=16384, c=1024, d=256, p=64, name="qwen-small")
+    idx = synth.make_index(cfg)
+    H = synth.make_queries(cfg, 3)
+    targets = synth.make_targets(cfg.v, 3, 8)
+    # make some targets likely: include each query's dense argmax
+    z = widen(H, "bf16") @ widen(idx.E, "bf16").T
+    targets[:, 0] = np.argmax(z, axis=1)
+    I = load(fh, idx)
+    N = 2000
+    mean, se = fh.mc_token_prob(I, dev(H, "bf16"), dev(targets, "i32"), cfg.p, 1.0, N, synth.MC_SEED)
+    mean, se = mean.cpu().numpy(), se.cpu().numpy()
+    o = orc.mc(idx, H, targets, cfg.p, 1.0, synth.MC_SEED, n_draws=N)
+    tol = np.maximum(1e-4, 0.1 * o["se"])
+    assert np.all(np.abs(mean - o["mean"]) <= tol), (mean, o["mean"])
+    assert np.all(np.abs(se - o["se"]) <= np.maximum(1e-5, 0.1 * o["se"]))
+
+
+def test_mc_p_equals_c_is_dense_softmax(fh):
+    cfg = synth.scaled(synth.CONFIGS["qwen"], v=4096, c=256, d=128, p=256, name="qwen-pc")
+    idx = synth.make_index(cfg)
+    H = synth.make_queries(cfg, 2)
+    targets = np.array([[0, 1, 2, 3], [4000, 17, 256, 4095]], np.int32)
+    I = load(fh, idx)
+    mean, se = fh.mc_token_prob(I, dev(H, "bf16"), dev(targets, "i32"), cfg.c, 0.7, 50, 1)
+    logits = torch.empty((2, cfg.v), dtype=torch.float32, device=DEV)
+    fh.dense_head(I, dev(H, "bf16"), logits=logits)
+    soft = torch.softmax(logits.double() / 0.7, dim=1).cpu().numpy()
+    np.testing.assert_allclose(mean.cpu().numpy(), np.take_along_axis(soft, targets, 1), rtol=1e-5)
+    assert np.all(se.cpu().numpy() < 1e-9)
+
+
+# ----------------------------------------------------------------------------- robustness
+
+
+def test_determinism(fh, mid):
+    idx, H = mid
+    I = load(fh, idx)
+    Hd = dev(H[:1], "bf16")
+    runs = [fh.head_sample(I, Hd, idx.cfg.p, 0.8, 1, 2).item() for _ in range(3)]
+    assert len(set(runs)) == 1
+    a = [fh.head_greedy(I, dev(H[:8], "bf16"), idx.cfg.p).cpu().numpy() for _ in range(2)]
+    assert np.array_equal(a[0], a[1])
+
+
+def test_bad_c2t_rejected(fh):
+    idx = synth.random_index(v=256, d=64, c=16, seed=3, dtype="bf16")
+    bad = idx.C2T.copy()
+    bad[3, 2] = bad[5, 1]                       # duplicate id
+    with pytest.raises(fh.FlashHeadError) as e:
+        fh.index_from_host(idx.E, idx.C, bad, "bf16")
+    assert e.value.status == 3
+    bad = idx.C2T.copy()
+    bad[0, 0] = 256                             # out of range
+    with pytest.raises(fh.FlashHeadError):
+        fh.index_from_host(idx.E, idx.C, bad, "bf16")
+
+
+def test_workspace_status_clean(fh, mid):
+    idx, H = mid
+    I = load(fh, idx)
+    ws = I.workspace(fh.FH_OP_GREEDY, 1, idx.cfg.p)
+    fh.head_greedy(I, dev(H[:1], "bf16"), idx.cfg.p, ws=ws)
+    fh.ws_status(ws)
+    with pytest.raises(fh.FlashHeadError) as e:
+        fh.head_greedy(I, dev(H[:1], "bf16"), idx.cfg.p, ws=ws[:100])
+    assert e.value.status == 4
+
+
+# ----------------------------------------------------------------------------- full size
+
+
+@pytest.fixture(scope="module")
+def llama():
+    cfg = synth.CONFIGS["llama"]
+    return synth.make_index(cfg), synth.make_queries(cfg, 4)
+
+
+def test_llama_full_size_batch1_sampled(fh, orc, llama):
+    """The Llama-shaped head (v=128256, d=2048, c=8016, p=512) at batch 1 with the fused selection,
+    the configuration the benchmark times; four queries greedy and two sampled."""
+    idx, H = llama
+    for q in range(4):
+        _check_head(fh, orc, idx, H[q:q + 1], idx.cfg.p)
+    for q in range(2):
+        _check_head(fh, orc, idx, H[q:q + 1], idx.cfg.p, sample=True, tau=0.8,
+                    seed=synth.SAMPLE_SEED, step=q)

@@ -40,8 +40,6 @@ size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int elem_bytes(int dtype) { return dtype == FH_BF16 ? 2 : 4; }
-
 // Workspace regions of one call; offsets from the workspace base.
 struct Layout {
   size_t keys = 0, sel = 0, part = 0, z = 0, s = 0, zmax = 0, Z = 0, cluster_of = 0, per_draw = 0;
@@ -89,8 +87,13 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   return FH_OK;
 }
 
+// Workspace header (first kHeaderBytes): status word at 0, per-query tickets at 16 (64 x 4 bytes),
+// the persistent head's grid-barrier counter / generation / ticket at 512, 516, 520 and its packed
+// arg-max at 528.  Counters return to zero at the end of every call; a new workspace must start
+// zeroed (fh_ws_status re-zeroes the header after reporting a device-side error).
 uint32_t* status_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16); }
+uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
 
 fh_status check_batch(const fh_index* idx, const void* H, int B) {
   if (!idx) return fail(FH_ERR_ARG, "index handle is NULL");
@@ -133,7 +136,39 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   float* keys = reinterpret_cast<float*>(base + L.keys);
   int32_t* sel = reinterpret_cast<int32_t*>(base + L.sel);
 
-  const bool fused = (B == 1) && D.c <= 256 * 64;
+  cudaError_t e;
+  if (B == 1 && fh::head1_threads(D.c) != 0) {
+    fh::Head1Params h = {};
+    h.C = D.C;
+    h.q4 = D.C_q4;
+    h.scales = D.C_scales;
+    h.H = H;
+    h.E = D.E;
+    h.E_perm = D.E_perm;
+    h.C2T = D.C2T;
+    h.keys = keys;
+    h.c = D.c;
+    h.d = D.d;
+    h.b = D.b;
+    h.p = p;
+    h.sample = sample;
+    h.tau = tau;
+    h.seed = seed;
+    h.step = step;
+    h.bar_count = word_at(ws, 512);
+    h.bar_gen = word_at(ws, 516);
+    h.ticket = word_at(ws, 520);
+    h.best = reinterpret_cast<unsigned long long*>(word_at(ws, 528));
+    h.out_tok = out_tok;
+    h.dbg_sel = dbg ? dbg->sel : nullptr;
+    h.dbg_tok = dbg ? dbg->cand_tok : nullptr;
+    h.dbg_logit = dbg ? dbg->cand_logit : nullptr;
+    h.status = status_of(ws);
+    e = fh::launch_head1(h, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st);
+    if (e != cudaSuccess) return cuda_fail(e, "persistent head launch");
+    return FH_OK;
+  }
+  const bool fused = false;
   fh::Stage1Params s1 = stage1_params(idx, H, B, keys, ws);
   s1.sample = sample;
   s1.tau = tau;
@@ -142,8 +177,7 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   s1.rng_stream = FH_RNG_STAGE1;
   s1.tickets_to_clear = tickets_of(ws);
   s1.n_tickets = B;
-  cudaError_t e = fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st,
-                                    fused);
+  e = fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st, fused);
   if (e != cudaSuccess) return cuda_fail(e, "stage-1 launch");
   if (!fused) {
     if ((e = fh::launch_select(keys, sel, B, D.c, p, st)) != cudaSuccess)
@@ -158,8 +192,8 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   s2.E_perm = D.E_perm;
   s2.C2T = D.C2T;
   s2.H = H;
-  s2.keys = fused ? keys : nullptr;
-  s2.sel = fused ? nullptr : sel;
+  s2.keys = nullptr;
+  s2.sel = sel;
   s2.v = D.v;
   s2.d = D.d;
   s2.c = D.c;
@@ -173,11 +207,11 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   s2.part = reinterpret_cast<unsigned long long*>(base + L.part);
   s2.tickets = tickets_of(ws);
   s2.out_tok = out_tok;
-  s2.dbg_sel = (dbg && fused) ? dbg->sel : nullptr;
+  s2.dbg_sel = nullptr;
   s2.dbg_tok = dbg ? dbg->cand_tok : nullptr;
   s2.dbg_logit = dbg ? dbg->cand_logit : nullptr;
   s2.status = status_of(ws);
-  if ((e = fh::launch_stage2(s2, D.dtype, idx->num_sms, st, fused)) != cudaSuccess)
+  if ((e = fh::launch_stage2(s2, D.dtype, idx->num_sms, st)) != cudaSuccess)
     return cuda_fail(e, "stage-2 launch");
   return FH_OK;
 }
@@ -271,7 +305,7 @@ fh_status fh_ws_status(void* ws, fh_stream stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   if (status != 0) {
-    e = cudaMemsetAsync(ws, 0, 4, st);
+    e = cudaMemsetAsync(ws, 0, kHeaderBytes, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "status clear");
     if (status == FH_ERR_TIMEOUT) return fail(FH_ERR_TIMEOUT, "a device-side wait timed out");

@@ -18,73 +18,13 @@
 #include "fh_kernels.cuh"
 #include "fh_device.cuh"
 #include "fh_select.cuh"
+#include "fh_stream.cuh"
 
 namespace fh {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSelThreads = 512;
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// Lane-partial dot product of a staged row (shared address row_s) with a staged query vector
-// (shared address h_s); nch = row bytes / 16.
-template <int ELEM>
-__device__ __forceinline__ float row_dot_partial(uint32_t row_s, uint32_t h_s, int nch, int lane) {
-  float acc = 0.0f;
-#pragma unroll 4
-  for (int ch = lane; ch < nch; ch += 32) {
-    const uint4 a = lds_v4(row_s + ch * 16);
-    const uint4 h = lds_v4(h_s + ch * 16);
-    acc = (ELEM == kBF16) ? dot8_bf16(a, h, acc) : dot4_f32(a, h, acc);
-  }
-  return acc;
-}
-
-// Copy `bytes` (multiple of 16) from global to shared memory with 16-byte loads by the whole block.
-__device__ __forceinline__ void block_copy_g2s(void* dst, const void* src, int bytes) {
-  for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(dst)[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
-}
-
-// The per-warp streaming loop.  Rows first, first+W, first+2W, ... below `hi` are brought into the
-// warp's ring (K slots of row_bytes) and handed to body(row, shared address) in order.  src(row)
-// gives the global address of a row.  Returns false if a wait timed out (status already set).
-template <typename Src, typename Body>
-__device__ __forceinline__ bool warp_stream_rows(int64_t first, int64_t hi, int W, int lane,
-                                                 uint8_t* ring, uint64_t* bars, int K,
-                                                 uint32_t row_bytes, const Src& src,
-                                                 const Body& body, uint32_t* status) {
-  if (first >= hi) return true;
-  const int64_t nw = (hi - first + W - 1) / W;
-  if (lane == 0) {
-    for (int n = 0; n < K && n < nw; ++n) {
-      mbar_arrive_expect_tx(&bars[n], row_bytes);
-      bulk_g2s(ring + (size_t)n * row_bytes, src(first + (int64_t)W * n), row_bytes, &bars[n]);
-    }
-  }
-  for (int64_t n = 0; n < nw; ++n) {
-    const int slot = (int)(n % K);
-    const uint32_t parity = (uint32_t)((n / K) & 1);
-    if (!mbar_wait(&bars[slot], parity, status)) {
-      // Give the copies still in flight a bounded chance to land before the block exits.
-      for (int64_t m = n + 1; m < nw && m < n + K; ++m)
-        mbar_wait(&bars[m % K], (uint32_t)((m / K) & 1), nullptr, 50000000ull);
-      return false;
-    }
-    body(first + (int64_t)W * n, smem_addr(ring + (size_t)slot * row_bytes));
-    __syncwarp();
-    if (lane == 0 && n + K < nw) {
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&bars[slot], row_bytes);
-      bulk_g2s(ring + (size_t)slot * row_bytes, src(first + (int64_t)W * (n + K)), row_bytes,
-               &bars[slot]);
-    }
-  }
-  return true;
-}
 
 // ============================================================================ Stage 1 (dense C)
 
@@ -138,24 +78,6 @@ __global__ void __launch_bounds__(kThreads) k_stage1(const Stage1Params prm, int
 // One query per blockIdx.y.  Lane l handles the 16-byte chunks l, l+32, ... of a row (one chunk =
 // one 32-column group), so its slice of h lives in registers as fp32.  A nibble n decodes to
 // q = (n ^ 8) - 8 through the float pattern 0x4B000000 | (n ^ 8) = 2^23 + (n ^ 8), exactly.
-
-__device__ __forceinline__ float int4_group_dot(const uint4 w, const float* hg) {
-  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-  float acc = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t even = (words[i] & 0x0F0F0F0Fu) ^ 0x08080808u;         // columns 8i + 0,2,4,6
-    const uint32_t odd = ((words[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;   // columns 8i + 1,3,5,7
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float qe = __uint_as_float(__byte_perm(even, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
-      const float qo = __uint_as_float(__byte_perm(odd, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
-      acc = fmaf(qe, hg[8 * i + 2 * j], acc);
-      acc = fmaf(qo, hg[8 * i + 2 * j + 1], acc);
-    }
-  }
-  return acc;
-}
 
 template <int MCH>
 __global__ void __launch_bounds__(kThreads) k_stage1_int4(const Stage1Params prm, int K,
@@ -273,52 +195,44 @@ __global__ void k_cand_logits(const void* E, int64_t d, const void* H, int B, co
 
 // ============================================================================ selection kernel
 
-template <int KPT>
-__global__ void __launch_bounds__(kSelThreads) k_select(const float* keys, int32_t* sel, int64_t c,
-                                                        int p) {
-  __shared__ SelectSmem<kSelThreads> sm;
+template <int NT, int KPT>
+__global__ void __launch_bounds__(NT) k_select(const float* keys, int32_t* sel, int64_t c, int p) {
+  __shared__ SelectSmem<NT> sm;
   const int q = blockIdx.x;
-  const float* row = keys + (size_t)q * c;
-  float x[KPT];
-  const int base = threadIdx.x * KPT;
-#pragma unroll
-  for (int j = 0; j < KPT; ++j) x[j] = (base + j < c) ? row[base + j] : 0.0f;
-  block_select_topp<kSelThreads, KPT>(x, (int)c, p, sm, sel + (size_t)q * p);
+  uint32_t key[KPT];
+  load_key_images<KPT>(keys + (size_t)q * c, (int)c, key);
+  block_select_topp<NT, KPT>(key, (int)c, p, sm, sel + (size_t)q * p);
 }
 
-// ============================================================================ rows + arg-max
-// MODE_FUSED: candidates of query blockIdx.y; the block first selects S itself from the Stage-1 keys.
-// MODE_SEL:   candidates of query blockIdx.y from the given probe sets.
-// MODE_DENSE: all v rows of E.
-enum { MODE_FUSED = 0, MODE_SEL = 1, MODE_DENSE = 2 };
+// ============================================================================ Stage 2 (batched)
+// Candidates of query blockIdx.y from the given probe sets; dot, decision key, running arg-max, partial
+// results per block and a last-block reduction per query.
 
 struct RowsSmemLayout {
-  uint32_t bars, hs, ring, selsm, sel, tok, total;
+  uint32_t bars, hs, ring, sel, tok, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline RowsSmemLayout rows_layout(uint32_t row_bytes, int K, int p,
-                                                      int rows_max, int mode) {
+__host__ __device__ inline RowsSmemLayout rows_layout(uint32_t row_bytes, int K, int p, int rows_max) {
   RowsSmemLayout L;
   L.bars = 0;
   L.hs = 1024;
   L.ring = align_up(L.hs + row_bytes, 128);
-  L.selsm = align_up(L.ring + (uint32_t)kWarps * K * row_bytes, 128);
-  L.sel = align_up(L.selsm + (mode == MODE_FUSED ? (uint32_t)sizeof(SelectSmem<kThreads>) : 0u), 16);
-  L.tok = align_up(L.sel + (mode == MODE_DENSE ? 0u : (uint32_t)p * 4u), 16);
-  L.total = align_up(L.tok + (mode == MODE_DENSE ? 0u : (uint32_t)rows_max * 4u), 128);
+  L.sel = align_up(L.ring + (uint32_t)kWarps * K * row_bytes, 16);
+  L.tok = align_up(L.sel + (uint32_t)p * 4u, 16);
+  L.total = align_up(L.tok + (uint32_t)rows_max * 4u, 128);
   return L;
 }
 
-template <int ELEM, int MODE, int KPT>
+template <int ELEM>
 __global__ void __launch_bounds__(kThreads) k_rows(const Stage2Params prm, int K, int rows_max) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int q = blockIdx.y;
   const uint32_t row_bytes = (uint32_t)(prm.d * (ELEM == kBF16 ? 2 : 4));
   const int nch = (int)(row_bytes / 16);
-  const RowsSmemLayout L = rows_layout(row_bytes, K, prm.p, rows_max, MODE);
+  const RowsSmemLayout L = rows_layout(row_bytes, K, prm.p, rows_max);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint8_t* hs = smem + L.hs;
   uint8_t* ring = smem + L.ring;
@@ -327,85 +241,45 @@ __global__ void __launch_bounds__(kThreads) k_rows(const Stage2Params prm, int K
   __shared__ unsigned long long warp_best[kWarps];
   __shared__ bool is_last;
 
-  // ---- prologue (independent of the previous kernel)
   if (tid < kWarps * K) mbar_init(&bars[tid], 1);
   fence_mbar_init();
   block_copy_g2s(hs, static_cast<const uint8_t*>(prm.H) + (size_t)q * row_bytes, row_bytes);
-  pdl_wait_prior();
-
-  // ---- probe set S of this query
-  const int64_t b = prm.b;
-  if (MODE == MODE_FUSED) {
-    SelectSmem<kThreads>& ssm = *reinterpret_cast<SelectSmem<kThreads>*>(smem + L.selsm);
-    const float* krow = prm.keys + (size_t)q * prm.c;
-    float x[KPT];
-    const int base = tid * KPT;
-#pragma unroll
-    for (int j = 0; j < KPT; ++j) x[j] = (base + j < prm.c) ? krow[base + j] : 0.0f;
-    block_select_topp<kThreads, KPT>(x, (int)prm.c, prm.p, ssm, sel_s);
-    if (prm.dbg_sel && blockIdx.x == 0)
-      for (int r = tid; r < prm.p; r += kThreads) prm.dbg_sel[(size_t)q * prm.p + r] = sel_s[r];
-  } else if (MODE == MODE_SEL) {
-    for (int r = tid; r < prm.p; r += kThreads) sel_s[r] = prm.sel[(size_t)q * prm.p + r];
-  }
+  for (int r = tid; r < prm.p; r += kThreads) sel_s[r] = prm.sel[(size_t)q * prm.p + r];
   __syncthreads();
 
-  const int64_t rows = (MODE == MODE_DENSE) ? prm.v : (int64_t)prm.p * b;
-  const int64_t lo = rows * blockIdx.x / gridDim.x;
-  const int64_t hi = rows * (blockIdx.x + 1) / gridDim.x;
+  const int64_t b = prm.b;
+  const int64_t P = (int64_t)prm.p * b;
+  const int64_t lo = P * blockIdx.x / gridDim.x;
+  const int64_t hi = P * (blockIdx.x + 1) / gridDim.x;
   const uint8_t* E = static_cast<const uint8_t*>(prm.E);
   const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
-  const bool perm = (MODE != MODE_DENSE) && Ep != nullptr;
-
-  // token ids of this block's rows (candidates only)
-  auto load_toks = [&]() {
-    for (int64_t i = lo + tid; i < hi; i += kThreads)
-      tok_s[i - lo] = prm.C2T[(int64_t)sel_s[i / b] * b + i % b];
-  };
+  const bool perm = Ep != nullptr;
   auto src = [&](int64_t i) -> const uint8_t* {
-    if (MODE == MODE_DENSE) return E + (size_t)i * row_bytes;
     if (perm) return Ep + (size_t)((int64_t)sel_s[i / b] * b + i % b) * row_bytes;
     return E + (size_t)tok_s[i - lo] * row_bytes;
   };
-  // The first K rows of each warp are issued before the token ids are known when the cluster-major
-  // copy gives their addresses directly.
   const int64_t first = lo + warp;
   int64_t nw = (first < hi) ? (hi - first + kWarps - 1) / kWarps : 0;
-  if (MODE != MODE_DENSE) {
-    if (perm && lane == 0)
-      for (int n = 0; n < K && n < nw; ++n) {
-        mbar_arrive_expect_tx(&bars[warp * K + n], row_bytes);
-        bulk_g2s(ring + ((size_t)warp * K + n) * row_bytes, src(first + (int64_t)kWarps * n),
-                 row_bytes, &bars[warp * K + n]);
-      }
-    load_toks();
-    __syncthreads();
-    if (!perm && lane == 0)
-      for (int n = 0; n < K && n < nw; ++n) {
-        mbar_arrive_expect_tx(&bars[warp * K + n], row_bytes);
-        bulk_g2s(ring + ((size_t)warp * K + n) * row_bytes, src(first + (int64_t)kWarps * n),
-                 row_bytes, &bars[warp * K + n]);
-      }
-  } else if (lane == 0) {
-    for (int n = 0; n < K && n < nw; ++n) {
-      mbar_arrive_expect_tx(&bars[warp * K + n], row_bytes);
-      bulk_g2s(ring + ((size_t)warp * K + n) * row_bytes, src(first + (int64_t)kWarps * n),
-               row_bytes, &bars[warp * K + n]);
-    }
-  }
-
-  // ---- stream the rows: dot, decision key, running arg-max
-  const uint32_t hs_addr = smem_addr(hs);
-  const int64_t P = (MODE == MODE_DENSE) ? prm.v : (int64_t)prm.p * b;
-  unsigned long long best = 0ull;
   uint8_t* ring_w = ring + (size_t)warp * K * row_bytes;
   uint64_t* bars_w = bars + warp * K;
+  // With the cluster-major copy the first rows are issued before the token ids are loaded.
+  if (perm && lane == 0)
+    for (int n = 0; n < K && n < nw; ++n)
+      issue_row(ring_w + (size_t)n * row_bytes, src(first + (int64_t)kWarps * n), row_bytes, &bars_w[n]);
+  for (int64_t i = lo + tid; i < hi; i += kThreads)
+    tok_s[i - lo] = prm.C2T[(int64_t)sel_s[i / b] * b + i % b];
+  __syncthreads();
+  if (!perm && lane == 0)
+    for (int n = 0; n < K && n < nw; ++n)
+      issue_row(ring_w + (size_t)n * row_bytes, src(first + (int64_t)kWarps * n), row_bytes, &bars_w[n]);
+
+  const uint32_t hs_addr = smem_addr(hs);
+  unsigned long long best = 0ull;
   for (int64_t n = 0; n < nw; ++n) {
     const int slot = (int)(n % K);
     if (!mbar_wait(&bars_w[slot], (uint32_t)((n / K) & 1), prm.status)) {
       for (int64_t m = n + 1; m < nw && m < n + K; ++m)
         mbar_wait(&bars_w[m % K], (uint32_t)((m / K) & 1), nullptr, 50000000ull);
-      nw = n;
       break;
     }
     const int64_t i = first + (int64_t)kWarps * n;
@@ -415,11 +289,10 @@ __global__ void __launch_bounds__(kThreads) k_rows(const Stage2Params prm, int K
     if (lane == 0) {
       if (n + K < nw) {
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&bars_w[slot], row_bytes);
-        bulk_g2s(ring_w + (size_t)slot * row_bytes, src(first + (int64_t)kWarps * (n + K)), row_bytes,
-                 &bars_w[slot]);
+        issue_row(ring_w + (size_t)slot * row_bytes, src(first + (int64_t)kWarps * (n + K)), row_bytes,
+                  &bars_w[slot]);
       }
-      const uint32_t tok = (MODE == MODE_DENSE) ? (uint32_t)i : (uint32_t)tok_s[i - lo];
+      const uint32_t tok = (uint32_t)tok_s[i - lo];
       float val = z;
       if (prm.sample)
         val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, 1u, tok));
@@ -430,7 +303,6 @@ __global__ void __launch_bounds__(kThreads) k_rows(const Stage2Params prm, int K
     }
   }
 
-  // ---- block arg-max, then the last block of this query reduces all partial results
   if (lane == 0) warp_best[warp] = best;
   __syncthreads();
   if (tid == 0) {
@@ -442,19 +314,17 @@ __global__ void __launch_bounds__(kThreads) k_rows(const Stage2Params prm, int K
     is_last = (t == gridDim.x - 1);
   }
   __syncthreads();
-  if (is_last) {
+  if (is_last && warp == 0) {
     __threadfence();
     unsigned long long bb = 0ull;
     for (uint32_t g = lane; g < gridDim.x; g += 32) {
       const unsigned long long v = __ldcg(&prm.part[(size_t)q * gridDim.x + g]);
       bb = v > bb ? v : bb;
     }
-    if (warp == 0) {
-      bb = warp_max_u64(bb);
-      if (lane == 0) {
-        if (prm.out_tok) prm.out_tok[q] = (int32_t)best_id(bb);
-        prm.tickets[q] = 0u;
-      }
+    bb = warp_max_u64(bb);
+    if (lane == 0) {
+      if (prm.out_tok) prm.out_tok[q] = (int32_t)best_id(bb);
+      prm.tickets[q] = 0u;
     }
   }
 }
@@ -467,7 +337,7 @@ __global__ void __launch_bounds__(kThreads) k_dense(const DenseParams prm, int K
   const int q = blockIdx.y;
   const uint32_t row_bytes = (uint32_t)(prm.d * (ELEM == kBF16 ? 2 : 4));
   const int nch = (int)(row_bytes / 16);
-  const RowsSmemLayout L = rows_layout(row_bytes, K, 0, 0, MODE_DENSE);
+  const RowsSmemLayout L = rows_layout(row_bytes, K, 0, 0);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint8_t* hs = smem + L.hs;
   uint8_t* ring = smem + L.ring;
@@ -591,7 +461,7 @@ __global__ void k_mc_partition(const float* z, const int32_t* C2T, int64_t v, in
   }
 }
 
-constexpr int kMcThreads = 256;
+constexpr int kMcThreads = 512;
 
 template <int KPT>
 __global__ void __launch_bounds__(kMcThreads) k_mc_draws(const McParams prm) {
@@ -626,26 +496,27 @@ __global__ void __launch_bounds__(kMcThreads) k_mc_draws(const McParams prm) {
   const int64_t lo = prm.N * blockIdx.x / gridDim.x;
   const int64_t hi = prm.N * (blockIdx.x + 1) / gridDim.x;
   for (int64_t i = lo; i < hi; ++i) {
-    float x[KPT];
+    uint32_t key[KPT];
 #pragma unroll
     for (int g = 0; g < KPT / 4; ++g) {
       const uint4 w = philox_block(prm.seed, (uint64_t)i, (uint32_t)q, 2u, (uint32_t)((base >> 2) + g));
-      x[4 * g + 0] = sdiv[4 * g + 0] + gumbel_from_u32(w.x);
-      x[4 * g + 1] = sdiv[4 * g + 1] + gumbel_from_u32(w.y);
-      x[4 * g + 2] = sdiv[4 * g + 2] + gumbel_from_u32(w.z);
-      x[4 * g + 3] = sdiv[4 * g + 3] + gumbel_from_u32(w.w);
-    }
-    const uint64_t mine = block_select_topp<kMcThreads, KPT>(x, (int)c, prm.p, sm, nullptr);
-    double acc = 0.0;
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int j = 0; j < KPT; ++j)
-      if (mine >> j & 1ull) acc += prm.Z[(size_t)q * c + base + j];
+      for (int e = 0; e < 4; ++e) {
+        const int j = 4 * g + e;
+        key[j] = (base + j < c) ? float_key(sdiv[j] + gumbel_from_u32(wv[e])) : 0u;
+      }
+    }
+    const uint32_t mine = block_select_topp<kMcThreads, KPT>(key, (int)c, prm.p, sm, nullptr);
+    double acc = 0.0;
+    for (uint32_t bits = mine; bits; bits &= bits - 1)
+      acc += prm.Z[(size_t)q * c + base + __ffs(bits) - 1];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
     if (lane == 0) red[wid] = acc;
     for (int j = 0; j < prm.T; ++j) {
       const int k = tcl[j];
-      if (k >= base && k < base + KPT) tsel[j] = (mine >> (k - base)) & 1ull ? 1 : 0;
+      if (k >= base && k < base + KPT) tsel[j] = (mine >> (k - base)) & 1u ? 1 : 0;
     }
     __syncthreads();
     if (tid == 0) {
@@ -655,7 +526,7 @@ __global__ void __launch_bounds__(kMcThreads) k_mc_draws(const McParams prm) {
     }
     __syncthreads();
     for (int j = tid; j < prm.T; j += kMcThreads)
-      prm.per_draw[((size_t)q * prm.N + i) * prm.T + j] = tsel[j] ? tnum[j] / denom_s : 0.0;
+      prm.per_draw[((size_t)q * prm.N + i) * prm.T + j] = (tcl[j] >= 0 && tsel[j]) ? tnum[j] / denom_s : 0.0;
     __syncthreads();
   }
 }
@@ -748,14 +619,11 @@ cudaError_t launch_gumbel_keys(const float* s, float* keys, int B, int64_t c, fl
 }
 
 cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p, cudaStream_t st) {
-  const int64_t kpt = (c + kSelThreads - 1) / kSelThreads;
-#define FH_SEL(KP) k_select<KP><<<B, kSelThreads, 0, st>>>(keys, sel, c, p)
-  if (kpt <= 4) FH_SEL(4);
-  else if (kpt <= 8) FH_SEL(8);
-  else if (kpt <= 16) FH_SEL(16);
-  else if (kpt <= 32) FH_SEL(32);
-  else FH_SEL(64);
-#undef FH_SEL
+  if (c <= 512 * 4) k_select<512, 4><<<B, 512, 0, st>>>(keys, sel, c, p);
+  else if (c <= 512 * 8) k_select<512, 8><<<B, 512, 0, st>>>(keys, sel, c, p);
+  else if (c <= 512 * 16) k_select<512, 16><<<B, 512, 0, st>>>(keys, sel, c, p);
+  else if (c <= 512 * 32) k_select<512, 32><<<B, 512, 0, st>>>(keys, sel, c, p);
+  else k_select<1024, 32><<<B, 1024, 0, st>>>(keys, sel, c, p);
   return cudaGetLastError();
 }
 
@@ -766,46 +634,22 @@ int stage2_blocks(int64_t rows, int B, int num_sms) {
   return (int)(g < 1 ? 1 : g);
 }
 
-cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st,
-                          bool pdl_secondary) {
+cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st) {
   const uint32_t row_bytes = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
   const int K = ring_slots(row_bytes, 128 * 1024);
   const int64_t P = (int64_t)prm.p * prm.b;
   const int G = stage2_blocks(P, prm.B, num_sms);
   const int rows_max = (int)((P + G - 1) / G);
-  const int mode = prm.keys ? MODE_FUSED : MODE_SEL;
-  const RowsSmemLayout L = rows_layout(row_bytes, K, prm.p, rows_max, mode);
+  const RowsSmemLayout L = rows_layout(row_bytes, K, prm.p, rows_max);
   const size_t smem = L.total;
-  const int64_t kpt = (prm.c + kThreads - 1) / kThreads;
-
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(G, prm.B);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl_secondary ? 1 : 0;
   cudaError_t e;
-#define FH_ROWS(EL, MO, KP)                                                        \
-  do {                                                                             \
-    if ((e = set_smem(k_rows<EL, MO, KP>, smem)) != cudaSuccess) return e;         \
-    e = cudaLaunchKernelEx(&cfg, k_rows<EL, MO, KP>, prm, K, rows_max);            \
-  } while (0)
-#define FH_ROWS_E(EL)                                     \
-  do {                                                    \
-    if (mode == MODE_SEL) FH_ROWS(EL, MODE_SEL, 1);       \
-    else if (kpt <= 8) FH_ROWS(EL, MODE_FUSED, 8);        \
-    else if (kpt <= 16) FH_ROWS(EL, MODE_FUSED, 16);      \
-    else if (kpt <= 32) FH_ROWS(EL, MODE_FUSED, 32);      \
-    else FH_ROWS(EL, MODE_FUSED, 64);                     \
-  } while (0)
-  if (elem == kBF16) FH_ROWS_E(kBF16); else FH_ROWS_E(kF32);
-#undef FH_ROWS_E
-#undef FH_ROWS
-  if (e != cudaSuccess) return e;
+  if (elem == kBF16) {
+    if ((e = set_smem(k_rows<kBF16>, smem)) != cudaSuccess) return e;
+    k_rows<kBF16><<<dim3(G, prm.B), kThreads, smem, st>>>(prm, K, rows_max);
+  } else {
+    if ((e = set_smem(k_rows<kF32>, smem)) != cudaSuccess) return e;
+    k_rows<kF32><<<dim3(G, prm.B), kThreads, smem, st>>>(prm, K, rows_max);
+  }
   return cudaGetLastError();
 }
 
@@ -813,7 +657,7 @@ cudaError_t launch_dense(const DenseParams& prm, int elem, int num_sms, cudaStre
   const uint32_t row_bytes = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
   const int K = ring_slots(row_bytes, 128 * 1024);
   const int G = stage2_blocks(prm.v, prm.B, num_sms);
-  const RowsSmemLayout L = rows_layout(row_bytes, K, 0, 0, MODE_DENSE);
+  const RowsSmemLayout L = rows_layout(row_bytes, K, 0, 0);
   const size_t smem = L.total;
   cudaError_t e;
   if (elem == kBF16) {
@@ -872,17 +716,17 @@ cudaError_t launch_mc(const McParams& prm, int num_sms, cudaStream_t st) {
   k_mc_partition<<<1024, 256, 0, st>>>(prm.z, prm.C2T, prm.v, prm.c, prm.b, prm.tau, prm.zmax, prm.Z,
                                        prm.B);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int64_t kpt = (prm.c + kMcThreads - 1) / kMcThreads;
   int64_t gd = (4 * (int64_t)num_sms + prm.B - 1) / prm.B;
   if (gd > prm.N) gd = prm.N;
   dim3 grid((unsigned)gd, prm.B);
 #define FH_MC(KP) k_mc_draws<KP><<<grid, kMcThreads, 0, st>>>(prm)
-  if (kpt <= 4) FH_MC(4);
-  else if (kpt <= 8) FH_MC(8);
-  else if (kpt <= 16) FH_MC(16);
-  else if (kpt <= 32) FH_MC(32);
-  else if (kpt <= 40) FH_MC(40);
-  else FH_MC(64);
+  if (prm.c <= kMcThreads * 4) FH_MC(4);
+  else if (prm.c <= kMcThreads * 8) FH_MC(8);
+  else if (prm.c <= kMcThreads * 12) FH_MC(12);
+  else if (prm.c <= kMcThreads * 16) FH_MC(16);
+  else if (prm.c <= kMcThreads * 20) FH_MC(20);
+  else if (prm.c <= kMcThreads * 24) FH_MC(24);
+  else FH_MC(32);
 #undef FH_MC
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const int warps = prm.B * prm.T;

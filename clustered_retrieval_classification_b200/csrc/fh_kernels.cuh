@@ -85,6 +85,38 @@ struct McParams {
   uint32_t* status;
 };
 
+// The batch-1 persistent head (fh_head1.cu).
+struct Head1Params {
+  const void* C;               // c x d (dense Stage 1) or null
+  const uint8_t* q4;           // c x d/2 (INT4 Stage 1) or null
+  const uint16_t* scales;      // c x d/32
+  const void* H;               // 1 x d
+  const void* E;               // v x d
+  const void* E_perm;          // v x d cluster-major copy, or null
+  const int32_t* C2T;          // c x b
+  float* keys;                 // c: Stage-1 keys (workspace)
+  int64_t c, d, b;
+  int p;
+  int sample;
+  float tau;
+  uint64_t seed, step;
+  uint32_t* bar_count;         // grid barrier arrival counter (zero between calls)
+  uint32_t* bar_gen;           // grid barrier generation
+  uint32_t* ticket;            // arrival counter of the final reduction (zero between calls)
+  unsigned long long* best;    // packed (key, ~token) maximum (zero between calls)
+  int32_t* out_tok;
+  int32_t* dbg_sel;            // p or null
+  int32_t* dbg_tok;            // p*b or null
+  float* dbg_logit;            // p*b or null
+  uint32_t* status;
+  int k1, k2;                  // ring slots per warp in Stage 1 / Stage 2 (set by the launcher)
+  uint32_t ring_bytes;         // (set by the launcher)
+};
+
+// Threads per block of the persistent head for c clusters (0: not supported, use the batched path).
+int head1_threads(int64_t c);
+cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaStream_t st);
+
 // ---- launchers (return cudaGetLastError() of the launch) ----
 cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_sms,
                           cudaStream_t st, bool pdl_primary);
@@ -93,8 +125,7 @@ cudaError_t launch_gumbel_keys(const float* s, float* keys, int B, int64_t c, fl
                                cudaStream_t st);
 cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p,
                           cudaStream_t st);
-cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st,
-                          bool pdl_secondary);
+cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st);
 cudaError_t launch_dense(const DenseParams& prm, int elem, int num_sms, cudaStream_t st);
 cudaError_t launch_gather(const int32_t* C2T, int64_t b, const int32_t* sel, int B, int p,
                           int32_t* cand, cudaStream_t st);

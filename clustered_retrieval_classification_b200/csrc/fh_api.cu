@@ -33,7 +33,7 @@ fh_status cuda_fail(cudaError_t e, const char* what) {
   return fail(FH_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
-constexpr size_t kHeaderBytes = 1024;   // status word + per-query tickets
+constexpr size_t kHeaderBytes = 1024 + 4096;  // control words, then the score histogram
 constexpr size_t kAlign = 256;
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -88,9 +88,11 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 // Workspace header (first kHeaderBytes): status word at 0, per-query tickets at 16 (64 x 4 bytes),
-// the persistent head's grid-barrier counter / generation / ticket at 512, 516, 520 and its packed
-// arg-max at 528.  Counters return to zero at the end of every call; a new workspace must start
-// zeroed (fh_ws_status re-zeroes the header after reporting a device-side error).
+// the persistent head's 64-bit grid-barrier arrival counter at 512, its 64-bit final-reduction
+// ticket at 520 and its packed arg-max at 528; bytes [1024, 5120) hold its 1024-bin score histogram
+// in every layout, so no other call ever writes there.  The two counters only grow (each call adds
+// one grid's worth); the arg-max and the histogram return to zero at the end of every call.  A new
+// workspace must start zeroed (fh_ws_status re-zeroes the header after a device-side error).
 uint32_t* status_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16); }
 uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
@@ -137,7 +139,9 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   int32_t* sel = reinterpret_cast<int32_t*>(base + L.sel);
 
   cudaError_t e;
-  if (B == 1 && fh::head1_threads(D.c) != 0) {
+  // The persistent batch-1 kernel copies 16-byte C2T chunks next to each row, so it needs C2T
+  // 16-byte aligned and v % 4 == 0 (no chunk runs past the end of C2T).
+  if (B == 1 && fh::head1_threads(D.c) != 0 && D.v % 4 == 0 && aligned16(D.C2T)) {
     fh::Head1Params h = {};
     h.C = D.C;
     h.q4 = D.C_q4;
@@ -155,10 +159,10 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     h.tau = tau;
     h.seed = seed;
     h.step = step;
-    h.bar_count = word_at(ws, 512);
-    h.bar_gen = word_at(ws, 516);
-    h.ticket = word_at(ws, 520);
+    h.bar_count = reinterpret_cast<unsigned long long*>(word_at(ws, 512));
+    h.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, 520));
     h.best = reinterpret_cast<unsigned long long*>(word_at(ws, 528));
+    h.hist = word_at(ws, 1024);
     h.out_tok = out_tok;
     h.dbg_sel = dbg ? dbg->sel : nullptr;
     h.dbg_tok = dbg ? dbg->cand_tok : nullptr;

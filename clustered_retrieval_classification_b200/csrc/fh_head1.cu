@@ -4,19 +4,25 @@
 // every launch boundary and every serial step between the two bandwidth phases shows.  One kernel
 // therefore runs the whole path (FlashHead notes, overall architecture and Figure 1):
 //
-//   1. Stage 1: every block bulk-copies its share of centroid rows (C, or the INT4 nibbles) into its
-//      shared-memory ring at once, computes s = C·h (or the Gumbel key s/τ + G) and writes the keys.
-//   2. Grid barrier (self-resetting arrival counter + generation word, bounded wait).
-//   3. Selection, redundantly in every block (FlashHead notes, Module 2): topp_bin finds the boundary
-//      bin; the clusters above it are certain, so their Stage-2 rows are issued right away, and the
-//      boundary bin is resolved (topp_resolve) while those copies are in flight.
+//   1. Stage 1: each block loads h, then bulk-copies its share of centroid rows (C, or the INT4
+//      nibbles) into its shared-memory ring at once, computes s = C·h (or the Gumbel key s/τ + G),
+//      writes the keys, and adds each key to a 1024-bin histogram in global memory.  The bins cover a
+//      range fixed in advance from ‖h‖ (unit centroids give |s| <= ‖h‖; the Gumbel term lies in
+//      [-2.9, 16.7]); keys outside are clamped into the end bins, so the binning is monotone for any
+//      input and only its resolution depends on the range.
+//   2. Grid barrier (monotonic 64-bit arrival counter, bounded wait).
+//   3. Selection, redundantly in every block (FlashHead notes, Module 2): the histogram gives the
+//      boundary bin; clusters above it are certain and their Stage-2 rows are issued at once; the
+//      boundary bin is then resolved exactly (rank, or radix passes when crowded) while they fly.
 //   4. Stage 2 (FlashHead notes, Module 1 and Figure 1): the block streams its slice of the p·b
-//      candidate rows (cluster-major copy E_perm when present, else E through C2T), computes the exact
-//      logits and keeps the arg-max of z (greedy, Eq. 2) or of z/τ + G' (sampling, Eq. 3).
+//      candidate rows, each together with the 16-byte C2T chunk holding its token id, computes the
+//      exact logits and keeps the arg-max of z (greedy, Eq. 2) or of z/τ + G' (sampling, Eq. 3).
 //   5. Each block folds its best (value, token) into one 64-bit atomicMax; the last block to arrive
-//      writes the token and resets the call's counters.
+//      writes the token and clears the histogram and the maximum for the next call.
 //
-// Slots of Stage 2 are ordered "certain clusters by ascending id, then the boundary clusters taken, by
+// No global load waits behind the bulk copies: every small dependent load (h, INT4 scales, keys,
+// histogram) is issued before the block's copies, and token ids arrive inside the row copies.
+// Stage-2 slots are ordered "certain clusters by ascending id, then the boundary clusters taken, by
 // ascending id"; the arg-max does not depend on the order, and the optional debug outputs are written
 // in the canonical ascending order.
 #include "fh_device.cuh"
@@ -26,46 +32,111 @@
 
 namespace fh {
 
+constexpr int kHistBins = 1024;
+
 struct Head1Layout {
-  uint32_t bars1, bars2, hs, sc, sel, rank_cl, asc, tok, ring, total;
+  uint32_t bars1, bars2, hs, sc, sel, hist, rank_cl, asc, tokc, ring, total;
 };
 
 __host__ __device__ inline uint32_t h1_align(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 template <int NT>
-__host__ __device__ inline Head1Layout head1_layout(uint32_t row2, int rows1_max, int nch4,
-                                                    int rmax, int rows2_max, uint32_t ring_bytes) {
+__host__ __device__ inline Head1Layout head1_layout(uint32_t row2, int rows1_max, int nch4, int rmax,
+                                                    int slots2, uint32_t ring_bytes) {
   Head1Layout L;
   L.bars1 = 0;
   L.bars2 = 1024;
   L.hs = 2048;
   L.sc = h1_align(L.hs + row2, 128);
-  L.sel = h1_align(L.sc + (uint32_t)rows1_max * nch4 * 2u, 128);
-  L.rank_cl = h1_align(L.sel + (uint32_t)sizeof(SelectSmem<NT>), 16);
+  L.sel = h1_align(L.sc + (uint32_t)rows1_max * nch4 * 2u + 4u, 128);
+  L.hist = h1_align(L.sel + (uint32_t)sizeof(SelectSmem<NT>), 16);
+  L.rank_cl = h1_align(L.hist + kHistBins * 4u, 16);
   L.asc = h1_align(L.rank_cl + (uint32_t)rmax * 4u, 16);
-  L.tok = h1_align(L.asc + (uint32_t)rmax * 4u, 16);
-  L.ring = h1_align(L.tok + (uint32_t)rows2_max * 4u, 128);
+  L.tokc = h1_align(L.asc + (uint32_t)rmax * 4u, 16);
+  L.ring = h1_align(L.tokc + (uint32_t)slots2 * 16u, 128);
   L.total = L.ring + ring_bytes;
   return L;
 }
 
-// Wait for the whole grid.  Returns false if the wait timed out (status set).
-__device__ __forceinline__ bool grid_barrier(uint32_t* count, uint32_t* gen, uint32_t nblocks,
+// Monotone binning of a key into [0, kHistBins): the same function in Stage 1 and in the selection.
+struct Binning {
+  float lo, scale;
+  __device__ __forceinline__ uint32_t operator()(float x) const {
+    const float t = (x - lo) * scale;
+    return (uint32_t)min(kHistBins - 1, max(0, (int)t));
+  }
+};
+
+// Smallest order-preserving key image u with bin(value of u) >= d (d in [1, kHistBins)), found by a
+// warp-wide 32-ary search over the images of finite floats; bin is monotone in u there, so a key is in
+// a bin >= d exactly when its image is >= the returned edge.  Called by a whole warp.
+__device__ __forceinline__ uint32_t bin_edge_image(const Binning& bin, uint32_t d) {
+  const int lane = threadIdx.x & 31;
+  uint32_t lo = 0x007FFFFFu, hi = 0xFF800000u;  // images of -inf and +inf
+  if (bin(key_float(hi)) < d) return 0xFFFFFFFFu;  // no finite key reaches bin d
+  if (bin(key_float(lo)) >= d) return lo;
+  // invariant: bin(lo) < d <= bin(hi); each round shrinks hi - lo by a factor of ~32
+  for (int round = 0; round < 12 && hi - lo > 1u; ++round) {
+    const uint32_t step = (hi - lo) / 32u + 1u;
+    const uint32_t u = min(hi, lo + step * (uint32_t)lane + step);
+    const bool ge = bin(key_float(u)) >= d;
+    const uint32_t mask = __ballot_sync(0xFFFFFFFFu, ge);  // lanes at and after the edge
+    const int first = __ffs(mask) - 1;
+    const uint32_t nhi = first >= 0 ? min(hi, lo + step * (uint32_t)first + step) : hi;
+    const uint32_t nlo = first > 0 ? lo + step * (uint32_t)(first - 1) + step : lo;
+    lo = nlo;
+    hi = nhi;
+  }
+  return hi;
+}
+
+// The same edge from the inverse of the binning, corrected by a few one-image steps; falls back to
+// the warp search when the correction does not settle.  Called by a whole warp.
+__device__ __forceinline__ uint32_t bin_edge(const Binning& bin, uint32_t d) {
+  bool ok = false;
+  uint32_t u = 0;
+  if (bin.scale > 0.0f) {
+    const float x0 = bin.lo + (float)d / bin.scale;
+    if (isfinite(x0)) {
+      u = float_key(x0);
+      for (int it = 0; it < 16 && u < 0xFF800000u && bin(key_float(u)) < d; ++it) ++u;
+      for (int it = 0; it < 16 && u > 0x00800000u && bin(key_float(u - 1u)) >= d; ++it) --u;
+      ok = u > 0x00800000u && u <= 0xFF800000u && bin(key_float(u)) >= d &&
+           bin(key_float(u - 1u)) < d;
+    }
+  }
+  return ok ? u : bin_edge_image(bin, d);
+}
+
+// Every block computes the same ‖h‖ (same data, same reduction order) and from it the binning.
+__device__ __forceinline__ Binning make_binning(const float hnorm, int sample, float tau) {
+  Binning bn;
+  const float r = hnorm * 1.0625f + 1e-30f;
+  const float lo = sample ? -r / tau - 3.0f : -r;
+  const float hi = sample ? r / tau + 17.0f : r;
+  bn.lo = lo;
+  bn.scale = (float)kHistBins / (hi - lo);
+  if (!(isfinite(bn.scale) && bn.scale > 0.0f)) bn.scale = 0.0f;  // everything in bin 0
+  return bn;
+}
+
+// Grid barrier on a monotonic 64-bit arrival counter: the call's last arrival makes the counter a
+// multiple of the grid size.  Returns false if the wait timed out (status set).
+__device__ __forceinline__ bool grid_barrier(unsigned long long* count, uint32_t nblocks,
                                              uint32_t* status, bool* abort_s) {
   __syncthreads();
   if (threadIdx.x == 0) {
     bool ok = true;
-    const uint32_t g0 = *reinterpret_cast<volatile uint32_t*>(gen);
     __threadfence();
-    const uint32_t arrived = atomicAdd(count, 1u);
-    if (arrived == nblocks - 1) {
-      *reinterpret_cast<volatile uint32_t*>(count) = 0u;
-      __threadfence();
-      atomicAdd(gen, 1u);
-    } else {
+    const unsigned long long old = atomicAdd(count, 1ull);
+    const unsigned long long target = (old / nblocks + 1) * nblocks;
+    if (old + 1 != target) {
       const uint64_t t0 = global_timer_ns();
       uint32_t it = 0;
-      while (*reinterpret_cast<volatile uint32_t*>(gen) == g0) {
+      for (;;) {
+        unsigned long long now;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(now) : "l"(count) : "memory");
+        if (now >= target) break;
         if ((++it & 255u) == 0 && global_timer_ns() - t0 > 500000000ull) {
           set_status(status, kStatusTimeout);
           ok = false;
@@ -85,80 +156,132 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int W = NT / 32;
   __shared__ unsigned long long warp_best[W];
-  __shared__ bool abort_s;
+  __shared__ float red_s[W];
+  __shared__ bool abort_s, last_s;
+  __shared__ uint32_t dstar_s, above_s, total_s, edge_lo_s, edge_hi_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x, bid = blockIdx.x;
-  const int64_t c = prm.c, d = prm.d, b = prm.b;
-  const uint32_t row2 = (uint32_t)(d * (ELEM == kBF16 ? 2 : 4));   // E row bytes
-  const uint32_t row1 = INT4_MCH ? (uint32_t)(d / 2) : row2;        // stage-1 row bytes
+  const int64_t c = prm.c, d = prm.d;
+  const int b = (int)prm.b;
+  const uint32_t row2 = (uint32_t)(d * (ELEM == kBF16 ? 2 : 4));  // E row bytes
+  const uint32_t row1 = INT4_MCH ? (uint32_t)(d / 2) : row2;       // Stage-1 row bytes
   const int nch2 = (int)(row2 / 16);
   const int nch4 = INT4_MCH ? (int)(d / 32) : 0;
-  const int64_t P = (int64_t)prm.p * b;
+  const int P = prm.p * b;
   const int rows1_max = (int)((c + G - 1) / G);
   const int rows2_max = (int)((P + G - 1) / G);
   const int rmax = (int)(rows2_max / b) + 2;
-  const Head1Layout L =
-      head1_layout<NT>(row2, INT4_MCH ? rows1_max : 0, nch4, rmax, rows2_max, prm.ring_bytes);
+  const int K1 = prm.k1, K2 = prm.k2;
+  const Head1Layout L = head1_layout<NT>(row2, INT4_MCH ? rows1_max : 0, nch4, rmax, W * K2,
+                                         prm.ring_bytes);
   uint64_t* bars1 = reinterpret_cast<uint64_t*>(smem + L.bars1);
   uint64_t* bars2 = reinterpret_cast<uint64_t*>(smem + L.bars2);
   uint8_t* hs = smem + L.hs;
   uint16_t* sc_s = reinterpret_cast<uint16_t*>(smem + L.sc);
   SelectSmem<NT>& sm = *reinterpret_cast<SelectSmem<NT>*>(smem + L.sel);
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L.hist);
   int* rank_cl = reinterpret_cast<int*>(smem + L.rank_cl);
   int* asc_of = reinterpret_cast<int*>(smem + L.asc);
-  int32_t* tok_s = reinterpret_cast<int32_t*>(smem + L.tok);
+  uint4* tokc = reinterpret_cast<uint4*>(smem + L.tokc);
   uint8_t* ring = smem + L.ring;
-  const int K1 = prm.k1, K2 = prm.k2;
 
+  // ------------------------------------------------------------------ prologue: h before any copy
+  uint4 hv[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int ch = tid + u * NT;
+    if (ch < nch2) hv[u] = __ldg(reinterpret_cast<const uint4*>(prm.H) + ch);
+  }
+  const int64_t lo1 = c * bid / G, hi1 = c * (bid + 1) / G;
+  uint32_t scv[4];  // INT4: this block's group scales, two per 32-bit word
+  const int nsc = INT4_MCH ? (int)((hi1 - lo1) * nch4) : 0;
+  const int sc_words = (nsc + 1) / 2;
+  if constexpr (INT4_MCH > 0) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int w = tid + u * NT;
+      if (w < sc_words) {
+        const int64_t e = lo1 * nch4 + 2 * (int64_t)w;  // scales are read as pairs
+        const uint32_t a = prm.scales[e];
+        const uint32_t bb = (2 * w + 1 < nsc) ? prm.scales[e + 1] : 0u;
+        scv[u] = a | (bb << 16);
+      }
+    }
+  }
   if (tid < W * K1) mbar_init(&bars1[tid], 1);
   if (tid < W * K2) mbar_init(&bars2[tid], 1);
+  uint64_t* bar_keys = &bars2[127];  // keys + histogram copy after the grid barrier
+  if (tid == 0) mbar_init(bar_keys, 1);
   fence_mbar_init();
   __syncthreads();
 
   // ------------------------------------------------------------------ Stage 1
-  const int64_t lo1 = c * bid / G, hi1 = c * (bid + 1) / G;
   const int64_t first1 = lo1 + warp;
-  const int64_t n1 = (first1 < hi1) ? (hi1 - first1 + W - 1) / W : 0;
+  const int n1 = (first1 < hi1) ? (int)((hi1 - first1 + W - 1) / W) : 0;
   uint8_t* ring1 = ring + (size_t)warp * K1 * row1;
   uint64_t* b1 = bars1 + warp * K1;
   const uint8_t* src1 = INT4_MCH ? static_cast<const uint8_t*>(static_cast<const void*>(prm.q4))
                                  : static_cast<const uint8_t*>(prm.C);
-  if (lane == 0)
-    for (int n = 0; n < K1 && n < n1; ++n)
-      issue_row(ring1 + (size_t)n * row1, src1 + (size_t)(first1 + (int64_t)W * n) * row1, row1, &b1[n]);
-  block_copy_g2s(hs, static_cast<const uint8_t*>(prm.H), (int)row2);
+  if (lane < K1 && lane < n1)  // the first K1 rows of the warp, one lane each
+    issue_row(ring1 + (size_t)lane * row1, src1 + (size_t)(first1 + (int64_t)W * lane) * row1, row1,
+              &b1[lane]);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int ch = tid + u * NT;
+    if (ch < nch2) reinterpret_cast<uint4*>(hs)[ch] = hv[u];
+  }
+  if constexpr (INT4_MCH > 0) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int w = tid + u * NT;
+      if (w < sc_words) reinterpret_cast<uint32_t*>(sc_s)[w] = scv[u];
+    }
+  }
+  for (int i = tid; i < kHistBins; i += NT) hist_s[i] = 0u;
+  __syncthreads();
+  // ‖h‖ (fixed reduction order, identical in every block) and the key binning
+  float hsq = 0.0f;
+  for (int ch = tid; ch < nch2; ch += NT) {
+    const uint4 v = reinterpret_cast<const uint4*>(hs)[ch];
+    hsq = (ELEM == kBF16) ? dot8_bf16(v, v, hsq) : dot4_f32(v, v, hsq);
+  }
+  hsq = warp_sum(hsq);
+  if (lane == 0) red_s[warp] = hsq;
   float hreg[INT4_MCH ? INT4_MCH : 1][INT4_MCH ? 32 : 1];
   if constexpr (INT4_MCH > 0) {
-    for (int64_t i = tid; i < (hi1 - lo1) * nch4; i += NT) sc_s[i] = prm.scales[lo1 * nch4 + i];
-    const uint16_t* Hh = static_cast<const uint16_t*>(prm.H);
+    const uint16_t* Hs = reinterpret_cast<const uint16_t*>(hs);
 #pragma unroll
-    for (int m = 0; m < (INT4_MCH ? INT4_MCH : 1); ++m) {
+    for (int m = 0; m < INT4_MCH; ++m) {
       const int ch = lane + 32 * m;
 #pragma unroll
-      for (int e = 0; e < (INT4_MCH ? 32 : 1); ++e)
-        hreg[m][e] = (ch < nch4) ? __uint_as_float((uint32_t)Hh[32 * ch + e] << 16) : 0.0f;
+      for (int e = 0; e < 32; ++e)
+        hreg[m][e] = (ch < nch4) ? __uint_as_float((uint32_t)Hs[32 * ch + e] << 16) : 0.0f;
     }
   }
   __syncthreads();
+  float hn2 = 0.0f;
+#pragma unroll
+  for (int w = 0; w < W; ++w) hn2 += red_s[w];
+  const Binning bin = make_binning(sqrtf(hn2), prm.sample, prm.tau);
+
   const uint32_t hs_addr = smem_addr(hs);
-  for (int64_t n = 0; n < n1; ++n) {
-    const int slot = (int)(n % K1);
-    if (!mbar_wait(&b1[slot], (uint32_t)((n / K1) & 1), prm.status)) {
-      for (int64_t m = n + 1; m < n1 && m < n + K1; ++m)
+  for (int n = 0, slot = 0, phase = 0; n < n1; ++n) {
+    if (!mbar_wait(&b1[slot], (uint32_t)phase, prm.status)) {
+      for (int m = n + 1; m < n1 && m < n + K1; ++m)
         mbar_wait(&b1[m % K1], (uint32_t)((m / K1) & 1), nullptr, 50000000ull);
       break;
     }
-    const int64_t k = first1 + (int64_t)W * n;
+    const int k = (int)first1 + W * n;
     const uint32_t row_s = smem_addr(ring1 + (size_t)slot * row1);
     float s;
     if constexpr (INT4_MCH > 0) {
       float part = 0.0f;
 #pragma unroll
-      for (int m = 0; m < (INT4_MCH ? INT4_MCH : 1); ++m) {
+      for (int m = 0; m < INT4_MCH; ++m) {
         const int ch = lane + 32 * m;
         if (ch < nch4) {
           const uint4 w = lds_v4(row_s + ch * 16);
-          const float scale = __uint_as_float((uint32_t)sc_s[(k - lo1) * nch4 + ch] << 16);
+          const float scale = __uint_as_float((uint32_t)sc_s[(k - (int)lo1) * nch4 + ch] << 16);
           part = fmaf(scale, int4_group_dot(w, hreg[m]), part);
         }
       }
@@ -177,111 +300,220 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       if (prm.sample)
         key = s / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 0u, (uint32_t)k));
       prm.keys[k] = key;
+      atomicAdd(&hist_s[bin(key_float(float_key(key)))], 1u);
+    }
+    if (++slot == K1) {
+      slot = 0;
+      phase ^= 1;
     }
   }
+  __syncthreads();
+  for (int i = tid; i < kHistBins; i += NT)
+    if (hist_s[i]) atomicAdd(&prm.hist[i], hist_s[i]);
 
   // ------------------------------------------------------------------ grid barrier
-  if (!grid_barrier(prm.bar_count, prm.bar_gen, (uint32_t)G, prm.status, &abort_s)) return;
+  if (!grid_barrier(prm.bar_count, (uint32_t)G, prm.status, &abort_s)) return;
 
-  // ------------------------------------------------------------------ selection
+  // ------------------------------------------------------------------ boundary bin
+  // The keys written by every block and the summed histogram come in with one bulk copy into the
+  // ring, which is idle between the stages (the workspace pads the keys to a multiple of 16 bytes).
+  const uint32_t keys_bytes = (uint32_t)((c * 4 + 15) / 16 * 16);
+  float* keys_s = reinterpret_cast<float*>(ring);
+  uint32_t* histg_s = reinterpret_cast<uint32_t*>(ring + keys_bytes);
+  if (tid == 0) {
+    asm volatile("fence.proxy.async;" ::: "memory");  // other blocks' keys, seen via the barrier
+    mbar_arrive_expect_tx(bar_keys, keys_bytes + kHistBins * 4u);
+    bulk_g2s(keys_s, prm.keys, keys_bytes, bar_keys);
+    bulk_g2s(histg_s, prm.hist, kHistBins * 4u, bar_keys);
+  }
+  if (!mbar_wait(bar_keys, 0u, prm.status)) return;
   uint32_t key[KPT];
-  load_key_images<KPT>(prm.keys, (int)c, key);
-  const SelState st = topp_bin<NT, KPT>(key, (int)c, prm.p, sm);
-  const int base = tid * KPT;
-  const int64_t s0 = P * bid / G, s1 = P * (bid + 1) / G;
-  const int64_t r0 = s0 / b, r1 = (s1 + b - 1) / b;   // ranks this block touches
-  const int64_t certain_rows = (int64_t)st.above * b;
   {
-    const unsigned long long ex = block_scan2<NT>(__popc(st.certain), 0u, sm, 0);
-    int64_t r = (int64_t)(ex >> 32);
+    const int kb = tid * KPT;
+#pragma unroll
+    for (int j = 0; j < KPT; j += 4) {
+      if (kb + j + 4 <= c) {
+        const float4 f = *reinterpret_cast<const float4*>(keys_s + kb + j);
+        key[j] = float_key(f.x);
+        key[j + 1] = float_key(f.y);
+        key[j + 2] = float_key(f.z);
+        key[j + 3] = float_key(f.w);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) key[j + e] = (kb + j + e < c) ? float_key(keys_s[kb + j + e]) : 0u;
+      }
+    }
+  }
+  constexpr int HPT = kHistBins / NT;  // histogram bins per thread
+  uint32_t hb[HPT];
+  uint32_t htot = 0;
+#pragma unroll
+  for (int u = 0; u < HPT; ++u) {
+    hb[u] = histg_s[tid * HPT + u];
+    htot += hb[u];
+  }
+  for (int i = tid; i < 1025; i += NT) sm.selbits[i] = 0u;
+  if (tid == 0) {
+    sm.cand_count = 0u;
+    dstar_s = 0u;
+    above_s = 0u;
+  }
+  const bool all = prm.p >= c;
+  {
+    const unsigned long long ex = block_scan2<NT>(0u, htot, sm, 0);
+    const uint32_t before = (uint32_t)(ex & 0xFFFFFFFFull);
+    if (tid == NT - 1) total_s = before + htot;
+    __syncthreads();
+    uint32_t cum = total_s - before - htot;  // keys in bins above this thread's bins
+#pragma unroll
+    for (int u = HPT - 1; u >= 0; --u) {
+      if (!all && cum < (uint32_t)prm.p && cum + hb[u] >= (uint32_t)prm.p) {
+        dstar_s = (uint32_t)(tid * HPT + u);
+        above_s = cum;
+      }
+      cum += hb[u];
+    }
+    __syncthreads();
+    if (total_s != (uint32_t)c) {  // a Stage-1 wait gave up somewhere: nothing below is valid
+      if (tid == 0) set_status(prm.status, kStatusTimeout);
+      return;
+    }
+  }
+  SelState st;
+  {
+    const uint32_t dstar = all ? 0u : dstar_s;
+    st.above = all ? (uint32_t)c : above_s;
+    st.need = (uint32_t)prm.p - st.above;
+    // key images at the lower edges of bins d* and d*+1 (warps 0 and 1 search them)
+    if (warp == 0) {
+      const uint32_t e = (dstar == 0u) ? 1u : bin_edge(bin, dstar);
+      if (lane == 0) edge_lo_s = e;
+    } else if (warp == 1) {
+      const uint32_t e = (dstar + 1u >= (uint32_t)kHistBins) ? 0xFFFFFFFFu : bin_edge(bin, dstar + 1u);
+      if (lane == 0) edge_hi_s = e;
+    }
+    __syncthreads();
+    const uint32_t elo = edge_lo_s, ehi = edge_hi_s;
+    st.certain = 0u;
+    st.boundary = 0u;
+    const uint32_t all_u = all ? 1u : 0u;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {  // branch-free: plain 0/1 arithmetic per key
+      const uint32_t kj = key[j];
+      const uint32_t real = (uint32_t)(kj != 0u);
+      const uint32_t above = (uint32_t)(kj >= ehi);
+      const uint32_t inbin = (uint32_t)(kj >= elo) & (above ^ 1u);
+      st.certain |= (real & (all_u | above)) << j;
+      st.boundary |= (real & (all_u ^ 1u) & inbin) << j;
+    }
+  }
+  const int base = tid * KPT;
+  const int s0 = (int)((int64_t)P * bid / G), s1 = (int)((int64_t)P * (bid + 1) / G);
+  const int r0 = s0 / b, r1 = (s1 + b - 1) / b;  // ranks this block touches
+  const int certain_rows = (int)st.above * b;
+  {
+    const unsigned long long ex = block_scan2<NT>(__popc(st.certain), 0u, sm, 1);
+    int r = (int)(ex >> 32);
     for (uint32_t bits = st.certain; bits; bits &= bits - 1, ++r)
       if (r >= r0 && r < r1) rank_cl[r - r0] = base + __ffs(bits) - 1;
   }
   __syncthreads();
+
+  // ------------------------------------------------------------------ Stage-2 copies of certain rows
   const uint8_t* E = static_cast<const uint8_t*>(prm.E);
   const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
   const bool perm = Ep != nullptr;
-  const int64_t first2 = s0 + warp;
-  const int64_t n2 = (first2 < s1) ? (s1 - first2 + W - 1) / W : 0;
+  const int first2 = s0 + warp;
+  const int n2 = (first2 < s1) ? (s1 - first2 + W - 1) / W : 0;
   uint8_t* ring2 = ring + (size_t)warp * K2 * row2;
   uint64_t* b2 = bars2 + warp * K2;
-  auto row_src = [&](int64_t i) -> const uint8_t* {
-    const int64_t cl = rank_cl[i / b - r0];
-    if (perm) return Ep + (size_t)(cl * b + i % b) * row2;
-    return E + (size_t)tok_s[i - s0] * row2;
+  uint4* tokc_w = tokc + warp * K2;
+  // slot n of this warp: row i = first2 + W*n of cluster rank_cl[i/b - r0], row i % b within it
+  auto issue2 = [&](int n) {
+    const int slot = n % K2;
+    const int i = first2 + W * n;
+    const int q = i / b;
+    const int e = rank_cl[q - r0] * b + (i - q * b);  // flat C2T index = row of the cluster-major copy
+    const int32_t* chunk = prm.C2T + (e & ~3);        // 16-byte chunk holding the token id
+    mbar_arrive_expect_tx(&b2[slot], row2 + 16u);
+    bulk_g2s(&tokc_w[slot], chunk, 16u, &b2[slot]);
+    const uint8_t* src = perm ? Ep + (size_t)e * row2 : E + (size_t)__ldg(prm.C2T + e) * row2;
+    bulk_g2s(ring2 + (size_t)slot * row2, src, row2, &b2[slot]);
   };
-  // certain rows: tokens, then (cluster-major copy) the first copies of each warp
-  for (int64_t i = s0 + tid; i < s1 && i < certain_rows; i += NT)
-    tok_s[i - s0] = prm.C2T[(int64_t)rank_cl[i / b - r0] * b + i % b];
+  // the first K2 slots of each warp that fall in certain clusters, one lane each
   int issued = 0;
-  if (lane == 0) fence_proxy_async_smem();  // the ring was last read by Stage 1
-  if (perm && lane == 0)
-    for (int n = 0; n < K2 && n < n2; ++n) {
-      const int64_t i = first2 + (int64_t)W * n;
-      if (i >= certain_rows) break;
-      issue_row(ring2 + (size_t)n * row2, row_src(i), row2, &b2[n]);
-      issued = n + 1;
-    }
-  // resolve the boundary bin while those copies fly
+  while (issued < K2 && issued < n2 && first2 + W * issued < certain_rows) ++issued;
+  if (lane < issued) {
+    fence_proxy_async_smem();  // the ring was last read by Stage 1 and the key copy
+    issue2(lane);
+  }
+
+  // ------------------------------------------------------------------ resolve the boundary bin
   const uint32_t bsel = topp_resolve<NT, KPT>(key, st, sm);
   {
-    const unsigned long long ex = block_scan2<NT>(__popc(bsel), 0u, sm, 1);
-    int64_t r = (int64_t)st.above + (int64_t)(ex >> 32);
+    const unsigned long long ex = block_scan2<NT>(__popc(bsel), 0u, sm, 2);
+    int r = (int)st.above + (int)(ex >> 32);
     for (uint32_t bits = bsel; bits; bits &= bits - 1, ++r)
       if (r >= r0 && r < r1) rank_cl[r - r0] = base + __ffs(bits) - 1;
   }
   const bool want_dbg = prm.dbg_sel || prm.dbg_tok || prm.dbg_logit;
   if (want_dbg) {  // ascending rank of every selected cluster, for the canonical debug order
     const uint32_t sel = st.certain | bsel;
-    const unsigned long long ex = block_scan2<NT>(__popc(sel), 0u, sm, 2);
-    int64_t a = (int64_t)(ex >> 32);
-    const unsigned long long exc = block_scan2<NT>(__popc(st.certain), __popc(bsel), sm, 0);
-    int64_t rc = (int64_t)(exc >> 32), rb = (int64_t)st.above + (int64_t)(exc & 0xFFFFFFFFull);
+    __syncthreads();
+    const unsigned long long ex = block_scan2<NT>(__popc(sel), 0u, sm, 0);
+    int a = (int)(ex >> 32);
+    __syncthreads();
+    const unsigned long long exc = block_scan2<NT>(__popc(st.certain), __popc(bsel), sm, 1);
+    int rc = (int)(exc >> 32), rb = (int)st.above + (int)(exc & 0xFFFFFFFFull);
     for (uint32_t bits = sel; bits; bits &= bits - 1, ++a) {
       const int j = __ffs(bits) - 1;
-      const int64_t r = (st.certain >> j & 1u) ? rc++ : rb++;
+      const int r = (st.certain >> j & 1u) ? rc++ : rb++;
       if (r >= r0 && r < r1) asc_of[r - r0] = (int)a;
       if (prm.dbg_sel && bid == 0) prm.dbg_sel[a] = base + j;
     }
   }
   __syncthreads();
-  for (int64_t i = (certain_rows > s0 ? certain_rows : s0) + tid; i < s1; i += NT)
-    tok_s[i - s0] = prm.C2T[(int64_t)rank_cl[i / b - r0] * b + i % b];
-  __syncthreads();
-  if (lane == 0)
-    for (int n = issued; n < K2 && n < n2; ++n)
-      issue_row(ring2 + (size_t)n * row2, row_src(first2 + (int64_t)W * n), row2, &b2[n]);
+  if (lane >= issued && lane < K2 && lane < n2) {
+    fence_proxy_async_smem();
+    issue2(lane);
+  }
 
   // ------------------------------------------------------------------ Stage 2
   unsigned long long best = 0ull;
-  for (int64_t n = 0; n < n2; ++n) {
-    const int slot = (int)(n % K2);
-    if (!mbar_wait(&b2[slot], (uint32_t)((n / K2) & 1), prm.status)) {
-      for (int64_t m = n + 1; m < n2 && m < n + K2; ++m)
+  for (int n = 0, slot = 0, phase = 0; n < n2; ++n) {
+    if (!mbar_wait(&b2[slot], (uint32_t)phase, prm.status)) {
+      for (int m = n + 1; m < n2 && m < n + K2; ++m)
         mbar_wait(&b2[m % K2], (uint32_t)((m / K2) & 1), nullptr, 50000000ull);
       break;
     }
-    const int64_t i = first2 + (int64_t)W * n;
+    const int i = first2 + W * n;
     const float z = warp_sum(row_dot_partial<ELEM>(smem_addr(ring2 + (size_t)slot * row2), hs_addr,
                                                    nch2, lane));
     __syncwarp();
     if (lane == 0) {
+      const int q = i / b;
+      const int e = rank_cl[q - r0] * b + (i - q * b);
+      const uint4 ch = tokc_w[slot];
+      const uint32_t q4i = (uint32_t)(e & 3);
+      const uint32_t tok = q4i == 0 ? ch.x : q4i == 1 ? ch.y : q4i == 2 ? ch.z : ch.w;
       if (n + K2 < n2) {
         fence_proxy_async_smem();
-        issue_row(ring2 + (size_t)slot * row2, row_src(first2 + (int64_t)W * (n + K2)), row2,
-                  &b2[slot]);
+        issue2(n + K2);
       }
-      const uint32_t tok = (uint32_t)tok_s[i - s0];
       float val = z;
       if (prm.sample)
         val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 1u, tok));
       const unsigned long long pk = pack_best(val, tok);
       best = pk > best ? pk : best;
       if (want_dbg) {
-        const int64_t ai = (int64_t)asc_of[i / b - r0] * b + i % b;
+        const int ai = asc_of[q - r0] * b + (i - q * b);
         if (prm.dbg_logit) prm.dbg_logit[ai] = z;
         if (prm.dbg_tok) prm.dbg_tok[ai] = (int32_t)tok;
       }
+    }
+    if (++slot == K2) {
+      slot = 0;
+      phase ^= 1;
     }
   }
 
@@ -293,14 +525,17 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     for (int w = 0; w < W; ++w) bb = warp_best[w] > bb ? warp_best[w] : bb;
     if (bb) atomicMax(prm.best, bb);
     __threadfence();
-    const uint32_t t = atomicAdd(prm.ticket, 1u);
-    if (t == (uint32_t)G - 1) {
-      __threadfence();
+    const unsigned long long t = atomicAdd(prm.ticket, 1ull);
+    last_s = ((t + 1) % (unsigned long long)G) == 0ull;
+  }
+  __syncthreads();
+  if (last_s) {
+    __threadfence();
+    for (int i = tid; i < kHistBins; i += NT) prm.hist[i] = 0u;
+    if (tid == 0) {
       const unsigned long long fin = atomicAdd(prm.best, 0ull);
       prm.out_tok[0] = (int32_t)best_id(fin);
-      *prm.best = 0ull;
-      *prm.ticket = 0u;
-      __threadfence();
+      atomicExch(prm.best, 0ull);
     }
   }
 }
@@ -316,29 +551,34 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
   const int G = num_sms;
   const uint32_t row2 = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
   const uint32_t row1 = int4 ? (uint32_t)(prm.d / 2) : row2;
+  if (row2 / 16 > 4u * (uint32_t)NT) return cudaErrorInvalidValue;  // h: 4 chunks per thread
   const int nch4 = int4 ? (int)(prm.d / 32) : 0;
   const int64_t P = (int64_t)prm.p * prm.b;
   const int rows1_max = (int)((prm.c + G - 1) / G);
+  if (int4 && (rows1_max * nch4 + 1) / 2 > 4 * NT) return cudaErrorInvalidValue;
   const int rows2_max = (int)((P + G - 1) / G);
   const int rmax = (int)(rows2_max / prm.b) + 2;
-  const uint32_t fixed = (NT == 256 ? head1_layout<256>(row2, int4 ? rows1_max : 0, nch4, rmax,
-                                                        rows2_max, 0)
-                                    : head1_layout<512>(row2, int4 ? rows1_max : 0, nch4, rmax,
-                                                        rows2_max, 0)).total;
+  auto fixed_for = [&](int k2) {
+    return (NT == 256 ? head1_layout<256>(row2, int4 ? rows1_max : 0, nch4, rmax, W * k2, 0)
+                      : head1_layout<512>(row2, int4 ? rows1_max : 0, nch4, rmax, W * k2, 0)).total;
+  };
   const uint32_t budget = 220u * 1024u;
-  if (fixed + (uint32_t)W * row2 > budget) return cudaErrorInvalidValue;
+  const int kcap = (1024 / 8 - 1) / W;  // barriers per stage (the last one of bars2 is the key copy's)
+  const uint32_t fixed = fixed_for(kcap);
+  if (fixed + (uint32_t)W * (row2 > row1 ? row2 : row1) > budget) return cudaErrorInvalidValue;
   const uint32_t ring_bytes = (budget - fixed) / 128u * 128u;
   auto slots = [&](uint32_t row, int64_t rows) {
     int64_t k = ring_bytes / ((uint64_t)W * row);
     const int64_t per_warp = (rows + W - 1) / W;
     if (k > per_warp) k = per_warp;
-    if (k > 1024 / 8 / W) k = 1024 / 8 / W;
+    if (k > kcap) k = kcap;
     return (int)(k < 1 ? 1 : k);
   };
+  if (ring_bytes < (uint32_t)((prm.c * 4 + 15) / 16 * 16) + 4096u) return cudaErrorInvalidValue;
   prm.k1 = slots(row1, rows1_max);
   prm.k2 = slots(row2, rows2_max);
   prm.ring_bytes = ring_bytes;
-  const size_t smem = fixed + ring_bytes;
+  const size_t smem = fixed_for(prm.k2) + ring_bytes;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
@@ -354,12 +594,12 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
   cudaError_t e = cudaSuccess;
 #define FH_H1(EL, M4, NTT, KP)                                                                     \
   do {                                                                                            \
-    static bool attr_set = false;                                                                 \
-    if (!attr_set) {                                                                              \
+    static size_t attr_bytes = 0;                                                                 \
+    if (smem > attr_bytes) {                                                                      \
       e = cudaFuncSetAttribute(k_head1<EL, M4, NTT, KP>,                                          \
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);          \
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
       if (e != cudaSuccess) return e;                                                             \
-      attr_set = true;                                                                            \
+      attr_bytes = smem;                                                                          \
     }                                                                                             \
     e = cudaLaunchKernelEx(&cfg, k_head1<EL, M4, NTT, KP>, prm);                                  \
   } while (0)

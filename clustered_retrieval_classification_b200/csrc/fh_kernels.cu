@@ -15,6 +15,9 @@
 //   k_gather, k_cand_logits, k_gumbel_keys, k_philox                                    (single steps)
 //   k_validate_c2t, k_build_perm                                                        (index load)
 //   k_mc_*                                                                              (Monte Carlo)
+#include <mutex>
+#include <unordered_map>
+
 #include "fh_kernels.cuh"
 #include "fh_device.cuh"
 #include "fh_select.cuh"
@@ -560,9 +563,19 @@ static int ring_slots(uint32_t row_bytes, uint32_t budget) {
   return k < 1 ? 1 : (k > 8 ? 8 : k);
 }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes`, remembering the limits already set so
+// that repeated launches skip the driver call.
 template <typename Kern>
 static cudaError_t set_smem(Kern kern, size_t bytes) {
-  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  static std::mutex mu;
+  static std::unordered_map<const void*, size_t> limit;
+  std::lock_guard<std::mutex> lock(mu);
+  const void* key = reinterpret_cast<const void*>(kern);
+  auto it = limit.find(key);
+  if (it != limit.end() && it->second >= bytes) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) limit[key] = bytes;
+  return e;
 }
 
 cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_sms,

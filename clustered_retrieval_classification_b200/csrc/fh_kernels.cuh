@@ -100,10 +100,10 @@ struct Head1Params {
   int sample;
   float tau;
   uint64_t seed, step;
-  uint32_t* bar_count;         // grid barrier arrival counter (zero between calls)
-  uint32_t* bar_gen;           // grid barrier generation
-  uint32_t* ticket;            // arrival counter of the final reduction (zero between calls)
-  unsigned long long* best;    // packed (key, ~token) maximum (zero between calls)
+  unsigned long long* bar_count;  // grid-barrier arrivals (grows by gridDim.x per call)
+  unsigned long long* ticket;     // final-reduction arrivals (grows by gridDim.x per call)
+  unsigned long long* best;       // packed (key, ~token) maximum (zero between calls)
+  uint32_t* hist;                 // 1024-bin key histogram (zero between calls)
   int32_t* out_tok;
   int32_t* dbg_sel;            // p or null
   int32_t* dbg_tok;            // p*b or null

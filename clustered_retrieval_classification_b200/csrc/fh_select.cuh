@@ -214,23 +214,53 @@ __device__ __forceinline__ uint32_t topp_resolve(const uint32_t (&key)[KPT], con
     return st.boundary;
   }
   if (m <= (uint32_t)kSelCandMax) {
-    // rank each boundary key against the others under (key desc, id asc)
-    for (uint32_t bits = st.boundary; bits; bits &= bits - 1) {
-      const int j = __ffs(bits) - 1;
-      const uint32_t pos = atomicAdd(&sm.cand_count, 1u);
-      sm.cand_key[pos] = __uint_as_float(key[j]);  // the image itself orders correctly as uint32
-      sm.cand_id[pos] = base + j;
+    // rank each boundary key against the others under (key desc, id asc): candidates are compacted
+    // to shared memory, every lane keeps up to kSelCandMax/32 of them in registers, and each warp
+    // ranks a share of the candidates with one comparison sweep and one warp reduction apiece.
+    // compaction: one shared atomic per warp, then predicated stores at scanned positions
+    const int lane = tid & 31;
+    const uint32_t nb = __popc(st.boundary);
+    uint32_t incl = nb;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t o = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+      incl += (lane >= off) ? o : 0u;
+    }
+    const uint32_t wtot = __shfl_sync(0xFFFFFFFFu, incl, 31);
+    uint32_t wbase = 0;
+    if (lane == 0 && wtot) wbase = atomicAdd(&sm.cand_count, wtot);
+    uint32_t pos = __shfl_sync(0xFFFFFFFFu, wbase, 0) + incl - nb;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {  // static indices keep key[] in registers
+      const uint32_t bit = st.boundary >> j & 1u;
+      if (bit) {
+        sm.cand_key[pos] = __uint_as_float(key[j]);  // the image itself orders correctly as uint32
+        sm.cand_id[pos] = base + j;
+      }
+      pos += bit;
     }
     __syncthreads();
-    for (uint32_t i = tid; i < m; i += NT) {
+    // rank each boundary key against the others under (key desc, id asc): every lane keeps up to
+    // kSelCandMax/32 candidates in registers (absent ones as image 0, which no key equals or is below),
+    // and each warp ranks a share of the candidates with one branch-free sweep and a warp reduction.
+    constexpr int kPer = kSelCandMax / 32;
+    uint32_t ck[kPer];
+    int cid[kPer];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const uint32_t q = (uint32_t)(lane + 32 * u);
+      ck[u] = q < m ? __float_as_uint(sm.cand_key[q]) : 0u;
+      cid[u] = q < m ? sm.cand_id[q] : 0x7FFFFFFF;
+    }
+    for (uint32_t i = wid; i < m; i += NT / 32) {
       const uint32_t ki = __float_as_uint(sm.cand_key[i]);
       const int ii = sm.cand_id[i];
       uint32_t rank = 0;
-      for (uint32_t q = 0; q < m; ++q) {
-        const uint32_t kq = __float_as_uint(sm.cand_key[q]);
-        rank += (kq > ki) || (kq == ki && sm.cand_id[q] < ii);
-      }
-      if (rank < st.need) atomicOr(&sm.selbits[ii >> 5], 1u << (ii & 31));
+#pragma unroll
+      for (int u = 0; u < kPer; ++u)
+        rank += (uint32_t)(ck[u] > ki) + ((uint32_t)(ck[u] == ki) & (uint32_t)(cid[u] < ii));
+      rank = __reduce_add_sync(0xFFFFFFFFu, rank);
+      if (lane == 0 && rank < st.need) atomicOr(&sm.selbits[ii >> 5], 1u << (ii & 31));
     }
     __syncthreads();
   } else {
@@ -239,10 +269,10 @@ __device__ __forceinline__ uint32_t topp_resolve(const uint32_t (&key)[KPT], con
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int i = tid; i < 256; i += NT) sm.hist[i] = 0u;
       __syncthreads();
-      for (uint32_t bits = st.boundary; bits; bits &= bits - 1) {
-        const int j = __ffs(bits) - 1;
-        if ((key[j] & pmask) == prefix) atomicAdd(&sm.hist[(key[j] >> shift) & 255u], 1u);
-      }
+#pragma unroll
+      for (int j = 0; j < KPT; ++j)
+        if ((st.boundary >> j & 1u) && (key[j] & pmask) == prefix)
+          atomicAdd(&sm.hist[(key[j] >> shift) & 255u], 1u);
       __syncthreads();
       if (wid == 0) find_boundary_bin(sm, rem);
       __syncthreads();
@@ -251,10 +281,10 @@ __device__ __forceinline__ uint32_t topp_resolve(const uint32_t (&key)[KPT], con
       rem -= sm.found_above;
     }
     uint32_t gt = 0, eq = 0;
-    for (uint32_t bits = st.boundary; bits; bits &= bits - 1) {
-      const int j = __ffs(bits) - 1;
-      gt |= (key[j] > prefix ? 1u : 0u) << j;
-      eq |= (key[j] == prefix ? 1u : 0u) << j;
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) {
+      gt |= ((st.boundary >> j & 1u) && key[j] > prefix ? 1u : 0u) << j;
+      eq |= ((st.boundary >> j & 1u) && key[j] == prefix ? 1u : 0u) << j;
     }
     // the `rem` lowest ids among the keys equal to T
     const unsigned long long ex = block_scan2<NT>(0u, __popc(eq), sm, 1);

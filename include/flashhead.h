@@ -134,12 +134,14 @@ void fh_index_free(fh_index* idx);
 
 /* Device workspace bytes one call of `op` needs at batch B, probes p, T targets per query and N
    Monte Carlo draws (T and N are ignored unless op == FH_OP_MC).  Returns 0 for invalid arguments.
-   Workspaces must be 256-byte aligned.  A workspace may be reused by consecutive calls on the same
+   Workspaces must be 256-byte aligned and zero-filled before their first use (the calls leave
+   them ready for the next call).  A workspace may be reused by consecutive calls on the same
    stream; calls that overlap in time need separate workspaces. */
 size_t fh_workspace_bytes(const fh_index* idx, int op, int B, int p, int T, int64_t N);
 
 /* Read and clear the status word of a workspace (synchronises `stream`).  Returns FH_OK, or the
-   device-side error a previous call recorded there (FH_ERR_TIMEOUT, FH_ERR_INDEX). */
+   device-side error a previous call recorded there (FH_ERR_TIMEOUT, FH_ERR_INDEX); after an error
+   the workspace's control block is zeroed again so that it can be reused. */
 fh_status fh_ws_status(void* ws, fh_stream stream);
 
 /* Thread-local description of the last error returned on this thread ("" if none). */

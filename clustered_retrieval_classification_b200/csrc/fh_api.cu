@@ -222,6 +222,9 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
 
 }  // namespace
 
+// Used by fh_static.cu to report its own errors through fh_last_error().
+fh_status fh_internal_set_error(fh_status st, const char* msg) { return fail(st, "%s", msg); }
+
 extern "C" {
 
 const char* fh_last_error(void) { return g_err; }

@@ -64,6 +64,7 @@ SIGNATURES = {
     "fh_gather_candidates": (_i, [_p, _p, _i, _i, _p, _p]),
     "fh_candidate_logits": (_i, [_p, _p, _i, _p, _i64, _p, _p]),
     "fh_philox_u32": (_i, [_u64, _u64, _u32, _u32, _i64, _p, _p]),
+    "fh_head_greedy_static": (_i, [_p, _p, _i, _p, _p]),
 }
 
 
@@ -278,6 +279,16 @@ def candidate_logits(index: Index, H, cand, out=None, stream=None):
 def philox_u32(seed, step, row, rng_stream, n, device="cuda", stream=None):
     out = torch.empty(n, dtype=torch.int32, device=device)
     _check(load().fh_philox_u32(seed, step, row, rng_stream, n, _ptr(out), _stream(stream)))
+    return out
+
+
+def head_greedy_static(index: Index, H, p, out=None, stream=None):
+    """Batch-1 greedy head that uses the library's static device scratch instead of a workspace."""
+    _need(H, "H")
+    if H.shape[0] != 1:
+        raise ValueError("head_greedy_static takes one query")
+    out = out if out is not None else torch.empty(1, dtype=torch.int32, device=H.device)
+    _check(load().fh_head_greedy_static(index.handle, _ptr(H), p, _ptr(out), _stream(stream)))
     return out
 
 

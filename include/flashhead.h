@@ -217,6 +217,24 @@ fh_status fh_candidate_logits(const fh_index* idx, const void* H, int B, const i
 fh_status fh_philox_u32(uint64_t seed, uint64_t step, uint32_t row, uint32_t rng_stream, int64_t n,
                         uint32_t* out, fh_stream stream);
 
+/* ---------------------------------------------------------------- allocation-free call ----- */
+/* No counterpart in the pages: an integration convenience of this library.
+   Greedy head at batch 1 (the same computation and kernels as fh_head_greedy with B = 1) for callers
+   that can neither allocate device memory nor lend a workspace — for example code inside a host
+   framework that owns the whole device heap, or a decode loop that cannot afford cudaMalloc's
+   implicit device synchronisation.  The call's scratch lives in a file-scope device array of
+   FH_STATIC_SCRATCH_BYTES bytes that every GPU loading the library keeps until process exit.
+   H: device, 1 x d; out_tok: device, 1 int32.  Allocates nothing: it calls no cudaMalloc/cudaFree
+   and no allocating library routine; it clears the part of the array it uses with cudaMemsetAsync.
+   The first call on a device looks up the array's device address (cudaGetSymbolAddress, with that
+   device current); make that first call before any stream capture.  Calls share the one array, so
+   calls that overlap in time on the GPU (on different streams) race; serialise them.
+   Returns FH_ERR_WORKSPACE with a message when the index needs more scratch than the array holds
+   (roughly c*4 + 8 KiB bytes, so c up to about 30,000 clusters). */
+enum { FH_STATIC_SCRATCH_BYTES = 131072 };
+fh_status fh_head_greedy_static(const fh_index* idx, const void* H, int p, int32_t* out_tok,
+                                fh_stream stream);
+
 #ifdef __cplusplus
 }
 #endif

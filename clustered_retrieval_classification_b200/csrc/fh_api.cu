@@ -34,6 +34,7 @@ fh_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 constexpr size_t kHeaderBytes = 1024 + 4096;  // control words, then the score histogram
+constexpr size_t kGenOffset = 536;             // batch-1 head: tag of the last completed call
 constexpr size_t kAlign = 256;
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -42,7 +43,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Workspace regions of one call; offsets from the workspace base.
 struct Layout {
-  size_t keys = 0, sel = 0, part = 0, z = 0, s = 0, zmax = 0, Z = 0, cluster_of = 0, per_draw = 0;
+  size_t keys = 0, sel = 0, part = 0, list = 0, bnd = 0, z = 0, s = 0, zmax = 0, Z = 0,
+         cluster_of = 0, per_draw = 0;
   size_t total = 0;
 };
 
@@ -61,6 +63,10 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
     L.keys = take((size_t)B * D.c * 4);
     L.sel = take((size_t)B * p * 4);
     L.part = take((size_t)G * B * 8);
+    if (B == 1) {  // the persistent batch-1 kernel's tagged selection entries
+      L.list = take((size_t)p * 8);
+      L.bnd = take((size_t)fh::kHead1BndMax * 16);
+    }
   } else if (op == FH_OP_DENSE) {
     const int G = fh::stage2_blocks(D.v, B, idx->num_sms);
     L.part = take((size_t)G * B * 8);
@@ -89,10 +95,11 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 // Workspace header (first kHeaderBytes): status word at 0, per-query tickets at 16 (64 x 4 bytes),
 // the persistent head's 64-bit grid-barrier arrival counter at 512, its 64-bit final-reduction
-// ticket at 520 and its packed arg-max at 528; bytes [1024, 5120) hold its 1024-bin score histogram
-// in every layout, so no other call ever writes there.  The two counters only grow (each call adds
-// one grid's worth); the arg-max and the histogram return to zero at the end of every call.  A new
-// workspace must start zeroed (fh_ws_status re-zeroes the header after a device-side error).
+// ticket at 520, its packed arg-max at 528 and its call generation at 536 (the tag of the last
+// completed call); bytes [1024, 5120) hold its 1024-bin score histogram in every layout, so no other
+// call ever writes there.  The two counters and the generation only grow; the arg-max and the
+// histogram return to zero at the end of every call.  A new workspace must start zeroed
+// (fh_ws_status re-zeroes the header after a device-side error, keeping the generation moving).
 uint32_t* status_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16); }
 uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
@@ -163,6 +170,9 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     h.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, 520));
     h.best = reinterpret_cast<unsigned long long*>(word_at(ws, 528));
     h.hist = word_at(ws, 1024);
+    h.gen = word_at(ws, kGenOffset);
+    h.order = reinterpret_cast<unsigned long long*>(base + L.list);
+    h.bnd = reinterpret_cast<unsigned long long*>(base + L.bnd);
     h.out_tok = out_tok;
     h.dbg_sel = dbg ? dbg->sel : nullptr;
     h.dbg_tok = dbg ? dbg->cand_tok : nullptr;
@@ -312,7 +322,15 @@ fh_status fh_ws_status(void* ws, fh_stream stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "status read");
   if (status != 0) {
-    e = cudaMemsetAsync(ws, 0, kHeaderBytes, st);
+    // Zero the control block, but move the call generation past every tag the failed call may have
+    // written, so that no entry it left behind is taken for a later call's.
+    uint32_t gen = 0;
+    e = cudaMemcpyAsync(&gen, static_cast<char*>(ws) + kGenOffset, 4, cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    gen += 1u;
+    if (e == cudaSuccess) e = cudaMemsetAsync(ws, 0, kHeaderBytes, st);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<char*>(ws) + kGenOffset, &gen, 4, cudaMemcpyHostToDevice, st);
     if (e == cudaSuccess) e = cudaStreamSynchronize(st);
     if (e != cudaSuccess) return cuda_fail(e, "status clear");
     if (status == FH_ERR_TIMEOUT) return fail(FH_ERR_TIMEOUT, "a device-side wait timed out");

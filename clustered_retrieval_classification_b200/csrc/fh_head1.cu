@@ -33,9 +33,10 @@
 namespace fh {
 
 constexpr int kHistBins = 1024;
+static_assert(kHead1BndMax == kSelCandMax, "boundary entries = ranked candidates");
 
 struct Head1Layout {
-  uint32_t bars1, bars2, hs, sc, sel, hist, rank_cl, asc, tokc, ring, total;
+  uint32_t bars1, bars2, hs, sc, sel, hist, ownk, ownp, rank_cl, asc, tokc, ring, total;
 };
 
 __host__ __device__ inline uint32_t h1_align(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -43,16 +44,20 @@ __host__ __device__ inline uint32_t h1_align(uint32_t x, uint32_t a) { return (x
 template <int NT>
 __host__ __device__ inline Head1Layout head1_layout(uint32_t row2, int rows1_max, int nch4, int rmax,
                                                     int slots2, uint32_t ring_bytes) {
+  // rows1_max: Stage-1 rows of the largest block (its own keys are kept); nch4: INT4 groups per row
+  const int sc_rows = nch4 ? rows1_max : 0;
   Head1Layout L;
   L.bars1 = 0;
   L.bars2 = 1024;
   L.hs = 2048;
   L.sc = h1_align(L.hs + row2, 128);
-  L.sel = h1_align(L.sc + (uint32_t)rows1_max * nch4 * 2u + 4u, 128);
+  L.sel = h1_align(L.sc + (uint32_t)sc_rows * nch4 * 2u + 4u, 128);
   L.hist = h1_align(L.sel + (uint32_t)sizeof(SelectSmem<NT>), 16);
-  L.rank_cl = h1_align(L.hist + kHistBins * 4u, 16);
-  L.asc = h1_align(L.rank_cl + (uint32_t)rmax * 4u, 16);
-  L.tokc = h1_align(L.asc + (uint32_t)rmax * 4u, 16);
+  L.ownk = h1_align(L.hist + kHistBins * 4u, 16);
+  L.ownp = h1_align(L.ownk + (uint32_t)rows1_max * 4u, 16);
+  L.rank_cl = h1_align(L.ownp + (uint32_t)rows1_max * 4u, 16);
+  L.asc = h1_align(L.rank_cl + 2u * (uint32_t)rmax * 4u, 16);
+  L.tokc = h1_align(L.asc + 2u * (uint32_t)rmax * 4u, 16);
   L.ring = h1_align(L.tokc + (uint32_t)slots2 * 16u, 128);
   L.total = L.ring + ring_bytes;
   return L;
@@ -151,6 +156,65 @@ __device__ __forceinline__ bool grid_barrier(unsigned long long* count, uint32_t
   return !*abort_s;
 }
 
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Poll a 64-bit word until its upper half equals `tag`, then return it (payload in the lower half).
+// Bounded: after 0.5 s it records a timeout, clears `ok` and returns 0.
+__device__ __forceinline__ unsigned long long poll_tagged(const unsigned long long* p, uint32_t tag,
+                                                          uint32_t* status, bool& ok) {
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    unsigned long long v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    if ((uint32_t)(v >> 32) == tag) return v;
+    if ((it & 63u) == 0 && global_timer_ns() - t0 > 500000000ull) {
+      set_status(status, kStatusTimeout);
+      ok = false;
+      return 0ull;
+    }
+  }
+}
+
+// Rank the m (<= 32*KP) boundary candidates under (key desc, id asc) and write the ids of the `need`
+// best into bsel_rank in rank order.  Every lane keeps KP candidates in registers (absent ones as
+// image 0, below every key); each warp ranks four candidates per pass, branch-free.
+template <int KP>
+__device__ __forceinline__ void rank_boundary(const float* cand_key, const int* cand_id, uint32_t m,
+                                              uint32_t need, int* bsel_rank, int lane, int warp,
+                                              int nwarps) {
+  uint32_t ck[KP];
+  int cid[KP];
+#pragma unroll
+  for (int u = 0; u < KP; ++u) {
+    const uint32_t q = (uint32_t)(lane + 32 * u);
+    ck[u] = q < m ? __float_as_uint(cand_key[q]) : 0u;
+    cid[u] = q < m ? cand_id[q] : 0x7FFFFFFF;
+  }
+  for (uint32_t i0 = (uint32_t)warp * 4u; i0 < m; i0 += (uint32_t)nwarps * 4u) {
+    uint32_t ki[4], rk[4];
+    int ii[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t i = i0 + t;
+      ki[t] = i < m ? __float_as_uint(cand_key[i]) : 0xFFFFFFFFu;
+      ii[t] = i < m ? cand_id[i] : 0;
+      rk[t] = 0u;
+    }
+#pragma unroll
+    for (int u = 0; u < KP; ++u)
+#pragma unroll
+      for (int t = 0; t < 4; ++t)
+        rk[t] += (uint32_t)(ck[u] > ki[t]) + ((uint32_t)(ck[u] == ki[t]) & (uint32_t)(cid[u] < ii[t]));
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t r = __reduce_add_sync(0xFFFFFFFFu, rk[t]);
+      if (lane == 0 && i0 + t < m && r < need) bsel_rank[r] = ii[t];
+    }
+  }
+}
+
 template <int ELEM, int INT4_MCH, int NT, int KPT>
 __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   extern __shared__ __align__(128) uint8_t smem[];
@@ -158,7 +222,7 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   __shared__ unsigned long long warp_best[W];
   __shared__ float red_s[W];
   __shared__ bool abort_s, last_s;
-  __shared__ uint32_t dstar_s, above_s, total_s, edge_lo_s, edge_hi_s;
+  __shared__ uint32_t dstar_s, above_s, total_s, edge_lo_s, edge_hi_s, m_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x, bid = blockIdx.x;
   const int64_t c = prm.c, d = prm.d;
@@ -172,14 +236,15 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   const int rows2_max = (int)((P + G - 1) / G);
   const int rmax = (int)(rows2_max / b) + 2;
   const int K1 = prm.k1, K2 = prm.k2;
-  const Head1Layout L = head1_layout<NT>(row2, INT4_MCH ? rows1_max : 0, nch4, rmax, W * K2,
-                                         prm.ring_bytes);
+  const Head1Layout L = head1_layout<NT>(row2, rows1_max, nch4, rmax, W * K2, prm.ring_bytes);
   uint64_t* bars1 = reinterpret_cast<uint64_t*>(smem + L.bars1);
   uint64_t* bars2 = reinterpret_cast<uint64_t*>(smem + L.bars2);
   uint8_t* hs = smem + L.hs;
   uint16_t* sc_s = reinterpret_cast<uint16_t*>(smem + L.sc);
   SelectSmem<NT>& sm = *reinterpret_cast<SelectSmem<NT>*>(smem + L.sel);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L.hist);
+  float* own_keys = reinterpret_cast<float*>(smem + L.ownk);
+  uint32_t* own_pos = reinterpret_cast<uint32_t*>(smem + L.ownp);
   int* rank_cl = reinterpret_cast<int*>(smem + L.rank_cl);
   int* asc_of = reinterpret_cast<int*>(smem + L.asc);
   uint4* tokc = reinterpret_cast<uint4*>(smem + L.tokc);
@@ -193,6 +258,7 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     if (ch < nch2) hv[u] = __ldg(reinterpret_cast<const uint4*>(prm.H) + ch);
   }
   const int64_t lo1 = c * bid / G, hi1 = c * (bid + 1) / G;
+  const uint32_t tag = __ldcg(prm.gen) + 1u;  // this call's tag on its selection entries
   uint32_t scv[4];  // INT4: this block's group scales, two per 32-bit word
   const int nsc = INT4_MCH ? (int)((hi1 - lo1) * nch4) : 0;
   const int sc_words = (nsc + 1) / 2;
@@ -300,7 +366,8 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       if (prm.sample)
         key = s / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 0u, (uint32_t)k));
       prm.keys[k] = key;
-      atomicAdd(&hist_s[bin(key_float(float_key(key)))], 1u);
+      own_keys[k - (int)lo1] = key;
+      own_pos[k - (int)lo1] = atomicAdd(&hist_s[bin(key_float(float_key(key)))], 1u);
     }
     if (++slot == K1) {
       slot = 0;
@@ -308,42 +375,25 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     }
   }
   __syncthreads();
-  for (int i = tid; i < kHistBins; i += NT)
-    if (hist_s[i]) atomicAdd(&prm.hist[i], hist_s[i]);
+  // Add the block's counts to the global histogram; each add returns the block's first position in
+  // that bin, so every key gets a distinct position among the keys of its bin.
+  for (int i = tid; i < kHistBins; i += NT) {
+    const uint32_t n = hist_s[i];
+    if (n) hist_s[i] = atomicAdd(&prm.hist[i], n);
+  }
 
   // ------------------------------------------------------------------ grid barrier
   if (!grid_barrier(prm.bar_count, (uint32_t)G, prm.status, &abort_s)) return;
 
   // ------------------------------------------------------------------ boundary bin
-  // The keys written by every block and the summed histogram come in with one bulk copy into the
-  // ring, which is idle between the stages (the workspace pads the keys to a multiple of 16 bytes).
-  const uint32_t keys_bytes = (uint32_t)((c * 4 + 15) / 16 * 16);
-  float* keys_s = reinterpret_cast<float*>(ring);
-  uint32_t* histg_s = reinterpret_cast<uint32_t*>(ring + keys_bytes);
+  // The summed histogram comes in with one bulk copy into the ring, idle between the stages.
+  uint32_t* histg_s = reinterpret_cast<uint32_t*>(ring);
   if (tid == 0) {
-    asm volatile("fence.proxy.async;" ::: "memory");  // other blocks' keys, seen via the barrier
-    mbar_arrive_expect_tx(bar_keys, keys_bytes + kHistBins * 4u);
-    bulk_g2s(keys_s, prm.keys, keys_bytes, bar_keys);
+    asm volatile("fence.proxy.async;" ::: "memory");  // written by other blocks, seen via the barrier
+    mbar_arrive_expect_tx(bar_keys, kHistBins * 4u);
     bulk_g2s(histg_s, prm.hist, kHistBins * 4u, bar_keys);
   }
   if (!mbar_wait(bar_keys, 0u, prm.status)) return;
-  uint32_t key[KPT];
-  {
-    const int kb = tid * KPT;
-#pragma unroll
-    for (int j = 0; j < KPT; j += 4) {
-      if (kb + j + 4 <= c) {
-        const float4 f = *reinterpret_cast<const float4*>(keys_s + kb + j);
-        key[j] = float_key(f.x);
-        key[j + 1] = float_key(f.y);
-        key[j + 2] = float_key(f.z);
-        key[j + 3] = float_key(f.w);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) key[j + e] = (kb + j + e < c) ? float_key(keys_s[kb + j + e]) : 0u;
-      }
-    }
-  }
   constexpr int HPT = kHistBins / NT;  // histogram bins per thread
   uint32_t hb[HPT];
   uint32_t htot = 0;
@@ -367,9 +417,11 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     uint32_t cum = total_s - before - htot;  // keys in bins above this thread's bins
 #pragma unroll
     for (int u = HPT - 1; u >= 0; --u) {
+      histg_s[tid * HPT + u] = cum;  // from here on: keys in bins above bin tid*HPT+u
       if (!all && cum < (uint32_t)prm.p && cum + hb[u] >= (uint32_t)prm.p) {
         dstar_s = (uint32_t)(tid * HPT + u);
         above_s = cum;
+        m_s = hb[u];
       }
       cum += hb[u];
     }
@@ -379,12 +431,155 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       return;
     }
   }
-  SelState st;
-  {
-    const uint32_t dstar = all ? 0u : dstar_s;
-    st.above = all ? (uint32_t)c : above_s;
-    st.need = (uint32_t)prm.p - st.above;
-    // key images at the lower edges of bins d* and d*+1 (warps 0 and 1 search them)
+  const uint32_t dstar = all ? 0u : dstar_s;
+  const uint32_t above_n = all ? (uint32_t)c : above_s;
+  const uint32_t need = (uint32_t)prm.p - above_n;
+  const uint32_t m_total = all ? 0u : m_s;
+  // Stage-2 rows of this block: its share of the certain rows [c0, c1) and of the boundary rows
+  // [d0, d1) (global rows in list order: rank r = row / b, certain ranks first).  Local row l is
+  // c0 + l below nc and d0 + (l - nc) above, so certain rows stream while the boundary is resolved.
+  const int CR = (int)above_n * b, BR = (int)need * b;
+  const int c0 = (int)((int64_t)CR * bid / G), c1 = (int)((int64_t)CR * (bid + 1) / G);
+  const int d0 = CR + (int)((int64_t)BR * bid / G), d1 = CR + (int)((int64_t)BR * (bid + 1) / G);
+  const int nc = c1 - c0, nr = nc + (d1 - d0);
+  const int rc0 = c0 / b, rc1 = (c1 + b - 1) / b;  // certain ranks touched
+  const int rb0 = d0 / b, rb1 = (d1 + b - 1) / b;  // boundary ranks touched
+  int* rk_c = rank_cl;
+  int* rk_b = rank_cl + rmax;
+  int* asc_c = asc_of;
+  int* asc_b = asc_of + rmax;
+  const bool want_dbg = prm.dbg_sel || prm.dbg_tok || prm.dbg_logit;
+
+  const uint8_t* E = static_cast<const uint8_t*>(prm.E);
+  const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
+  const bool perm = Ep != nullptr;
+  const int n2 = (warp < nr) ? (nr - warp + W - 1) / W : 0;
+  uint8_t* ring2 = ring + (size_t)warp * K2 * row2;
+  uint64_t* b2 = bars2 + warp * K2;
+  uint4* tokc_w = tokc + warp * K2;
+  auto global_row = [&](int l) { return l < nc ? c0 + l : d0 + (l - nc); };
+  auto row_e = [&](int g) {  // flat C2T index (= row of the cluster-major copy) of global row g
+    const int r = g / b;
+    const int cl = (r < (int)above_n) ? rk_c[r - rc0] : rk_b[r - rb0];
+    return cl * b + (g - r * b);
+  };
+  auto issue2 = [&](int n) {
+    const int slot = n % K2;
+    const int e = row_e(global_row(warp + W * n));
+    const int32_t* chunk = prm.C2T + (e & ~3);  // 16-byte chunk holding the token id
+    mbar_arrive_expect_tx(&b2[slot], row2 + 16u);
+    bulk_g2s(&tokc_w[slot], chunk, 16u, &b2[slot]);
+    const uint8_t* src = perm ? Ep + (size_t)e * row2 : E + (size_t)__ldg(prm.C2T + e) * row2;
+    bulk_g2s(ring2 + (size_t)slot * row2, src, row2, &b2[slot]);
+  };
+  // the first K2 slots of each warp that hold certain rows
+  int issued = 0;
+  while (issued < K2 && issued < n2 && warp + W * issued < nc) ++issued;
+  const bool fast = all || m_total <= (uint32_t)kSelCandMax;
+
+  if (fast) {
+    // ---------------------------------------------------------------- distributed selection
+    // A cluster's rank in the Stage-2 list is (keys in higher bins) + (its position in its bin), known
+    // to the block that scored it as soon as the histogram is: each block writes the ids of its
+    // certain clusters at their ranks, and the (key, id) of its boundary-bin clusters at their
+    // positions, each as one 64-bit word tagged with the call's tag.  Every block then polls only the
+    // words its rows need (and the boundary bin, which it ranks itself): no counters, no fences.
+    const int nk = (int)(hi1 - lo1);
+    if (tid < nk) {
+      const uint32_t img = float_key(own_keys[tid]);
+      const uint32_t dg = bin(key_float(img));
+      const uint32_t pos = hist_s[dg] + own_pos[tid];
+      const unsigned long long tg = (unsigned long long)tag << 32;
+      const uint32_t id = (uint32_t)(lo1 + tid);
+      if (all || dg > dstar) {
+        st_relaxed_u64(prm.order + histg_s[dg] + pos, tg | id);
+      } else if (dg == dstar) {
+        st_relaxed_u64(prm.bnd + 2 * pos, tg | img);
+        st_relaxed_u64(prm.bnd + 2 * pos + 1, tg | id);
+      }
+      // Whichever block streams them, the rows of this block's selected and boundary clusters start
+      // moving into L2 now (cluster-major copy: one range per cluster).
+      if (perm && (all || dg >= dstar)) bulk_prefetch_l2(Ep + (size_t)id * b * row2, (uint32_t)b * row2);
+    }
+    const bool rank_here = need > 0u && (d1 > d0 || want_dbg);
+    bool ok = true;
+    for (int r = rc0 + tid; r < rc1; r += NT)
+      rk_c[r - rc0] = (int)(uint32_t)poll_tagged(prm.order + r, tag, prm.status, ok);
+    if (rank_here) {
+      for (uint32_t q = tid; q < m_total; q += NT) {
+        sm.cand_key[q] = __uint_as_float((uint32_t)poll_tagged(prm.bnd + 2 * q, tag, prm.status, ok));
+        sm.cand_id[q] = (int)(uint32_t)poll_tagged(prm.bnd + 2 * q + 1, tag, prm.status, ok);
+      }
+    }
+    if (want_dbg)  // the debug outputs read the whole certain list below
+      for (uint32_t q = tid; q < above_n; q += NT) poll_tagged(prm.order + q, tag, prm.status, ok);
+    if (!__syncthreads_and(ok)) return;  // a wait gave up (status set); no copy is in flight yet
+    if (lane < issued) {
+      fence_proxy_async_smem();  // the ring was last read by Stage 1 and the histogram copy
+      issue2(lane);
+    }
+    // boundary ranks: every block with boundary rows ranks the boundary bin while its certain rows fly
+    int* bsel_rank = reinterpret_cast<int*>(sm.selbits);
+    if (rank_here) {
+      if (m_total <= 128u)
+        rank_boundary<4>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
+      else
+        rank_boundary<kSelCandMax / 32>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
+      __syncthreads();
+      for (int r = rb0 + tid; r < rb1; r += NT) rk_b[r - rb0] = bsel_rank[r - (int)above_n];
+      __syncthreads();
+    }
+    if (want_dbg) {
+      // canonical (ascending) positions: count the selected clusters below each of this block's
+      auto cert_at = [&](uint32_t q) { return (int)(uint32_t)__ldcg(prm.order + q); };
+      const int ncr = rc1 - rc0, nbr = rb1 - rb0;
+      for (int t = warp; t < ncr + nbr; t += W) {
+        const int x = t < ncr ? rk_c[t] : rk_b[t - ncr];
+        uint32_t cnt = 0;
+        for (uint32_t q = lane; q < above_n; q += 32) cnt += (uint32_t)(cert_at(q) < x);
+        for (uint32_t q = lane; q < need; q += 32) cnt += (uint32_t)(bsel_rank[q] < x);
+        cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
+        if (lane == 0) {
+          if (t < ncr) asc_c[t] = (int)cnt;
+          else asc_b[t - ncr] = (int)cnt;
+        }
+      }
+      if (prm.dbg_sel && bid == 0) {
+        for (uint32_t q = tid; q < (uint32_t)prm.p; q += NT) {
+          const int x = q < above_n ? cert_at(q) : bsel_rank[q - above_n];
+          uint32_t cnt = 0;
+          for (uint32_t y = 0; y < above_n; ++y) cnt += (uint32_t)(cert_at(y) < x);
+          for (uint32_t y = 0; y < need; ++y) cnt += (uint32_t)(bsel_rank[y] < x);
+          prm.dbg_sel[cnt] = x;
+        }
+      }
+      __syncthreads();
+    }
+    if (lane >= issued && lane < K2 && lane < n2) {
+      fence_proxy_async_smem();
+      issue2(lane);
+    }
+  } else {
+    // ---------------------------------------------------------------- full selection (crowded bin)
+    // More than kSelCandMax keys share the boundary bin: every block loads all keys and selects
+    // with the block-wide selector (exact radix passes on the boundary bin).
+    const uint32_t keys_bytes = (uint32_t)((c * 4 + 15) / 16 * 16);
+    float* keys_s = reinterpret_cast<float*>(ring + kHistBins * 4);
+    __syncthreads();
+    if (tid == 0) {
+      mbar_arrive_expect_tx(bar_keys, keys_bytes);
+      bulk_g2s(keys_s, prm.keys, keys_bytes, bar_keys);
+    }
+    if (!mbar_wait(bar_keys, 1u, prm.status)) return;
+    uint32_t key[KPT];
+    {
+      const int kb = tid * KPT;
+#pragma unroll
+      for (int j = 0; j < KPT; ++j) key[j] = (kb + j < c) ? float_key(keys_s[kb + j]) : 0u;
+    }
+    SelState st;
+    st.above = above_n;
+    st.need = need;
     if (warp == 0) {
       const uint32_t e = (dstar == 0u) ? 1u : bin_edge(bin, dstar);
       if (lane == 0) edge_lo_s = e;
@@ -396,88 +591,47 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     const uint32_t elo = edge_lo_s, ehi = edge_hi_s;
     st.certain = 0u;
     st.boundary = 0u;
-    const uint32_t all_u = all ? 1u : 0u;
 #pragma unroll
-    for (int j = 0; j < KPT; ++j) {  // branch-free: plain 0/1 arithmetic per key
+    for (int j = 0; j < KPT; ++j) {
       const uint32_t kj = key[j];
       const uint32_t real = (uint32_t)(kj != 0u);
-      const uint32_t above = (uint32_t)(kj >= ehi);
-      const uint32_t inbin = (uint32_t)(kj >= elo) & (above ^ 1u);
-      st.certain |= (real & (all_u | above)) << j;
-      st.boundary |= (real & (all_u ^ 1u) & inbin) << j;
+      const uint32_t abv = (uint32_t)(kj >= ehi);
+      st.certain |= (real & abv) << j;
+      st.boundary |= (real & (uint32_t)(kj >= elo) & (abv ^ 1u)) << j;
     }
-  }
-  const int base = tid * KPT;
-  const int s0 = (int)((int64_t)P * bid / G), s1 = (int)((int64_t)P * (bid + 1) / G);
-  const int r0 = s0 / b, r1 = (s1 + b - 1) / b;  // ranks this block touches
-  const int certain_rows = (int)st.above * b;
-  {
-    const unsigned long long ex = block_scan2<NT>(__popc(st.certain), 0u, sm, 1);
-    int r = (int)(ex >> 32);
-    for (uint32_t bits = st.certain; bits; bits &= bits - 1, ++r)
-      if (r >= r0 && r < r1) rank_cl[r - r0] = base + __ffs(bits) - 1;
-  }
-  __syncthreads();
-
-  // ------------------------------------------------------------------ Stage-2 copies of certain rows
-  const uint8_t* E = static_cast<const uint8_t*>(prm.E);
-  const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
-  const bool perm = Ep != nullptr;
-  const int first2 = s0 + warp;
-  const int n2 = (first2 < s1) ? (s1 - first2 + W - 1) / W : 0;
-  uint8_t* ring2 = ring + (size_t)warp * K2 * row2;
-  uint64_t* b2 = bars2 + warp * K2;
-  uint4* tokc_w = tokc + warp * K2;
-  // slot n of this warp: row i = first2 + W*n of cluster rank_cl[i/b - r0], row i % b within it
-  auto issue2 = [&](int n) {
-    const int slot = n % K2;
-    const int i = first2 + W * n;
-    const int q = i / b;
-    const int e = rank_cl[q - r0] * b + (i - q * b);  // flat C2T index = row of the cluster-major copy
-    const int32_t* chunk = prm.C2T + (e & ~3);        // 16-byte chunk holding the token id
-    mbar_arrive_expect_tx(&b2[slot], row2 + 16u);
-    bulk_g2s(&tokc_w[slot], chunk, 16u, &b2[slot]);
-    const uint8_t* src = perm ? Ep + (size_t)e * row2 : E + (size_t)__ldg(prm.C2T + e) * row2;
-    bulk_g2s(ring2 + (size_t)slot * row2, src, row2, &b2[slot]);
-  };
-  // the first K2 slots of each warp that fall in certain clusters, one lane each
-  int issued = 0;
-  while (issued < K2 && issued < n2 && first2 + W * issued < certain_rows) ++issued;
-  if (lane < issued) {
-    fence_proxy_async_smem();  // the ring was last read by Stage 1 and the key copy
-    issue2(lane);
-  }
-
-  // ------------------------------------------------------------------ resolve the boundary bin
-  const uint32_t bsel = topp_resolve<NT, KPT>(key, st, sm);
-  {
-    const unsigned long long ex = block_scan2<NT>(__popc(bsel), 0u, sm, 2);
-    int r = (int)st.above + (int)(ex >> 32);
-    for (uint32_t bits = bsel; bits; bits &= bits - 1, ++r)
-      if (r >= r0 && r < r1) rank_cl[r - r0] = base + __ffs(bits) - 1;
-  }
-  const bool want_dbg = prm.dbg_sel || prm.dbg_tok || prm.dbg_logit;
-  if (want_dbg) {  // ascending rank of every selected cluster, for the canonical debug order
+    const int base = tid * KPT;
+    const uint32_t bsel = topp_resolve<NT, KPT>(key, st, sm);
     const uint32_t sel = st.certain | bsel;
+    {
+      const unsigned long long exc = block_scan2<NT>(__popc(st.certain), __popc(bsel), sm, 1);
+      const unsigned long long exa = block_scan2<NT>(__popc(sel), 0u, sm, 2);
+      int rc = (int)(exc >> 32), rb = (int)above_n + (int)(exc & 0xFFFFFFFFull);
+      int a = (int)(exa >> 32);
+      for (uint32_t bits = sel; bits; bits &= bits - 1, ++a) {
+        const int j = __ffs(bits) - 1;
+        if (st.certain >> j & 1u) {
+          if (rc >= rc0 && rc < rc1) {
+            rk_c[rc - rc0] = base + j;
+            asc_c[rc - rc0] = a;
+          }
+          ++rc;
+        } else {
+          if (rb >= rb0 && rb < rb1) {
+            rk_b[rb - rb0] = base + j;
+            asc_b[rb - rb0] = a;
+          }
+          ++rb;
+        }
+        if (prm.dbg_sel && bid == 0) prm.dbg_sel[a] = base + j;
+      }
+    }
     __syncthreads();
-    const unsigned long long ex = block_scan2<NT>(__popc(sel), 0u, sm, 0);
-    int a = (int)(ex >> 32);
-    __syncthreads();
-    const unsigned long long exc = block_scan2<NT>(__popc(st.certain), __popc(bsel), sm, 1);
-    int rc = (int)(exc >> 32), rb = (int)st.above + (int)(exc & 0xFFFFFFFFull);
-    for (uint32_t bits = sel; bits; bits &= bits - 1, ++a) {
-      const int j = __ffs(bits) - 1;
-      const int r = (st.certain >> j & 1u) ? rc++ : rb++;
-      if (r >= r0 && r < r1) asc_of[r - r0] = (int)a;
-      if (prm.dbg_sel && bid == 0) prm.dbg_sel[a] = base + j;
+    if (lane < K2 && lane < n2) {
+      fence_proxy_async_smem();  // the ring was last read by the key copy
+      issue2(lane);
     }
   }
   __syncthreads();
-  if (lane >= issued && lane < K2 && lane < n2) {
-    fence_proxy_async_smem();
-    issue2(lane);
-  }
-
   // ------------------------------------------------------------------ Stage 2
   unsigned long long best = 0ull;
   for (int n = 0, slot = 0, phase = 0; n < n2; ++n) {
@@ -486,13 +640,13 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
         mbar_wait(&b2[m % K2], (uint32_t)((m / K2) & 1), nullptr, 50000000ull);
       break;
     }
-    const int i = first2 + W * n;
+    const int g = global_row(warp + W * n);
     const float z = warp_sum(row_dot_partial<ELEM>(smem_addr(ring2 + (size_t)slot * row2), hs_addr,
                                                    nch2, lane));
     __syncwarp();
     if (lane == 0) {
-      const int q = i / b;
-      const int e = rank_cl[q - r0] * b + (i - q * b);
+      const int q = g / b;
+      const int e = row_e(g);
       const uint4 ch = tokc_w[slot];
       const uint32_t q4i = (uint32_t)(e & 3);
       const uint32_t tok = q4i == 0 ? ch.x : q4i == 1 ? ch.y : q4i == 2 ? ch.z : ch.w;
@@ -506,7 +660,7 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       const unsigned long long pk = pack_best(val, tok);
       best = pk > best ? pk : best;
       if (want_dbg) {
-        const int ai = asc_of[q - r0] * b + (i - q * b);
+        const int ai = ((q < (int)above_n) ? asc_c[q - rc0] : asc_b[q - rb0]) * b + (g - q * b);
         if (prm.dbg_logit) prm.dbg_logit[ai] = z;
         if (prm.dbg_tok) prm.dbg_tok[ai] = (int32_t)tok;
       }
@@ -532,6 +686,11 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   if (last_s) {
     __threadfence();
     for (int i = tid; i < kHistBins; i += NT) prm.hist[i] = 0u;
+    if (fast) {  // the next call starts from zeroed entries (the tags already tell calls apart)
+      for (uint32_t q = tid; q < above_n; q += NT) prm.order[q] = 0ull;
+      for (uint32_t q = tid; q < 2u * m_total; q += NT) prm.bnd[q] = 0ull;
+    }
+    if (tid == 0) *prm.gen = tag;
     if (tid == 0) {
       const unsigned long long fin = atomicAdd(prm.best, 0ull);
       prm.out_tok[0] = (int32_t)best_id(fin);
@@ -559,8 +718,8 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
   const int rows2_max = (int)((P + G - 1) / G);
   const int rmax = (int)(rows2_max / prm.b) + 2;
   auto fixed_for = [&](int k2) {
-    return (NT == 256 ? head1_layout<256>(row2, int4 ? rows1_max : 0, nch4, rmax, W * k2, 0)
-                      : head1_layout<512>(row2, int4 ? rows1_max : 0, nch4, rmax, W * k2, 0)).total;
+    return (NT == 256 ? head1_layout<256>(row2, rows1_max, nch4, rmax, W * k2, 0)
+                      : head1_layout<512>(row2, rows1_max, nch4, rmax, W * k2, 0)).total;
   };
   const uint32_t budget = 220u * 1024u;
   const int kcap = (1024 / 8 - 1) / W;  // barriers per stage (the last one of bars2 is the key copy's)

@@ -86,6 +86,8 @@ struct McParams {
 };
 
 // The batch-1 persistent head (fh_head1.cu).
+constexpr int kHead1BndMax = 512;  // boundary-bin keys the distributed selection takes
+
 struct Head1Params {
   const void* C;               // c x d (dense Stage 1) or null
   const uint8_t* q4;           // c x d/2 (INT4 Stage 1) or null
@@ -104,6 +106,9 @@ struct Head1Params {
   unsigned long long* ticket;     // final-reduction arrivals (grows by gridDim.x per call)
   unsigned long long* best;       // packed (key, ~token) maximum (zero between calls)
   uint32_t* hist;                 // 1024-bin key histogram (zero between calls)
+  uint32_t* gen;                  // tag of the last completed call (a call tags its entries gen+1)
+  unsigned long long* order;      // p: (tag, cluster) at the rank of each cluster above the boundary bin
+  unsigned long long* bnd;        // 2*kHead1BndMax: (tag, key image), (tag, cluster) of the boundary bin
   int32_t* out_tok;
   int32_t* dbg_sel;            // p or null
   int32_t* dbg_tok;            // p*b or null

@@ -230,8 +230,8 @@ fh_status fh_philox_u32(uint64_t seed, uint64_t step, uint32_t row, uint32_t rng
    device current); make that first call before any stream capture.  Calls share the one array, so
    calls that overlap in time on the GPU (on different streams) race; serialise them.
    Returns FH_ERR_WORKSPACE with a message when the index needs more scratch than the array holds
-   (roughly c*4 + 8 KiB bytes, so c up to about 30,000 clusters). */
-enum { FH_STATIC_SCRATCH_BYTES = 131072 };
+   (about 4*c + 12*p + 15 KiB bytes: every c up to FH_MAX_C at p = 512, about 15,000 at p = c). */
+enum { FH_STATIC_SCRATCH_BYTES = 262144 };
 fh_status fh_head_greedy_static(const fh_index* idx, const void* H, int p, int32_t* out_tok,
                                 fh_stream stream);
 

@@ -326,6 +326,40 @@ def test_bad_c2t_rejected(fh):
         fh.index_from_host(idx.E, idx.C, bad, "bf16")
 
 
+def test_batch1_without_debug_outputs_on_one_workspace(fh, orc, mid):
+    """The timed configuration: batch 1, no debug outputs, one workspace reused by consecutive calls
+    whose p and mode change (each call must ignore what the earlier ones left behind).  Every token
+    must equal that of a call on a fresh zeroed workspace with debug outputs (the same selection and
+    the same fp32 dot products), and the oracle's wherever its margins decide it."""
+    idx, H = mid
+    cfg = idx.cfg
+    I = load(fh, idx)
+    ws = I.workspace(fh.FH_OP_GREEDY, 1, cfg.c)
+    plan = [(0, cfg.p, False), (1, 37, False), (2, cfg.p, True), (3, 1, False), (4, cfg.c, False),
+            (5, cfg.p, False), (6, 500, True), (7, cfg.p, False), (7, 37, False), (8, 2, True)]
+    checked = 0
+    for q, p, sample in plan:
+        Hd = dev(H[q:q + 1], cfg.dtype)
+        fresh = torch.zeros_like(ws)
+        dbg = dict(sel=torch.empty((1, p), dtype=torch.int32, device=DEV),
+                   cand_tok=torch.empty((1, p * cfg.b), dtype=torch.int32, device=DEV),
+                   cand_logit=torch.empty((1, p * cfg.b), dtype=torch.float32, device=DEV))
+        if sample:
+            args = (I, Hd, p, 0.8, synth.SAMPLE_SEED, q)
+            tok = fh.head_sample(*args, ws=ws).item()
+            ref = fh.head_sample(*args, ws=fresh, debug=dbg).item()
+        else:
+            tok = fh.head_greedy(I, Hd, p, ws=ws).item()
+            ref = fh.head_greedy(I, Hd, p, ws=fresh, debug=dbg).item()
+        assert tok == ref, (q, p, sample)
+        o = orc.head(idx, H[q:q + 1], p, sample=sample, tau=0.8, seed=synth.SAMPLE_SEED, step=q)
+        if (p == cfg.c or o["set_margin"][0] > MARGIN) and o["tok_margin"][0] > MARGIN:
+            assert tok == o["tok"][0], (q, p, sample)
+            checked += 1
+    fh.ws_status(ws)
+    assert checked >= 2
+
+
 def test_workspace_status_clean(fh, mid):
     idx, H = mid
     I = load(fh, idx)
@@ -355,3 +389,19 @@ def test_llama_full_size_batch1_sampled(fh, orc, llama):
     for q in range(2):
         _check_head(fh, orc, idx, H[q:q + 1], idx.cfg.p, sample=True, tau=0.8,
                     seed=synth.SAMPLE_SEED, step=q)
+
+
+@pytest.mark.parametrize("perturb", [0.0, 1e-3])
+def test_crowded_boundary_bin_batch1(fh, orc, perturb):
+    """More keys than the fast path ranks share the boundary bin (identical or nearly identical
+    centroids), so the batch-1 kernel takes its full-selection branch; ties break by cluster id."""
+    v, d, c = 8192, 64, 1024
+    idx = synth.random_index(v=v, d=d, c=c, seed=17, dtype="bf16")
+    rng = np.random.default_rng(3)
+    base = rng.standard_normal(d)
+    rows = base[None, :] + perturb * rng.standard_normal((c, d))
+    rows /= np.linalg.norm(rows, axis=1, keepdims=True)
+    idx.C = synth.store(rows.astype(np.float32), "bf16")
+    H = synth.store((rng.standard_normal((3, d)) * 2).astype(np.float32), "bf16")
+    for q in range(3):
+        _check_head(fh, orc, idx, H[q:q + 1], 100)

@@ -35,12 +35,12 @@ def test_static_scratch_matches_workspace_calls(fh):
 
 
 def test_static_scratch_rejects_indices_that_do_not_fit(fh):
-    c = 32768                                    # c*4 bytes of keys alone fill the array
+    c = 32768                                    # keys and probe set of p = c fill the array
     rng = np.random.default_rng(0)
     E = synth.store(rng.standard_normal((c, 8)).astype(np.float32), "bf16")
     C2T = rng.permutation(c).astype(np.int32).reshape(c, 1)
     I = fh.index_from_host(E, E[C2T[:, 0]], C2T, "bf16", cluster_major=False)
     H = fh.device_array(synth.store(rng.standard_normal((1, 8)).astype(np.float32), "bf16"), "bf16")
     with pytest.raises(fh.FlashHeadError) as e:
-        fh.head_greedy_static(I, H, 1)
+        fh.head_greedy_static(I, H, c)
     assert e.value.status == 4 and "static scratch" in str(e.value)

@@ -65,7 +65,7 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
     L.part = take((size_t)G * B * 8);
     if (B == 1) {  // the persistent batch-1 kernel's tagged selection entries
       L.list = take((size_t)p * 8);
-      L.bnd = take((size_t)fh::kHead1BndMax * 16);
+      L.bnd = take((size_t)fh::kHead1BndMax * 8);
     }
   } else if (op == FH_OP_DENSE) {
     const int G = fh::stage2_blocks(D.v, B, idx->num_sms);
@@ -94,12 +94,12 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 // Workspace header (first kHeaderBytes): status word at 0, per-query tickets at 16 (64 x 4 bytes),
-// the persistent head's 64-bit grid-barrier arrival counter at 512, its 64-bit final-reduction
-// ticket at 520, its packed arg-max at 528 and its call generation at 536 (the tag of the last
-// completed call); bytes [1024, 5120) hold its 1024-bin score histogram in every layout, so no other
-// call ever writes there.  The two counters and the generation only grow; the arg-max and the
-// histogram return to zero at the end of every call.  A new workspace must start zeroed
-// (fh_ws_status re-zeroes the header after a device-side error, keeping the generation moving).
+// the persistent head's 64-bit final-reduction ticket at 520, its packed arg-max at 528 and its call
+// generation at 536 (the tag of the last completed call); bytes [1024, 5120) hold its 1024-bin score
+// histogram in every layout, so no other call ever writes there.  The ticket and the generation only
+// grow; the arg-max, the histogram and the selection entries return to zero at the end of every call.
+// A new workspace must start zeroed (fh_ws_status re-zeroes the header after a device-side error,
+// keeping the generation moving).
 uint32_t* status_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16); }
 uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
@@ -148,7 +148,9 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   cudaError_t e;
   // The persistent batch-1 kernel copies 16-byte C2T chunks next to each row, so it needs C2T
   // 16-byte aligned and v % 4 == 0 (no chunk runs past the end of C2T).
-  if (B == 1 && fh::head1_threads(D.c) != 0 && D.v % 4 == 0 && aligned16(D.C2T)) {
+  // It also splits rows with 32-bit arithmetic: v * num_sms < 2^31.
+  if (B == 1 && fh::head1_threads(D.c) != 0 && D.v % 4 == 0 && aligned16(D.C2T) &&
+      D.v * (int64_t)idx->num_sms < (int64_t{1} << 31)) {
     fh::Head1Params h = {};
     h.C = D.C;
     h.q4 = D.C_q4;
@@ -166,7 +168,6 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     h.tau = tau;
     h.seed = seed;
     h.step = step;
-    h.bar_count = reinterpret_cast<unsigned long long*>(word_at(ws, 512));
     h.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, 520));
     h.best = reinterpret_cast<unsigned long long*>(word_at(ws, 528));
     h.hist = word_at(ws, 1024);

@@ -210,12 +210,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-// Hint: start moving [src, src + bytes) from HBM into L2 (bulk prefetch through the copy engine; no
-// data returns to the SM and nothing waits for it).  src 16-byte aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // ------------------------------------------------------------------------------ PDL
 // Programmatic dependent launch: the next kernel of the stream may start its prologue once every block
 // of this kernel has called launch_dependents; wait_prior blocks until the preceding kernel finished

@@ -125,35 +125,27 @@ __device__ __forceinline__ Binning make_binning(const float hnorm, int sample, f
   return bn;
 }
 
-// Grid barrier on a monotonic 64-bit arrival counter: the call's last arrival makes the counter a
-// multiple of the grid size.  Returns false if the wait timed out (status set).
-__device__ __forceinline__ bool grid_barrier(unsigned long long* count, uint32_t nblocks,
-                                             uint32_t* status, bool* abort_s) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    bool ok = true;
-    __threadfence();
-    const unsigned long long old = atomicAdd(count, 1ull);
-    const unsigned long long target = (old / nblocks + 1) * nblocks;
-    if (old + 1 != target) {
-      const uint64_t t0 = global_timer_ns();
-      uint32_t it = 0;
-      for (;;) {
-        unsigned long long now;
-        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(now) : "l"(count) : "memory");
-        if (now >= target) break;
-        if ((++it & 255u) == 0 && global_timer_ns() - t0 > 500000000ull) {
-          set_status(status, kStatusTimeout);
-          ok = false;
-          break;
-        }
-      }
-    }
-    __threadfence();
-    *abort_s = !ok;
+__device__ __forceinline__ uint32_t atom_add_release_u32(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
+// HPT consecutive histogram bins (16- or 8-byte aligned) with one relaxed gpu-scope vector load.
+template <int HPT>
+__device__ __forceinline__ void load_bins_relaxed(const uint32_t* p, uint32_t (&hb)[HPT]) {
+  if constexpr (HPT == 4) {
+    asm volatile("ld.relaxed.gpu.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(hb[0]), "=r"(hb[1]), "=r"(hb[2]), "=r"(hb[3]) : "l"(p) : "memory");
+  } else {
+    asm volatile("ld.relaxed.gpu.global.v2.u32 {%0, %1}, [%2];" : "=r"(hb[0]), "=r"(hb[1]) : "l"(p) : "memory");
   }
-  __syncthreads();
-  return !*abort_s;
+}
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
@@ -232,8 +224,11 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   const int nch2 = (int)(row2 / 16);
   const int nch4 = INT4_MCH ? (int)(d / 32) : 0;
   const int P = prm.p * b;
-  const int rows1_max = (int)((c + G - 1) / G);
-  const int rows2_max = (int)((P + G - 1) / G);
+  // 32-bit splits (the launcher keeps v * gridDim.x below 2^31): 64-bit division is a long software
+  // sequence on the GPU, and these sit on the path between the stages.
+  const uint32_t uG = (uint32_t)G, uc = (uint32_t)c;
+  const int rows1_max = (int)((uc + uG - 1u) / uG);
+  const int rows2_max = (int)(((uint32_t)P + uG - 1u) / uG);
   const int rmax = (int)(rows2_max / b) + 2;
   const int K1 = prm.k1, K2 = prm.k2;
   const Head1Layout L = head1_layout<NT>(row2, rows1_max, nch4, rmax, W * K2, prm.ring_bytes);
@@ -257,8 +252,10 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     const int ch = tid + u * NT;
     if (ch < nch2) hv[u] = __ldg(reinterpret_cast<const uint4*>(prm.H) + ch);
   }
-  const int64_t lo1 = c * bid / G, hi1 = c * (bid + 1) / G;
-  const uint32_t tag = __ldcg(prm.gen) + 1u;  // this call's tag on its selection entries
+  const int64_t lo1 = uc * (uint32_t)bid / uG, hi1 = uc * (uint32_t)(bid + 1) / uG;
+  // this call's tags on its selection entries: 32 bits on the certain ranks, 18 on the boundary bin
+  const uint32_t tag = __ldcg(prm.gen) + 1u;
+  const uint32_t tag_b = (tag & 0x3FFFFu) | (uint32_t)((tag & 0x3FFFFu) == 0u);
   uint32_t scv[4];  // INT4: this block's group scales, two per 32-bit word
   const int nsc = INT4_MCH ? (int)((hi1 - lo1) * nch4) : 0;
   const int sc_words = (nsc + 1) / 2;
@@ -276,7 +273,7 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   }
   if (tid < W * K1) mbar_init(&bars1[tid], 1);
   if (tid < W * K2) mbar_init(&bars2[tid], 1);
-  uint64_t* bar_keys = &bars2[127];  // keys + histogram copy after the grid barrier
+  uint64_t* bar_keys = &bars2[127];  // key copy of the full selection
   if (tid == 0) mbar_init(bar_keys, 1);
   fence_mbar_init();
   __syncthreads();
@@ -375,45 +372,52 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     }
   }
   __syncthreads();
-  // Add the block's counts to the global histogram; each add returns the block's first position in
-  // that bin, so every key gets a distinct position among the keys of its bin.
+  // Add the block's counts to the global histogram.  The adds are releases (whoever sees a count also
+  // sees the keys this block wrote), and each returns the block's first position in that bin, so every
+  // key gets a distinct position among the keys of its bin.
   for (int i = tid; i < kHistBins; i += NT) {
     const uint32_t n = hist_s[i];
-    if (n) hist_s[i] = atomicAdd(&prm.hist[i], n);
+    if (n) hist_s[i] = atom_add_release_u32(&prm.hist[i], n);
   }
 
-  // ------------------------------------------------------------------ grid barrier
-  if (!grid_barrier(prm.bar_count, (uint32_t)G, prm.status, &abort_s)) return;
-
-  // ------------------------------------------------------------------ boundary bin
-  // The summed histogram comes in with one bulk copy into the ring, idle between the stages.
-  uint32_t* histg_s = reinterpret_cast<uint32_t*>(ring);
-  if (tid == 0) {
-    asm volatile("fence.proxy.async;" ::: "memory");  // written by other blocks, seen via the barrier
-    mbar_arrive_expect_tx(bar_keys, kHistBins * 4u);
-    bulk_g2s(histg_s, prm.hist, kHistBins * 4u, bar_keys);
-  }
-  if (!mbar_wait(bar_keys, 0u, prm.status)) return;
+  // ------------------------------------------------------------------ histogram (grid barrier)
+  // The summed histogram is complete once its counts add up to c.  Every block polls it until then:
+  // the poll is the grid barrier, and its last round already holds the counts the selection needs.
   constexpr int HPT = kHistBins / NT;  // histogram bins per thread
+  static_assert(HPT == 2 || HPT == 4, "bins per thread");
   uint32_t hb[HPT];
-  uint32_t htot = 0;
-#pragma unroll
-  for (int u = 0; u < HPT; ++u) {
-    hb[u] = histg_s[tid * HPT + u];
-    htot += hb[u];
-  }
+  uint32_t htot = 0, before = 0;
   for (int i = tid; i < 1025; i += NT) sm.selbits[i] = 0u;
-  if (tid == 0) {
+  if (tid == 0) {  // (the polling loop's barriers order these before the boundary search)
     sm.cand_count = 0u;
     dstar_s = 0u;
     above_s = 0u;
   }
+  {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+      load_bins_relaxed<HPT>(prm.hist + tid * HPT, hb);
+      htot = 0;
+#pragma unroll
+      for (int u = 0; u < HPT; ++u) htot += hb[u];
+      const unsigned long long ex = block_scan2<NT>(0u, htot, sm, 0);
+      before = (uint32_t)(ex & 0xFFFFFFFFull);
+      if (tid == NT - 1) total_s = before + htot;
+      if (tid == 0) abort_s = (it & 15u) == 0u && global_timer_ns() - t0 > 500000000ull;
+      __syncthreads();
+      if (total_s >= (uint32_t)c || abort_s) break;  // the same decision in every thread
+      __syncthreads();                                 // total_s and the scan scratch are reused
+    }
+    if (total_s != (uint32_t)c) {  // a wait gave up somewhere: nothing below is valid
+      if (tid == 0) set_status(prm.status, kStatusTimeout);
+      return;
+    }
+  }
+
+  // ------------------------------------------------------------------ boundary bin
+  uint32_t* histg_s = reinterpret_cast<uint32_t*>(ring);  // keys in bins above each bin
   const bool all = prm.p >= c;
   {
-    const unsigned long long ex = block_scan2<NT>(0u, htot, sm, 0);
-    const uint32_t before = (uint32_t)(ex & 0xFFFFFFFFull);
-    if (tid == NT - 1) total_s = before + htot;
-    __syncthreads();
     uint32_t cum = total_s - before - htot;  // keys in bins above this thread's bins
 #pragma unroll
     for (int u = HPT - 1; u >= 0; --u) {
@@ -426,10 +430,6 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       cum += hb[u];
     }
     __syncthreads();
-    if (total_s != (uint32_t)c) {  // a Stage-1 wait gave up somewhere: nothing below is valid
-      if (tid == 0) set_status(prm.status, kStatusTimeout);
-      return;
-    }
   }
   const uint32_t dstar = all ? 0u : dstar_s;
   const uint32_t above_n = all ? (uint32_t)c : above_s;
@@ -439,8 +439,9 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   // [d0, d1) (global rows in list order: rank r = row / b, certain ranks first).  Local row l is
   // c0 + l below nc and d0 + (l - nc) above, so certain rows stream while the boundary is resolved.
   const int CR = (int)above_n * b, BR = (int)need * b;
-  const int c0 = (int)((int64_t)CR * bid / G), c1 = (int)((int64_t)CR * (bid + 1) / G);
-  const int d0 = CR + (int)((int64_t)BR * bid / G), d1 = CR + (int)((int64_t)BR * (bid + 1) / G);
+  const int c0 = (int)((uint32_t)CR * (uint32_t)bid / uG), c1 = (int)((uint32_t)CR * (uint32_t)(bid + 1) / uG);
+  const int d0 = CR + (int)((uint32_t)BR * (uint32_t)bid / uG);
+  const int d1 = CR + (int)((uint32_t)BR * (uint32_t)(bid + 1) / uG);
   const int nc = c1 - c0, nr = nc + (d1 - d0);
   const int rc0 = c0 / b, rc1 = (c1 + b - 1) / b;  // certain ranks touched
   const int rb0 = d0 / b, rb1 = (d1 + b - 1) / b;  // boundary ranks touched
@@ -472,9 +473,6 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     const uint8_t* src = perm ? Ep + (size_t)e * row2 : E + (size_t)__ldg(prm.C2T + e) * row2;
     bulk_g2s(ring2 + (size_t)slot * row2, src, row2, &b2[slot]);
   };
-  // the first K2 slots of each warp that hold certain rows
-  int issued = 0;
-  while (issued < K2 && issued < n2 && warp + W * issued < nc) ++issued;
   const bool fast = all || m_total <= (uint32_t)kSelCandMax;
 
   if (fast) {
@@ -482,8 +480,9 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     // A cluster's rank in the Stage-2 list is (keys in higher bins) + (its position in its bin), known
     // to the block that scored it as soon as the histogram is: each block writes the ids of its
     // certain clusters at their ranks, and the (key, id) of its boundary-bin clusters at their
-    // positions, each as one 64-bit word tagged with the call's tag.  Every block then polls only the
-    // words its rows need (and the boundary bin, which it ranks itself): no counters, no fences.
+    // positions, each as one 64-bit word tagged with the call's tag.  Block 0 resolves the boundary
+    // bin and writes the ranks it fills the same way.  Every block polls only the words its own rows
+    // need, so no word is read by more than a few blocks: no counters, no fences, no hot spot.
     const int nk = (int)(hi1 - lo1);
     if (tid < nk) {
       const uint32_t img = float_key(own_keys[tid]);
@@ -493,51 +492,79 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       const uint32_t id = (uint32_t)(lo1 + tid);
       if (all || dg > dstar) {
         st_relaxed_u64(prm.order + histg_s[dg] + pos, tg | id);
-      } else if (dg == dstar) {
-        st_relaxed_u64(prm.bnd + 2 * pos, tg | img);
-        st_relaxed_u64(prm.bnd + 2 * pos + 1, tg | id);
-      }
-      // Whichever block streams them, the rows of this block's selected and boundary clusters start
-      // moving into L2 now (cluster-major copy: one range per cluster).
-      if (perm && (all || dg >= dstar)) bulk_prefetch_l2(Ep + (size_t)id * b * row2, (uint32_t)b * row2);
-    }
-    const bool rank_here = need > 0u && (d1 > d0 || want_dbg);
-    bool ok = true;
-    for (int r = rc0 + tid; r < rc1; r += NT)
-      rk_c[r - rc0] = (int)(uint32_t)poll_tagged(prm.order + r, tag, prm.status, ok);
-    if (rank_here) {
-      for (uint32_t q = tid; q < m_total; q += NT) {
-        sm.cand_key[q] = __uint_as_float((uint32_t)poll_tagged(prm.bnd + 2 * q, tag, prm.status, ok));
-        sm.cand_id[q] = (int)(uint32_t)poll_tagged(prm.bnd + 2 * q + 1, tag, prm.status, ok);
+      } else if (dg == dstar) {  // (18-bit tag, 14-bit id, key image)
+        st_relaxed_u64(prm.bnd + pos, ((unsigned long long)tag_b << 46) |
+                                      ((unsigned long long)id << 32) | img);
       }
     }
-    if (want_dbg)  // the debug outputs read the whole certain list below
-      for (uint32_t q = tid; q < above_n; q += NT) poll_tagged(prm.order + q, tag, prm.status, ok);
-    if (!__syncthreads_and(ok)) return;  // a wait gave up (status set); no copy is in flight yet
-    if (lane < issued) {
-      fence_proxy_async_smem();  // the ring was last read by Stage 1 and the histogram copy
-      issue2(lane);
+    // Poll tagged words (each thread at most one of `words`, all loads of a round in flight together);
+    // false if a wait gave up (status set).
+    auto poll_words = [&](const unsigned long long* words, int n, int* dst) {
+      bool ok = true;
+      for (int q = tid; q < n; q += NT) dst[q] = (int)(uint32_t)poll_tagged(words + q, tag, prm.status, ok);
+      return ok;
+    };
+    // Every word this block needs is read before any of its Stage-2 copies is issued: a small load
+    // issued behind a block's bulk copies waits until they have drained.
+    if (need > 0u) {
+      if (bid == 0) {
+        // The resolver: reads the boundary bin's keys once, ranks them exactly, and writes the ids
+        // of the `need` best at ranks above_n .. p - 1, tagged like the certain ones.
+        bool ok = true;
+        {
+          const uint32_t qa = (uint32_t)tid, qb = (uint32_t)(tid + NT);
+          uint32_t pend = (qa < m_total ? 1u : 0u) | (qb < m_total ? 2u : 0u);
+          const uint64_t t0 = global_timer_ns();
+          for (uint32_t it = 1; pend; ++it) {
+            unsigned long long v0 = 0ull, v1 = 0ull;
+            if (pend & 1u) v0 = ld_relaxed_u64(prm.bnd + qa);
+            if (pend & 2u) v1 = ld_relaxed_u64(prm.bnd + qb);
+            if ((pend & 1u) && (uint32_t)(v0 >> 46) == tag_b) {
+              sm.cand_key[qa] = __uint_as_float((uint32_t)v0);
+              sm.cand_id[qa] = (int)((uint32_t)(v0 >> 32) & 0x3FFFu);
+              pend &= ~1u;
+            }
+            if ((pend & 2u) && (uint32_t)(v1 >> 46) == tag_b) {
+              sm.cand_key[qb] = __uint_as_float((uint32_t)v1);
+              sm.cand_id[qb] = (int)((uint32_t)(v1 >> 32) & 0x3FFFu);
+              pend &= ~2u;
+            }
+            if (pend && (it & 15u) == 0u && global_timer_ns() - t0 > 500000000ull) {
+              set_status(prm.status, kStatusTimeout);
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (!__syncthreads_and(ok)) return;
+        int* bsel_rank = reinterpret_cast<int*>(sm.selbits);
+        if (m_total <= 128u)
+          rank_boundary<4>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
+        else
+          rank_boundary<kSelCandMax / 32>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
+        __syncthreads();
+        const unsigned long long tg = (unsigned long long)tag << 32;
+        for (uint32_t r = tid; r < need; r += NT)
+          st_relaxed_u64(prm.order + above_n + r, tg | (uint32_t)bsel_rank[r]);
+      }
     }
-    // boundary ranks: every block with boundary rows ranks the boundary bin while its certain rows fly
-    int* bsel_rank = reinterpret_cast<int*>(sm.selbits);
-    if (rank_here) {
-      if (m_total <= 128u)
-        rank_boundary<4>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
-      else
-        rank_boundary<kSelCandMax / 32>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
-      __syncthreads();
-      for (int r = rb0 + tid; r < rb1; r += NT) rk_b[r - rb0] = bsel_rank[r - (int)above_n];
-      __syncthreads();
+    // the certain and the boundary ranks of this block's rows (the resolver reads back its own words)
+    {
+      bool ok = poll_words(prm.order + rc0, rc1 - rc0, rk_c);
+      if (rb1 > rb0) ok = poll_words(prm.order + rb0, rb1 - rb0, rk_b) && ok;
+      if (!__syncthreads_and(ok)) return;
     }
     if (want_dbg) {
       // canonical (ascending) positions: count the selected clusters below each of this block's
-      auto cert_at = [&](uint32_t q) { return (int)(uint32_t)__ldcg(prm.order + q); };
+      bool ok = true;
+      for (int q = tid; q < prm.p; q += NT) poll_tagged(prm.order + q, tag, prm.status, ok);
+      if (!__syncthreads_and(ok)) return;
+      auto sel_at = [&](int q) { return (int)(uint32_t)__ldcg(prm.order + q); };
       const int ncr = rc1 - rc0, nbr = rb1 - rb0;
       for (int t = warp; t < ncr + nbr; t += W) {
         const int x = t < ncr ? rk_c[t] : rk_b[t - ncr];
         uint32_t cnt = 0;
-        for (uint32_t q = lane; q < above_n; q += 32) cnt += (uint32_t)(cert_at(q) < x);
-        for (uint32_t q = lane; q < need; q += 32) cnt += (uint32_t)(bsel_rank[q] < x);
+        for (int q = lane; q < prm.p; q += 32) cnt += (uint32_t)(sel_at(q) < x);
         cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
         if (lane == 0) {
           if (t < ncr) asc_c[t] = (int)cnt;
@@ -545,18 +572,17 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
         }
       }
       if (prm.dbg_sel && bid == 0) {
-        for (uint32_t q = tid; q < (uint32_t)prm.p; q += NT) {
-          const int x = q < above_n ? cert_at(q) : bsel_rank[q - above_n];
+        for (int q = tid; q < prm.p; q += NT) {
+          const int x = sel_at(q);
           uint32_t cnt = 0;
-          for (uint32_t y = 0; y < above_n; ++y) cnt += (uint32_t)(cert_at(y) < x);
-          for (uint32_t y = 0; y < need; ++y) cnt += (uint32_t)(bsel_rank[y] < x);
+          for (int y = 0; y < prm.p; ++y) cnt += (uint32_t)(sel_at(y) < x);
           prm.dbg_sel[cnt] = x;
         }
       }
       __syncthreads();
     }
-    if (lane >= issued && lane < K2 && lane < n2) {
-      fence_proxy_async_smem();
+    if (lane < K2 && lane < n2) {
+      fence_proxy_async_smem();  // the ring was last read by Stage 1
       issue2(lane);
     }
   } else {
@@ -565,12 +591,16 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     // with the block-wide selector (exact radix passes on the boundary bin).
     const uint32_t keys_bytes = (uint32_t)((c * 4 + 15) / 16 * 16);
     float* keys_s = reinterpret_cast<float*>(ring + kHistBins * 4);
+    // Every thread saw some of the release adds of the histogram: its acquire fence makes the keys
+    // of those blocks visible, and the barrier passes that on to thread 0, which copies them.
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
     __syncthreads();
     if (tid == 0) {
+      asm volatile("fence.proxy.async;" ::: "memory");
       mbar_arrive_expect_tx(bar_keys, keys_bytes);
       bulk_g2s(keys_s, prm.keys, keys_bytes, bar_keys);
     }
-    if (!mbar_wait(bar_keys, 1u, prm.status)) return;
+    if (!mbar_wait(bar_keys, 0u, prm.status)) return;
     uint32_t key[KPT];
     {
       const int kb = tid * KPT;
@@ -687,8 +717,8 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     __threadfence();
     for (int i = tid; i < kHistBins; i += NT) prm.hist[i] = 0u;
     if (fast) {  // the next call starts from zeroed entries (the tags already tell calls apart)
-      for (uint32_t q = tid; q < above_n; q += NT) prm.order[q] = 0ull;
-      for (uint32_t q = tid; q < 2u * m_total; q += NT) prm.bnd[q] = 0ull;
+      for (uint32_t q = tid; q < (uint32_t)prm.p; q += NT) prm.order[q] = 0ull;
+      for (uint32_t q = tid; q < m_total; q += NT) prm.bnd[q] = 0ull;
     }
     if (tid == 0) *prm.gen = tag;
     if (tid == 0) {
@@ -713,6 +743,7 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
   if (row2 / 16 > 4u * (uint32_t)NT) return cudaErrorInvalidValue;  // h: 4 chunks per thread
   const int nch4 = int4 ? (int)(prm.d / 32) : 0;
   const int64_t P = (int64_t)prm.p * prm.b;
+  if ((prm.c * prm.b) * (int64_t)G >= (int64_t{1} << 31)) return cudaErrorInvalidValue;  // 32-bit splits
   const int rows1_max = (int)((prm.c + G - 1) / G);
   if (int4 && (rows1_max * nch4 + 1) / 2 > 4 * NT) return cudaErrorInvalidValue;
   const int rows2_max = (int)((P + G - 1) / G);

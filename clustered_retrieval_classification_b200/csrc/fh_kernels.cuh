@@ -102,13 +102,12 @@ struct Head1Params {
   int sample;
   float tau;
   uint64_t seed, step;
-  unsigned long long* bar_count;  // grid-barrier arrivals (grows by gridDim.x per call)
   unsigned long long* ticket;     // final-reduction arrivals (grows by gridDim.x per call)
   unsigned long long* best;       // packed (key, ~token) maximum (zero between calls)
   uint32_t* hist;                 // 1024-bin key histogram (zero between calls)
   uint32_t* gen;                  // tag of the last completed call (a call tags its entries gen+1)
   unsigned long long* order;      // p: (tag, cluster) at the rank of each cluster above the boundary bin
-  unsigned long long* bnd;        // 2*kHead1BndMax: (tag, key image), (tag, cluster) of the boundary bin
+  unsigned long long* bnd;        // kHead1BndMax: (tag, cluster, key image) of the boundary bin's keys
   int32_t* out_tok;
   int32_t* dbg_sel;            // p or null
   int32_t* dbg_tok;            // p*b or null

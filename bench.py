@@ -39,7 +39,10 @@ PAGES_TOKENS_PER_S = 1.0 / 0.40e-3
 
 # DRAM traffic per launch from the committed ncu captures (profiles/), valid only for the kernel
 # sources they were taken on (sha1 of the csrc files); null otherwise.
-TRAFFIC = {}
+TRAFFIC = {
+    # profiles/k_head1_llama_batch1.md: dram__bytes_read.sum + dram__bytes_write.sum of one launch
+    (1, "8df018758907"): 66_547_200 + 948_224,
+}
 
 L2_FLUSH_BYTES = 256 << 20
 
@@ -426,6 +429,22 @@ def run_reference(args):
 # ----------------------------------------------------------------------------- main
 
 
+def ncu_case(args):
+    """A few batch-1 greedy calls of the Llama-shaped head on a single index copy, nothing timed."""
+    from clustered_retrieval_classification_b200 import flashhead as F
+    F.load()
+    cfg = synth.CONFIGS["llama"]
+    idx = synth.make_index(cfg)
+    R = Replicated(F, idx, replicas=1)
+    Hd = F.device_array(synth.make_queries(cfg, 64), "bf16")
+    step = head_step(F, R, Hd, 1, cfg.p)
+    for k in range(min(args.steps, 64)):
+        step(k)
+    torch.cuda.synchronize()
+    print("ncu case: %d calls of the batch-1 greedy head, %s" % (min(args.steps, 64), cfg.name))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -435,10 +454,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--ncu-case", action="store_true",
+                    help="run --steps untimed calls of the headline configuration on one index copy "
+                         "(about 1.1 GB on the device) and exit: the case the committed ncu captures use")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         return run_reference(args)
+    if args.ncu_case:
+        return ncu_case(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -436,12 +436,17 @@ def ncu_case(args):
     cfg = synth.CONFIGS["llama"]
     idx = synth.make_index(cfg)
     R = Replicated(F, idx, replicas=1)
-    Hd = F.device_array(synth.make_queries(cfg, 64), "bf16")
-    step = head_step(F, R, Hd, 1, cfg.p)
+    Hd = F.device_array(synth.make_queries(cfg, 128), "bf16")
+    B = args.batch
+    if args.ncu_what == "dense":
+        step = dense_step(F, R, Hd, B)
+    else:
+        step = head_step(F, R, Hd, B, cfg.p, mode=args.ncu_what)
     for k in range(min(args.steps, 64)):
         step(k)
     torch.cuda.synchronize()
-    print("ncu case: %d calls of the batch-1 greedy head, %s" % (min(args.steps, 64), cfg.name))
+    print("ncu case: %d calls of the %s head at batch %d, %s" % (min(args.steps, 64), args.ncu_what, B,
+                                                               cfg.name))
     return 0
 
 
@@ -455,8 +460,10 @@ def main():
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--ncu-case", action="store_true",
-                    help="run --steps untimed calls of the headline configuration on one index copy "
-                         "(about 1.1 GB on the device) and exit: the case the committed ncu captures use")
+                    help="run --steps untimed calls on one index copy (about 1.1 GB on the device) and "
+                         "exit: the case the committed ncu captures use")
+    ap.add_argument("--ncu-what", default="greedy", choices=["greedy", "dense", "sample"],
+                    help="with --ncu-case: which head (at --batch queries) to call")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":

@@ -4,6 +4,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <algorithm>
 #include <cstring>
 #include <new>
 
@@ -35,6 +36,7 @@ fh_status cuda_fail(cudaError_t e, const char* what) {
 
 constexpr size_t kHeaderBytes = 1024 + 4096;  // control words, then the score histogram
 constexpr size_t kGenOffset = 536;             // batch-1 head: tag of the last completed call
+constexpr size_t kTcTicketOffset = 544;        // tensor-core head: arrival ticket (zero between calls)
 constexpr size_t kAlign = 256;
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -43,7 +45,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Workspace regions of one call; offsets from the workspace base.
 struct Layout {
-  size_t keys = 0, sel = 0, part = 0, list = 0, bnd = 0, z = 0, s = 0, zmax = 0, Z = 0,
+  size_t keys = 0, sel = 0, part = 0, list = 0, bnd = 0, qmask = 0, best = 0, tiles = 0, z = 0, s = 0,
+         zmax = 0, Z = 0,
          cluster_of = 0, per_draw = 0;
   size_t total = 0;
 };
@@ -63,6 +66,11 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
     L.keys = take((size_t)B * D.c * 4);
     L.sel = take((size_t)B * p * 4);
     L.part = take((size_t)G * B * 8);
+    if (B > 1) {  // tensor-core Stage 2: per-cluster query masks, the selected clusters, arg-maxima
+      L.qmask = take((size_t)D.c * 8);
+      L.best = take((size_t)B * 8);
+      L.tiles = take((size_t)(std::max<int64_t>(D.c, (D.v + 127) / 128) + 1) * 4);
+    }
     if (B == 1) {  // the persistent batch-1 kernel's tagged selection entries
       L.list = take((size_t)p * 8);
       L.bnd = take((size_t)fh::kHead1BndMax * 8);
@@ -70,6 +78,7 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
   } else if (op == FH_OP_DENSE) {
     const int G = fh::stage2_blocks(D.v, B, idx->num_sms);
     L.part = take((size_t)G * B * 8);
+    L.best = take((size_t)B * 8);
   } else if (op == FH_OP_MC) {
     const int G = fh::stage2_blocks(D.v, B, idx->num_sms);
     L.part = take((size_t)G * B * 8);
@@ -103,6 +112,17 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 uint32_t* status_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16); }
 uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
+
+// The tensor-core path: BF16 E (and, for FlashHead, its cluster-major copy), batches up to 64.  The
+// dense head takes it from 2 queries on; FlashHead from kTcMinBatchHead, below which the union of
+// the probe sets is sparse enough that the per-query CUDA-core Stage 2 reads fewer bytes.
+constexpr int kTcMinBatchDense = 2;
+constexpr int kTcMinBatchHead = 8;
+constexpr int kTcListTilesBatch = 16;  // from here on Stage 2 streams whole tiles instead of gathering
+bool tc_eligible(const fh_index* idx, int B, int min_batch) {
+  const fh_index_desc& D = idx->desc;
+  return B >= min_batch && D.dtype == FH_BF16 && fh::tc_supported(fh::kBF16, D.d, B);
+}
 
 fh_status check_batch(const fh_index* idx, const void* H, int B) {
   if (!idx) return fail(FH_ERR_ARG, "index handle is NULL");
@@ -184,23 +204,78 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     return FH_OK;
   }
   const bool fused = false;
-  fh::Stage1Params s1 = stage1_params(idx, H, B, keys, ws);
-  s1.sample = sample;
-  s1.tau = tau;
-  s1.seed = seed;
-  s1.step = step;
-  s1.rng_stream = FH_RNG_STAGE1;
-  s1.tickets_to_clear = tickets_of(ws);
-  s1.n_tickets = B;
-  e = fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st, fused);
-  if (e != cudaSuccess) return cuda_fail(e, "stage-1 launch");
-  if (!fused) {
+  const bool tc = tc_eligible(idx, B, kTcMinBatchHead) && !dbg && D.E_perm != nullptr;
+  if (tc && s1fmt(idx) == FH_STAGE1_DENSE) {
+    // Stage 1 on the tensor cores too: keys[q][k] = C[k]·h_q (+ the Gumbel term when sampling)
+    fh::TcParams tp = {};
+    tp.rows = D.c;
+    tp.d = D.d;
+    tp.B = B;
+    tp.b = 1;
+    tp.sample = sample;
+    tp.tau = tau;
+    tp.seed = seed;
+    tp.step = step;
+    tp.out_keys = keys;
+    tp.status = status_of(ws);
+    if ((e = fh::launch_tc_head(D.C, H, tp, idx->num_sms, st)) != cudaSuccess)
+      return cuda_fail(e, "tensor-core stage-1 launch");
     if ((e = fh::launch_select(keys, sel, B, D.c, p, st)) != cudaSuccess)
       return cuda_fail(e, "select launch");
-    if (dbg && dbg->sel &&
-        (e = cudaMemcpyAsync(dbg->sel, sel, (size_t)B * p * 4, cudaMemcpyDeviceToDevice, st)) !=
-            cudaSuccess)
-      return cuda_fail(e, "debug copy");
+  } else {
+    fh::Stage1Params s1 = stage1_params(idx, H, B, keys, ws);
+    s1.sample = sample;
+    s1.tau = tau;
+    s1.seed = seed;
+    s1.step = step;
+    s1.rng_stream = FH_RNG_STAGE1;
+    s1.tickets_to_clear = tickets_of(ws);
+    s1.n_tickets = B;
+    e = fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st, fused);
+    if (e != cudaSuccess) return cuda_fail(e, "stage-1 launch");
+    if (!fused) {
+      if ((e = fh::launch_select(keys, sel, B, D.c, p, st)) != cudaSuccess)
+        return cuda_fail(e, "select launch");
+      if (dbg && dbg->sel &&
+          (e = cudaMemcpyAsync(dbg->sel, sel, (size_t)B * p * 4, cudaMemcpyDeviceToDevice, st)) !=
+              cudaSuccess)
+        return cuda_fail(e, "debug copy");
+    }
+  }
+  if (tc) {
+    // Stage 2 on the tensor cores: every tile of the cluster-major copy that some query selected,
+    // masked per (cluster, query), the arg-max of each query fused in.
+    unsigned long long* qmask = reinterpret_cast<unsigned long long*>(base + L.qmask);
+    if ((e = cudaMemsetAsync(qmask, 0, (size_t)D.c * 8, st)) != cudaSuccess) return cuda_fail(e, "memset");
+    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st)) != cudaSuccess)
+      return cuda_fail(e, "mask launch");
+    fh::TcParams tp = {};
+    tp.rows = D.v;
+    tp.d = D.d;
+    tp.B = B;
+    tp.b = D.b;
+    tp.qmask = qmask;
+    tp.row_tok = D.C2T;  // row e of the cluster-major copy is token C2T[e]
+    tp.sample = sample;
+    tp.tau = tau;
+    tp.seed = seed;
+    tp.step = step;
+    tp.best = reinterpret_cast<unsigned long long*>(base + L.best);
+    tp.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, kTcTicketOffset));
+    tp.out_tok = out_tok;
+    if (B < kTcListTilesBatch && D.b % 8 == 0 && 128 % D.b == 0) {
+      // few queries: the union of the probe sets is sparse, gather its clusters into tiles
+      tp.cl_list = reinterpret_cast<int32_t*>(base + L.tiles) + 1;
+      tp.cl_count = reinterpret_cast<int32_t*>(base + L.tiles);
+    } else {
+      // many queries: the union covers most clusters, stream the contiguous tiles it touches
+      tp.tile_list = reinterpret_cast<int32_t*>(base + L.tiles) + 1;
+      tp.tile_count = reinterpret_cast<int32_t*>(base + L.tiles);
+    }
+    tp.status = status_of(ws);
+    if ((e = fh::launch_tc_head(D.E_perm, H, tp, idx->num_sms, st)) != cudaSuccess)
+      return cuda_fail(e, "tensor-core stage-2 launch");
+    return FH_OK;
   }
   fh::Stage2Params s2 = {};
   s2.E = D.E;
@@ -365,7 +440,27 @@ fh_status fh_dense_head(const fh_index* idx, const void* H, int B, int sample, f
   if ((r = check_ws(ws, ws_bytes, L.total)) != FH_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const fh_index_desc& D = idx->desc;
-  cudaError_t e = cudaMemsetAsync(tickets_of(ws), 0, (size_t)B * 4, st);
+  cudaError_t e;
+  if (tc_eligible(idx, B, kTcMinBatchDense)) {
+    fh::TcParams tp = {};
+    tp.rows = D.v;
+    tp.d = D.d;
+    tp.B = B;
+    tp.b = 1;
+    tp.sample = sample;
+    tp.tau = tau;
+    tp.seed = seed;
+    tp.step = step;
+    tp.best = reinterpret_cast<unsigned long long*>(static_cast<char*>(ws) + L.best);
+    tp.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, kTcTicketOffset));
+    tp.out_tok = out_tok;
+    tp.out_logits = out_logits;
+    tp.status = status_of(ws);
+    if ((e = fh::launch_tc_head(D.E, H, tp, idx->num_sms, st)) != cudaSuccess)
+      return cuda_fail(e, "tensor-core dense launch");
+    return FH_OK;
+  }
+  e = cudaMemsetAsync(tickets_of(ws), 0, (size_t)B * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   fh::DenseParams dp = {};
   dp.E = D.E;

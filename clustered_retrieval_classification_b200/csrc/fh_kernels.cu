@@ -640,6 +640,21 @@ cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int
   return cudaGetLastError();
 }
 
+// qmask[cluster] |= 1 << q for every cluster in query q's probe set (qmask zeroed beforehand).
+__global__ void k_build_qmask(const int32_t* __restrict__ sel, int B, int p, unsigned long long* qmask) {
+  const int64_t n = (int64_t)B * p;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    atomicOr(qmask + sel[i], 1ull << (uint32_t)(i / p));
+}
+
+cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
+                               cudaStream_t st) {
+  const int64_t n = (int64_t)B * p;
+  const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
+  k_build_qmask<<<blocks, 256, 0, st>>>(sel, B, p, qmask);
+  return cudaGetLastError();
+}
+
 int stage2_blocks(int64_t rows, int B, int num_sms) {
   int64_t g = (B == 1) ? num_sms : (2 * (int64_t)num_sms + B - 1) / B;
   const int64_t max_g = (rows + 7) / 8;  // at least ~8 rows per block

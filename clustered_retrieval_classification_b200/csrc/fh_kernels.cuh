@@ -85,6 +85,33 @@ struct McParams {
   uint32_t* status;
 };
 
+// Tensor-core logits for a batch of queries with the mask and the decision fused (fh_tc.cu).
+struct TcParams {
+  int64_t rows, d;                 // A operand: rows x d (E, or its cluster-major copy)
+  int B;                           // queries (<= 64)
+  int64_t b;                       // rows per cluster (the mask granularity)
+  const unsigned long long* qmask; // per cluster: bit q set when query q takes it (null: every row)
+  const int32_t* row_tok;          // token of each A row (C2T in cluster-major order); null: the row
+  int sample;
+  float tau;
+  uint64_t seed, step;
+  unsigned long long* best;        // B packed arg-maxima (zero between calls)
+  unsigned long long* ticket;      // arrival count (zero between calls)
+  int32_t* out_tok;                // B, or null
+  float* out_logits;               // B x rows indexed by token, or null
+  float* out_keys;                 // B x rows: write the raw products (Stage-1 keys) instead
+  int32_t* cl_list;                // rows/b scratch: gather the clusters some query takes, or null
+  int32_t* cl_count;               // 1 scratch word: their number
+  int32_t* tile_list;              // rows/128 scratch: or stream the 128-row tiles some query takes
+  int32_t* tile_count;             // 1 scratch word: their number (both lists null: every tile)
+  uint32_t* status;
+  int n_tiles;                     // set by the launcher
+};
+bool tc_supported(int elem, int64_t d, int B);
+cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms, cudaStream_t st);
+cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
+                               cudaStream_t st);
+
 // The batch-1 persistent head (fh_head1.cu).
 constexpr int kHead1BndMax = 512;  // boundary-bin keys the distributed selection takes
 

@@ -207,20 +207,29 @@ class _Null:
         pass
 
 
-def max_over_ranks(x: float, dist) -> float:
+def _all_reduce(x: float, op, dist) -> float:
     if not dist:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    # NCCL reduces device tensors; the gloo groups of the CPU tests reduce host tensors
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(x: float, dist) -> float:
+    """The job's time: the slowest rank's."""
+    return _all_reduce(x, torch.distributed.ReduceOp.MAX if dist else None, dist)
 
 
 def sum_over_ranks(x: float, dist) -> float:
-    if not dist:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
-    return float(t.item())
+    """The job's work: every rank's units added up."""
+    return _all_reduce(x, torch.distributed.ReduceOp.SUM if dist else None, dist)
+
+
+def rank_queries(cfg, n: int, rank: int):
+    """Each rank's own pool of queries (replicas only: the ranks share no work and no data)."""
+    return synth.make_queries(cfg, n, seed=cfg.query_seed + 17 * rank)
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -491,7 +500,7 @@ def main():
     idx = synth.make_index(cfg)
     R = Replicated(F, idx)
     B = args.batch
-    Hh = synth.make_queries(cfg, 1024, seed=cfg.query_seed + 17 * rank)
+    Hh = rank_queries(cfg, 1024, rank)
     Hd = F.device_array(Hh, "bf16")
     sampler = ClockSampler(local)
     step = head_step(F, R, Hd, B, cfg.p)

@@ -88,6 +88,7 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
     L.Z = take((size_t)B * D.c * 8);
     L.cluster_of = take((size_t)D.v * 4);
     L.per_draw = take((size_t)B * N * T * 8);
+    L.best = take((size_t)B * 8);
   }
   L.total = off;
   return L;
@@ -501,19 +502,33 @@ fh_status fh_mc_token_prob(const fh_index* idx, const void* H, int B, const int3
   cudaError_t e = cudaMemsetAsync(tickets_of(ws), 0, (size_t)B * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "memset");
   // exact logits over the vocabulary, once per query (S-independent)
-  fh::DenseParams dp = {};
-  dp.E = D.E;
-  dp.H = H;
-  dp.v = D.v;
-  dp.d = D.d;
-  dp.B = B;
-  dp.tau = 1.0f;
-  dp.part = reinterpret_cast<unsigned long long*>(base + L.part);
-  dp.tickets = tickets_of(ws);
-  dp.out_logits = reinterpret_cast<float*>(base + L.z);
-  dp.status = status_of(ws);
-  if ((e = fh::launch_dense(dp, D.dtype, idx->num_sms, st)) != cudaSuccess)
-    return cuda_fail(e, "MC logits launch");
+  if (tc_eligible(idx, B, kTcMinBatchDense)) {  // all v logits of every query, on the tensor cores
+    fh::TcParams tp = {};
+    tp.rows = D.v;
+    tp.d = D.d;
+    tp.B = B;
+    tp.b = 1;
+    tp.best = reinterpret_cast<unsigned long long*>(base + L.best);
+    tp.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, kTcTicketOffset));
+    tp.out_logits = reinterpret_cast<float*>(base + L.z);
+    tp.status = status_of(ws);
+    if ((e = fh::launch_tc_head(D.E, H, tp, idx->num_sms, st)) != cudaSuccess)
+      return cuda_fail(e, "tensor-core logits launch");
+  } else {
+    fh::DenseParams dp = {};
+    dp.E = D.E;
+    dp.H = H;
+    dp.v = D.v;
+    dp.d = D.d;
+    dp.B = B;
+    dp.tau = 1.0f;
+    dp.part = reinterpret_cast<unsigned long long*>(base + L.part);
+    dp.tickets = tickets_of(ws);
+    dp.out_logits = reinterpret_cast<float*>(base + L.z);
+    dp.status = status_of(ws);
+    if ((e = fh::launch_dense(dp, D.dtype, idx->num_sms, st)) != cudaSuccess)
+      return cuda_fail(e, "MC logits launch");
+  }
   // Stage-1 scores
   fh::Stage1Params s1 = stage1_params(idx, H, B, reinterpret_cast<float*>(base + L.s), ws);
   if ((e = fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st,

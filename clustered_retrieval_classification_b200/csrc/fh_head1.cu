@@ -784,13 +784,8 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
   cudaError_t e = cudaSuccess;
 #define FH_H1(EL, M4, NTT, KP)                                                                     \
   do {                                                                                            \
-    static size_t attr_bytes = 0;                                                                 \
-    if (smem > attr_bytes) {                                                                      \
-      e = cudaFuncSetAttribute(k_head1<EL, M4, NTT, KP>,                                          \
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
-      if (e != cudaSuccess) return e;                                                             \
-      attr_bytes = smem;                                                                          \
-    }                                                                                             \
+    e = set_smem_attr(reinterpret_cast<const void*>(k_head1<EL, M4, NTT, KP>), smem);            \
+    if (e != cudaSuccess) return e;                                                               \
     e = cudaLaunchKernelEx(&cfg, k_head1<EL, M4, NTT, KP>, prm);                                  \
   } while (0)
 #define FH_H1_NT(EL, M4)                                  \

@@ -567,14 +567,21 @@ static int ring_slots(uint32_t row_bytes, uint32_t budget) {
 // that repeated launches skip the driver call.
 template <typename Kern>
 static cudaError_t set_smem(Kern kern, size_t bytes) {
+  return set_smem_attr(reinterpret_cast<const void*>(kern), bytes);
+}
+
+cudaError_t set_smem_attr(const void* kernel, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   static std::mutex mu;
-  static std::unordered_map<const void*, size_t> limit;
+  static std::unordered_map<const void*, size_t> limit[kMaxDevices];
   std::lock_guard<std::mutex> lock(mu);
-  const void* key = reinterpret_cast<const void*>(kern);
-  auto it = limit.find(key);
-  if (it != limit.end() && it->second >= bytes) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-  if (e == cudaSuccess) limit[key] = bytes;
+  auto it = limit[dev].find(kernel);
+  if (it != limit[dev].end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) limit[dev][kernel] = bytes;
   return e;
 }
 

@@ -10,6 +10,12 @@ namespace fh {
 
 enum ElemKind : int { kF32 = 0, kBF16 = 1 };
 
+constexpr int kMaxDevices = 64;  // per-device host caches (kernel attributes)
+
+// Raise a kernel's dynamic shared-memory limit to `bytes` on the current device, once per
+// (kernel, device) and size.
+cudaError_t set_smem_attr(const void* kernel, size_t bytes);
+
 // Stage 1: s[q][k] = C[k]·h_q (or the Gumbel key s/τ + G when sample != 0).
 struct Stage1Params {
   const void* C;               // c x d (dense) — or null for INT4

@@ -122,21 +122,25 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 constexpr int kTcRows = 128;                       // E rows per tile (the MMA's N)
 constexpr int kTcWave = 512 / kTcRows;             // tiles whose accumulators fit tensor memory
 
-template <int S>
+template <int S, bool SAMPLE>
 struct TcLayout {
   static constexpr uint32_t kBlk = 128u * 128u;    // one K-block of H or of an E tile: 128 rows x 128 B
   static constexpr uint32_t kHOff = S * kBlk;      // S stages of E blocks, then 2 of H blocks
   static constexpr uint32_t kRowOff = kHOff + 2 * kBlk;            // tile rows: token, mask
   static constexpr uint32_t kClOff = kRowOff + kTcRows * 12u;        // the wave's cluster ids
-  static constexpr uint32_t kBars = kClOff + kTcWave * 16u * 4u + 64u;
+  static constexpr uint32_t kGumOff = kClOff + kTcWave * 16u * 4u;  // sampling: 4 warps x 32 x 32 G
+  static constexpr uint32_t kPairOff = kGumOff + (SAMPLE ? 4u * 32u * 32u * 4u : 0u);  // and pairs
+  static constexpr uint32_t kBars = kPairOff + (SAMPLE ? 4u * 64u * 4u : 0u) + 64u;
   static constexpr uint32_t kDyn = kBars + 1024u + 1024u;          // + barriers, + alignment slack
 };
 
-template <int S>
+// KEYS: write the products (Stage-1 keys) instead of reducing an arg-max; SAMPLE: add the Gumbel
+// term.  Separate instantiations keep each epilogue's code out of the other modes' instruction stream.
+template <int S, bool KEYS, bool SAMPLE>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_tc_head(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmH,
               const TcParams a) {
-  using Lay = TcLayout<S>;
+  using Lay = TcLayout<S, SAMPLE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
   uint32_t* tok_s = reinterpret_cast<uint32_t*>(smem + Lay::kRowOff);                     // 128
@@ -302,6 +306,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // ---------------------------------------------------------------- epilogue: one query per thread
     const int et = tid - 128;             // 0..127: this thread's query and its tile-row duty
     const int q = et;                     // lane q of tensor memory (warp quarter = warp % 4)
+    const bool q_live = q < a.B;          // lanes past the batch take no row but join every warp step
     uint32_t bk = 0u, bt = 0xFFFFFFFFu;   // best key image and its token
     auto group_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
     for (int w = 0; w < n_waves; ++w) {
@@ -335,33 +340,73 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tmem_ld16(tbase + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(v));
           tmem_ld16(tbase + (uint32_t)c0 + 16u, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
           tmem_ld_wait();
-          if (q >= a.B) continue;
-          if (a.out_keys) {  // Stage-1 keys (contiguous rows): s[q][row] or s/τ + G(q, stream 0, row)
+          if constexpr (KEYS) {  // Stage-1 keys (contiguous rows): s[q][row] or s/τ + G(q, stream 0, row)
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const int64_t row = row0 + c0 + i;
-              if (row < a.rows) {
+              if (q < a.B && row < a.rows) {
                 const float z = __uint_as_float(v[i]);
                 a.out_keys[(int64_t)q * a.rows + row] =
-                    a.sample ? z / a.tau + gumbel_from_u32(philox_word(a.seed, a.step, (uint32_t)q, 0u, (uint32_t)row)) : z;
+                    SAMPLE ? z / a.tau + gumbel_from_u32(philox_word(a.seed, a.step, (uint32_t)q, 0u, (uint32_t)row)) : z;
               }
             }
             continue;
           }
+          if constexpr (!SAMPLE) {
+            if (!q_live) continue;  // (uniform per warp when B is a multiple of 32)
+          }
+          float* gum = nullptr;
+          if constexpr (SAMPLE) {
+            // The Gumbel terms G(q, 1, token) of the (row, query) pairs this warp takes in the chunk,
+            // spread evenly over the lanes: a row is taken by few of the warp's 32 queries, so one
+            // evaluation per row and lane would leave most lanes idle.  Lane i lists row i's takers
+            // (a ballot), a scan gives each row its first pair, and pair k goes to lane k % 32.
+            uint32_t* bal_s = reinterpret_cast<uint32_t*>(smem + Lay::kPairOff) + (warp & 3) * 64;
+            gum = reinterpret_cast<float*>(smem + Lay::kGumOff) + (warp & 3) * 1024;
+            uint32_t my_bal = 0u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const uint32_t bi = __ballot_sync(0xFFFFFFFFu, q_live && ((msk_s[c0 + i] >> q) & 1ull));
+              if (lane == i) my_bal = bi;
+            }
+            const uint32_t my_cnt = __popc(my_bal);
+            uint32_t incl = my_cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+              if (lane >= o) incl += y;
+            }
+            bal_s[lane] = my_bal;
+            bal_s[32 + lane] = incl - my_cnt;  // the row's first pair
+            const uint32_t pairs = __shfl_sync(0xFFFFFFFFu, incl, 31);
+            __syncwarp();
+            for (uint32_t k = (uint32_t)lane; k < pairs; k += 32u) {
+              int i = 0;  // the last row whose first pair is <= k
+#pragma unroll
+              for (int step = 16; step > 0; step >>= 1)
+                if (i + step < 32 && bal_s[32 + i + step] <= k) i += step;
+              const uint32_t ql = __fns(bal_s[i], 0u, (int)(k - bal_s[32 + i]) + 1);
+              const uint32_t qq = (uint32_t)(32 * (warp & 3)) + ql;
+              gum[i * 32 + (int)ql] = gumbel_from_u32(philox_word(a.seed, a.step, qq, 1u, tok_s[c0 + i]));
+            }
+            __syncwarp();
+          }
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
             const unsigned long long mk = msk_s[c0 + i];
-            if (!((mk >> q) & 1ull)) continue;
+            if (!q_live || !((mk >> q) & 1ull)) continue;
             const uint32_t tk = tok_s[c0 + i];
             const float z = __uint_as_float(v[i]);
             if (a.out_logits) a.out_logits[(int64_t)q * a.rows + tk] = z;
-            const float val = a.sample ? z / a.tau + gumbel_from_u32(philox_word(a.seed, a.step, (uint32_t)q, 1u, tk)) : z;
+            float val = z;
+            if constexpr (SAMPLE) val = z / a.tau + gum[i * 32 + lane];
             const uint32_t key = float_key(val);
             if (key > bk || (key == bk && tk < bt)) {
               bk = key;
               bt = tk;
             }
           }
+          if constexpr (SAMPLE) __syncwarp();  // the warp's G buffer is rewritten for the next chunk
         }
         group_sync();  // the tile rows are rewritten for the next tile
       }
@@ -369,7 +414,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty);  // the next wave may overwrite the accumulators
     }
-    if (!a.out_keys && q < a.B && bk) atomicMax(a.best + q, ((unsigned long long)bk << 32) | (unsigned long long)(~bt));
+    if (!KEYS && q < a.B && bk) atomicMax(a.best + q, ((unsigned long long)bk << 32) | (unsigned long long)(~bt));
   }
 
   // ------------------------------------------------------------------ teardown and the grid arg-max
@@ -379,7 +424,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512u) : "memory");
   }
-  if (a.out_keys) return;  // Stage-1 keys: nothing to reduce
+  if constexpr (KEYS) return;  // Stage-1 keys: nothing to reduce
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -488,21 +533,15 @@ bool make_map(CUtensorMap* m, const void* base, int64_t d, int64_t rows, uint32_
 cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, const TcParams& p, int num_sms,
                           cudaStream_t st) {
   constexpr int S = (int)((kTcSmemBudget - 2u * 16384u - 4096u) / 16384u);
-  using Lay = TcLayout<S>;
-  static std::mutex mu;
-  static bool attr_set = false;
-  {
-    std::lock_guard<std::mutex> lock(mu);
-    if (!attr_set) {
-      cudaError_t e = cudaFuncSetAttribute(k_tc_head<S>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           (int)Lay::kDyn);
-      if (e != cudaSuccess) return e;
-      attr_set = true;
-    }
-  }
+  const bool keys = p.out_keys != nullptr, sample = p.sample != 0;
+  auto kern = keys ? (sample ? k_tc_head<S, true, true> : k_tc_head<S, true, false>)
+                   : (sample ? k_tc_head<S, false, true> : k_tc_head<S, false, false>);
+  const uint32_t dyn = sample ? TcLayout<S, true>::kDyn : TcLayout<S, false>::kDyn;
+  cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(kern), dyn);
+  if (e != cudaSuccess) return e;
   // every SM when the tiles are listed on the device; otherwise no more CTAs than tiles
   const int grid = (p.cl_list || p.tile_list || p.n_tiles >= num_sms) ? num_sms : p.n_tiles;
-  k_tc_head<S><<<grid, kTcThreads, Lay::kDyn, st>>>(mE, mH, p);
+  kern<<<grid, kTcThreads, dyn, st>>>(mE, mH, p);
   return cudaGetLastError();
 }
 

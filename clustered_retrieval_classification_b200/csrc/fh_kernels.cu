@@ -141,6 +141,85 @@ __global__ void __launch_bounds__(kThreads) k_stage1_int4(const Stage1Params prm
                    K, row_bytes, src, body, prm.status);
 }
 
+// Several queries per block: each INT4 row is read and each group decoded once for QB queries.  The
+// queries' h sit in shared memory as fp32, transposed so that the 32 lanes (32 consecutive groups)
+// read consecutive 16-byte chunks: hT[q][e/4][group][e%4] for column 32*group + e.
+template <int MCH, int QB>
+__global__ void __launch_bounds__(kThreads) k_stage1_int4_mq(const Stage1Params prm, int K,
+                                                             int rows_max) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid < prm.n_tickets) prm.tickets_to_clear[tid] = 0u;
+
+  const int q0 = blockIdx.y * QB;
+  const int nq = min(QB, prm.B - q0);
+  const int64_t d = prm.d;
+  const uint32_t row_bytes = (uint32_t)(d / 2);
+  const int nch = (int)(d / 32);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
+  uint16_t* sc_s = reinterpret_cast<uint16_t*>(smem + 1024);
+  float* hT = reinterpret_cast<float*>(smem + 1024 + (((size_t)rows_max * nch * 2 + 127) / 128) * 128);
+  uint8_t* ring = reinterpret_cast<uint8_t*>(hT + (size_t)QB * d);
+
+  const int64_t lo = prm.c * blockIdx.x / gridDim.x;
+  const int64_t hi = prm.c * (blockIdx.x + 1) / gridDim.x;
+  if (tid < kWarps * K) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
+  for (int64_t i = tid; i < (hi - lo) * nch; i += kThreads) sc_s[i] = prm.scales[lo * nch + i];
+  const uint16_t* H = static_cast<const uint16_t*>(prm.H);
+  for (int64_t i = tid; i < (int64_t)QB * d; i += kThreads) {
+    const int q = (int)(i / d), col = (int)(i % d);
+    const int ch = col >> 5, e = col & 31;
+    hT[(((size_t)q * 8 + (e >> 2)) * nch + ch) * 4 + (e & 3)] =
+        q < nq ? __uint_as_float((uint32_t)H[(size_t)(q0 + q) * d + col] << 16) : 0.0f;
+  }
+  __syncthreads();
+  const uint32_t hT_addr = smem_addr(hT);
+
+  auto src = [&](int64_t k) { return prm.q4 + (size_t)k * row_bytes; };
+  auto body = [&](int64_t k, uint32_t row_s) {
+    float acc[QB];
+#pragma unroll
+    for (int q = 0; q < QB; ++q) acc[q] = 0.0f;
+#pragma unroll
+    for (int m = 0; m < MCH; ++m) {
+      const int ch = lane + 32 * m;
+      if (ch < nch) {
+        float dq[32];
+        int4_decode32(lds_v4(row_s + ch * 16), dq);
+        const float scale = __uint_as_float((uint32_t)sc_s[(k - lo) * nch + ch] << 16);
+#pragma unroll
+        for (int q = 0; q < QB; ++q) {
+          float g = 0.0f;
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const uint4 hv = lds_v4(hT_addr + (uint32_t)((((size_t)q * 8 + e4) * nch + ch) * 16));
+            g = fmaf(dq[4 * e4 + 0], __uint_as_float(hv.x), g);
+            g = fmaf(dq[4 * e4 + 1], __uint_as_float(hv.y), g);
+            g = fmaf(dq[4 * e4 + 2], __uint_as_float(hv.z), g);
+            g = fmaf(dq[4 * e4 + 3], __uint_as_float(hv.w), g);
+          }
+          acc[q] = fmaf(scale, g, acc[q]);
+        }
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < QB; ++q) {
+      const float s = warp_sum(acc[q]);
+      if (lane == 0 && q < nq) {
+        float out = s;
+        if (prm.sample)
+          out = s / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)(q0 + q),
+                                                          prm.rng_stream, (uint32_t)k));
+        prm.out[(size_t)(q0 + q) * prm.c + k] = out;
+      }
+    }
+  };
+  warp_stream_rows(lo + warp, hi, kWarps, lane, ring + (size_t)warp * K * row_bytes, bars + warp * K,
+                   K, row_bytes, src, body, prm.status);
+}
+
 // ============================================================================ single steps
 
 __global__ void k_gumbel_keys(const float* s, float* keys, int B, int64_t c, float tau, uint64_t seed,
@@ -596,8 +675,24 @@ cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_s
     const int nch = (int)(prm.d / 32);
     const size_t smem = 1024 + (((size_t)rows_max * nch * 2 + 127) / 128) * 128 +
                         (size_t)kWarps * K * row_bytes;
-    dim3 grid(G, prm.B);
     cudaError_t e;
+    if (prm.B > 1) {  // eight queries per block
+      constexpr int QB = 8;
+      const size_t smem_mq = 1024 + (((size_t)rows_max * nch * 2 + 127) / 128) * 128 +
+                             (size_t)QB * prm.d * 4 + (size_t)kWarps * K * row_bytes;
+      dim3 grid_mq(G, (prm.B + QB - 1) / QB);
+#define FH_S1Q(M)                                                                   \
+  do {                                                                              \
+    if ((e = set_smem(k_stage1_int4_mq<M, QB>, smem_mq)) != cudaSuccess) return e;  \
+    k_stage1_int4_mq<M, QB><<<grid_mq, kThreads, smem_mq, st>>>(prm, K, rows_max);  \
+  } while (0)
+      if (nch <= 32) FH_S1Q(1);
+      else if (nch <= 64) FH_S1Q(2);
+      else FH_S1Q(4);
+#undef FH_S1Q
+      return cudaGetLastError();
+    }
+    dim3 grid(G, prm.B);
     if (nch <= 32) {
       if ((e = set_smem(k_stage1_int4<1>, smem)) != cudaSuccess) return e;
       k_stage1_int4<1><<<grid, kThreads, smem, st>>>(prm, K, rows_max);

@@ -97,4 +97,19 @@ __device__ __forceinline__ float int4_group_dot(const uint4 w, const float* hg) 
   return acc;
 }
 
+// The 32 values of one INT4 group (columns 0..31, low nibble = even column), decoded exactly.
+__device__ __forceinline__ void int4_decode32(const uint4 w, float (&dq)[32]) {
+  const uint32_t words[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t even = (words[i] & 0x0F0F0F0Fu) ^ 0x08080808u;
+    const uint32_t odd = ((words[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      dq[8 * i + 2 * j] = __uint_as_float(__byte_perm(even, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
+      dq[8 * i + 2 * j + 1] = __uint_as_float(__byte_perm(odd, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
+    }
+  }
+}
+
 }  // namespace fh

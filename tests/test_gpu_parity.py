@@ -116,11 +116,13 @@ def test_stage1_scores(fh, orc, tiny, mid):
         assert np.abs(g - o).max() <= LOGIT_TOL
 
 
-def test_stage1_scores_int4(fh, orc, mid_int4):
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_stage1_scores_int4(fh, orc, mid_int4, B):
+    """One query per block at B = 1; eight per block otherwise (a partial group at B = 3)."""
     idx, H = mid_int4
     I = load(fh, idx, int4=True)
-    g = fh.stage1_scores(I, dev(H[:3], "bf16")).cpu().numpy()
-    o = orc.stage1_scores(None, "bf16", H[:3], idx.c, idx.d, q4=idx.C_q4, scales=idx.C_scales)
+    g = fh.stage1_scores(I, dev(H[:B], "bf16")).cpu().numpy()
+    o = orc.stage1_scores(None, "bf16", H[:B], idx.c, idx.d, q4=idx.C_q4, scales=idx.C_scales)
     assert np.abs(g - o).max() <= LOGIT_TOL
 
 

@@ -41,7 +41,7 @@ PAGES_TOKENS_PER_S = 1.0 / 0.40e-3
 # sources they were taken on (sha1 of the csrc files); null otherwise.
 TRAFFIC = {
     # profiles/k_head1_llama_batch1.md: dram__bytes_read.sum + dram__bytes_write.sum of one launch
-    (1, "8df018758907"): 66_547_200 + 948_224,
+    (1, "344c7ac967af"): 66_547_456 + 565_760,
 }
 
 L2_FLUSH_BYTES = 256 << 20

@@ -41,16 +41,21 @@ PAGES_TOKENS_PER_S = 1.0 / 0.40e-3
 # sources they were taken on (sha1 of the csrc files); null otherwise.
 TRAFFIC = {
     # profiles/k_head1_llama_batch1.md: dram__bytes_read.sum + dram__bytes_write.sum of one launch
-    (1, "344c7ac967af"): 66_547_456 + 565_760,
+    (1, "d986aeee06e1"): 66_547_456 + 565_760,
 }
 
 L2_FLUSH_BYTES = 256 << 20
 
 
-def csrc_hash() -> str:
+# The sources the batch-1 head kernel is compiled from (its parameters, helpers and selection).
+HEAD1_SOURCES = ("fh_head1.cu", "fh_device.cuh", "fh_select.cuh", "fh_stream.cuh", "fh_kernels.cuh")
+
+
+def csrc_hash(files=HEAD1_SOURCES) -> str:
+    """sha1 of the kernel sources a traffic figure was taken on (the batch-1 head's, by default)."""
     h = hashlib.sha1()
     d = os.path.join(ROOT, "clustered_retrieval_classification_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in sorted(files):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:12]

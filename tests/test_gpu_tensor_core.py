@@ -73,11 +73,13 @@ def small(fh):
     return idx, synth.make_queries(SMALL, 64), fh.index_from_host(idx.E, idx.C, idx.C2T, "bf16")
 
 
-@pytest.mark.parametrize("B", [4, 16, 33, 64])
+@pytest.mark.parametrize("B", [4, 8, 12, 16, 33, 64])
 @pytest.mark.parametrize("sample", [False, True])
 def test_flashhead_batched_without_debug(fh, orc, small, B, sample):
     """Tokens equal the oracle's wherever its set and token margins decide them; every other token
-    comes from a cluster the oracle selected or one within the margin of its threshold."""
+    comes from a cluster the oracle selected or one within the margin of its threshold.  B = 4 runs on
+    CUDA cores, B = 8 and 12 gather the selected clusters into tensor-core tiles, B >= 16 streams
+    the tiles that hold a selected cluster."""
     idx, H, I = small
     cfg = idx.cfg
     Hd = dev(H[:B], "bf16")

@@ -27,7 +27,6 @@ namespace fh {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kSelThreads = 512;
 
 // ============================================================================ Stage 1 (dense C)
 

@@ -21,7 +21,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
+#include <mutex>  // std::call_once
 
 #include "fh_device.cuh"
 #include "fh_kernels.cuh"

@@ -54,6 +54,7 @@ def lib():
         L.orc_mc.argtypes = [_p, _p, _i32, _p, _p, _i32, _p, _i64, _i64, _i64, _i64, _p, _i32, _p,
                              _i32, _i32, _f64, _i64, _i64, _u64, _p, _p, _p]
         L.orc_num_threads.restype = _i32
+        L.orc_set_num_threads.argtypes = [_i32]
         _lib = L
     return _lib
 
@@ -68,6 +69,11 @@ def _c(a, dtype=None):
 
 def num_threads() -> int:
     return int(lib().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the oracle's parallel loops use from now on (timing only; results do not change)."""
+    lib().orc_set_num_threads(int(n))
 
 
 # ----------------------------------------------------------------------------- Philox

@@ -379,6 +379,16 @@ void orc_mc(const void* E, const void* C, int dtype, const uint8_t* q4, const ui
   free(s); free(z);
 }
 
+/* Threads for the next parallel regions (n >= 1; no effect without OpenMP). */
+void orc_set_num_threads(int n) {
+#ifdef _OPENMP
+  extern void omp_set_num_threads(int);
+  if (n >= 1) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
 /* Number of threads the OpenMP runtime will use (1 without OpenMP). */
 int orc_num_threads(void) {
 #ifdef _OPENMP

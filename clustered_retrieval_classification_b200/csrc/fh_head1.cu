@@ -6,25 +6,30 @@
 //
 //   1. Stage 1: each block loads h, then bulk-copies its share of centroid rows (C, or the INT4
 //      nibbles) into its shared-memory ring at once, computes s = C·h (or the Gumbel key s/τ + G),
-//      writes the keys, and adds each key to a 1024-bin histogram in global memory.  The bins cover a
-//      range fixed in advance from ‖h‖ (unit centroids give |s| <= ‖h‖; the Gumbel term lies in
+//      writes the keys, and counts each key in a 1024-bin block histogram.  The bins cover a range
+//      fixed in advance from ‖h‖ (unit centroids give |s| <= ‖h‖; the Gumbel term lies in
 //      [-2.9, 16.7]); keys outside are clamped into the end bins, so the binning is monotone for any
-//      input and only its resolution depends on the range.
-//   2. Grid barrier (monotonic 64-bit arrival counter, bounded wait).
-//   3. Selection, redundantly in every block (FlashHead notes, Module 2): the histogram gives the
-//      boundary bin; clusters above it are certain and their Stage-2 rows are issued at once; the
-//      boundary bin is then resolved exactly (rank, or radix passes when crowded) while they fly.
+//      input and only its resolution depends on the range.  The block adds its counts to the global
+//      histogram with returning release adds, which give every key a distinct position in its bin.
+//   2. Grid barrier = histogram poll: every block polls the summed histogram until its counts reach c
+//      (bounded wait); the last poll holds the counts, the boundary bin follows by a block scan.
+//   3. Selection without a global list (FlashHead notes, Module 2): a certain cluster's rank in the
+//      Stage-2 list is (keys in higher bins) + (its position in its bin); the block that scored it
+//      writes its id at that rank as one 64-bit word tagged with the call's generation, and the
+//      boundary bin's (key, id) pairs likewise.  Block 0 ranks the boundary bin exactly (warp rank,
+//      or radix passes when crowded — then every block selects on all keys) and writes the ids it
+//      selects at the remaining ranks.  Each block polls only the words of its own rows, all before
+//      it issues any Stage-2 copy.
 //   4. Stage 2 (FlashHead notes, Module 1 and Figure 1): the block streams its slice of the p·b
 //      candidate rows, each together with the 16-byte C2T chunk holding its token id, computes the
 //      exact logits and keeps the arg-max of z (greedy, Eq. 2) or of z/τ + G' (sampling, Eq. 3).
 //   5. Each block folds its best (value, token) into one 64-bit atomicMax; the last block to arrive
-//      writes the token and clears the histogram and the maximum for the next call.
+//      writes the token and clears the histogram, the selection words and the maximum.
 //
-// No global load waits behind the bulk copies: every small dependent load (h, INT4 scales, keys,
-// histogram) is issued before the block's copies, and token ids arrive inside the row copies.
-// Stage-2 slots are ordered "certain clusters by ascending id, then the boundary clusters taken, by
-// ascending id"; the arg-max does not depend on the order, and the optional debug outputs are written
-// in the canonical ascending order.
+// No small global load waits behind the bulk copies: h and the INT4 scales are loaded before the
+// Stage-1 copies, the rank words are polled before the Stage-2 copies, and token ids arrive inside the
+// row copies.  Stage-2 slots follow the rank order; the arg-max does not depend on it, and the
+// optional debug outputs are written in the canonical ascending order.
 #include "fh_device.cuh"
 #include "fh_kernels.cuh"
 #include "fh_select.cuh"

@@ -8,10 +8,14 @@
 //
 // Kernels:
 //   k_stage1<E,QB>   s = C·h for QB queries per block; optional Gumbel-key epilogue   (Stage 1)
-//   k_stage1_int4<M> the same from INT4 centroids with BF16 group scales               (Stage 1, INT4)
+//   k_stage1_int4<M> the same from INT4 centroids with BF16 group scales, one query    (Stage 1, INT4)
+//   k_stage1_int4_mq<M,QB> INT4 for QB queries per block, each group decoded once      (Stage 1, INT4)
 //   k_select<KPT>    top-p per query                                                    (selection)
+//   k_build_qmask    per-cluster bit masks of the queries that selected it              (tensor-core Stage 2)
 //   k_rows<E,MODE,KPT> candidates (fused selection or given sets) or all rows (dense):
 //                    dot, arg-max / Gumbel-max, partial results, last-block reduction   (Stage 2, dense)
+// The batch-1 head is one persistent kernel (fh_head1.cu); batched BF16 heads run on the tensor
+// cores (fh_tc.cu).
 //   k_gather, k_cand_logits, k_gumbel_keys, k_philox                                    (single steps)
 //   k_validate_c2t, k_build_perm                                                        (index load)
 //   k_mc_*                                                                              (Monte Carlo)

@@ -125,7 +125,7 @@ size_t fh_index_load_ws_bytes(const fh_index_desc* desc);
    (FlashHead notes, Module 1: every cluster holds exactly b tokens, so C2T is a dense c×b tensor).
    Builds E_perm when desc->E_perm is non-NULL.  ws: device scratch of fh_index_load_ws_bytes bytes.
    Synchronises `stream`.  Returns FH_ERR_INDEX if C2T is not a permutation; *out is then NULL.
-   The handle holds host metadata only (shapes, pointers, TMA descriptors). */
+   The handle holds host metadata only (shapes and pointers). */
 fh_status fh_index_load(const fh_index_desc* desc, void* ws, size_t ws_bytes, fh_stream stream,
                         fh_index** out);
 
@@ -141,7 +141,8 @@ size_t fh_workspace_bytes(const fh_index* idx, int op, int B, int p, int T, int6
 
 /* Read and clear the status word of a workspace (synchronises `stream`).  Returns FH_OK, or the
    device-side error a previous call recorded there (FH_ERR_TIMEOUT, FH_ERR_INDEX); after an error
-   the workspace's control block is zeroed again so that it can be reused. */
+   the workspace's control block is zeroed again so that it can be reused (its call generation moves
+   past every tag a failed call may have left in the selection words). */
 fh_status fh_ws_status(void* ws, fh_stream stream);
 
 /* Thread-local description of the last error returned on this thread ("" if none). */
@@ -153,7 +154,12 @@ const char* fh_last_error(void);
    H: device, B x d, dtype.  1 <= B <= FH_MAX_BATCH, 1 <= p <= c.
    For each query q: S_q = the p clusters with the largest s_q = C·h_q; candidates = the p·b tokens of
    S_q through C2T; out_tok[q] = argmax of their exact logits z_t = E[t]·h_q (fp32 accumulation).
-   out_tok: device, B int32.  dbg: optional intermediate outputs, or NULL. */
+   out_tok: device, B int32.  dbg: optional intermediate outputs, or NULL.
+   Execution (all paths compute the same thing): B = 1 runs one persistent kernel; BF16 batches of 8
+   or more run Stage 1 and Stage 2 on the tensor cores, reading each needed E row once for the whole
+   batch (debug outputs force the per-query Stage 2 instead); other batches run per-query CUDA-core
+   kernels.  The paths sum the fp32 logits in different orders, so their tokens can differ only where
+   two candidates' logits are within that rounding (~1e-6 relative); each path is deterministic. */
 fh_status fh_head_greedy(const fh_index* idx, const void* H, int B, int p, int32_t* out_tok,
                          void* ws, size_t ws_bytes, fh_stream stream, const fh_debug_out* dbg);
 
@@ -178,7 +184,8 @@ fh_status fh_mc_token_prob(const fh_index* idx, const void* H, int B, const int3
 
 /* Dense head over the whole vocabulary (FlashHead notes, Eq. 1–3): z = E·h_q for every token.
    sample == 0: out_tok[q] = argmax z; sample != 0: argmax of z_t/τ + G(seed, step, q, FH_RNG_STAGE2, t).
-   out_logits: device B x v fp32 logits z, or NULL. */
+   out_logits: device B x v fp32 logits z, or NULL.  BF16 batches of 2 or more run on the tensor
+   cores (one pass over E for the whole batch); batch 1 streams E on CUDA cores. */
 fh_status fh_dense_head(const fh_index* idx, const void* H, int B, int sample, float tau,
                         uint64_t seed, uint64_t step, int32_t* out_tok, float* out_logits,
                         void* ws, size_t ws_bytes, fh_stream stream);

@@ -224,6 +224,14 @@ def quantize_int4_g32(x: np.ndarray):
     return np.ascontiguousarray(packed), np.ascontiguousarray(scales_bits)
 
 
+def shift_centroids(C: np.ndarray, t: float) -> np.ndarray:
+    """C - t * mean(C) (rows), in float64: the offline reparameterisation of the centroids before
+    INT4 quantisation.  Every Stage-1 score of a query moves by the same t * mean(C)·h, so the top-p
+    set and softmax(s/τ) are unchanged in exact arithmetic; only the quantisation error changes."""
+    C = np.asarray(C, dtype=np.float64)
+    return C - t * C.mean(axis=0, keepdims=True)
+
+
 def make_queries(cfg: HeadConfig, n: int, seed: int | None = None) -> np.ndarray:
     """n hidden vectors h ~ N(0, I/d) * h_scale, rounded to the storage dtype."""
     rng = np.random.Generator(np.random.PCG64(cfg.query_seed if seed is None else seed))

@@ -362,6 +362,29 @@ def test_batch1_without_debug_outputs_on_one_workspace(fh, orc, mid):
     assert checked >= 2
 
 
+def test_bounded_wait_times_out_and_workspace_recovers(fh, mid):
+    """Failure detection without a fault: one histogram bin of the workspace is pre-set so that the
+    batch-1 kernel's grid barrier (a bounded poll of the histogram until its counts reach c) can never
+    complete.  Every block gives up after 0.5 s with no copy in flight; the call records
+    FH_ERR_TIMEOUT, fh_ws_status reports it once and resets the control block, and the same workspace
+    then gives the right token again."""
+    idx, H = mid
+    cfg = idx.cfg
+    I = load(fh, idx)
+    Hd = dev(H[:1], cfg.dtype)
+    ws = torch.zeros(I.workspace_bytes(fh.FH_OP_GREEDY, 1, cfg.p), dtype=torch.uint8, device=DEV)
+    ref = fh.head_greedy(I, Hd, cfg.p, ws=torch.zeros_like(ws)).item()
+    ws[1024:1028] = 0xFF                       # bin 0 = 2^32 - 1: the counts now sum to c - 1
+    fh.head_greedy(I, Hd, cfg.p, ws=ws)
+    torch.cuda.synchronize()
+    with pytest.raises(fh.FlashHeadError) as e:
+        fh.ws_status(ws)
+    assert e.value.status == 6                 # FH_ERR_TIMEOUT
+    fh.ws_status(ws)                           # reported once, then clear
+    assert fh.head_greedy(I, Hd, cfg.p, ws=ws).item() == ref
+    fh.ws_status(ws)
+
+
 def test_workspace_status_clean(fh, mid):
     idx, H = mid
     I = load(fh, idx)

@@ -515,6 +515,47 @@ def ncu_case(args):
     return 0
 
 
+def pc_sweep(args):
+    """The p/c trade-off of the pages (FlashHead summary, Table 7): the batch-1 greedy head over the
+    Llama-shaped vocabulary (v = 128256, d = 2048) at three cluster counts and three probe counts.
+    Timed like the headline (CUDA graph of back-to-back calls over 8 replicas, inputs larger than
+    L2); 16 queries per point are also checked against the oracle."""
+    import oracle
+    from clustered_retrieval_classification_b200 import flashhead as F
+    F.load()
+    peak, peak_kind = measured_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    T = Timer(False, lambda: flush_buf.fill_(1))
+    base = synth.CONFIGS["llama"]
+    K, W = min(args.steps, 512), max(args.warmup, 3)
+    points = {}
+    for c in (4008, 8016, 16032):
+        cfg = synth.scaled(base, v=base.v, c=c, d=base.d, p=base.p, name=f"llama-c{c}")
+        idx = synth.make_index(cfg)
+        R = Replicated(F, idx)
+        Hh = synth.make_queries(cfg, 1024)
+        Hd = F.device_array(Hh, "bf16")
+        for p in (128, 256, 512):
+            t, n, mode = T.b2b(head_step(F, R, Hd, 1, p), K, W)
+            us = 1e3 * t / n
+            by = costmodel.head_bytes(cfg.v, cfg.d, c, p, 1, p, 2)
+            gbs = by / (us * 1e-6) / 1e9
+            tok = np.array([int(F.head_greedy(R[0], Hd[q:q + 1], p).item()) for q in range(16)])
+            o = oracle.head(idx, Hh[:16], p)
+            decided = (o["set_margin"] > 4e-3) & (o["tok_margin"] > 4e-3)
+            points[f"c{c}_p{p}"] = {"b": cfg.b, "us_per_call": us, "tokens_per_s": 1e6 / us,
+                                    "bytes": by, "gbs": gbs, "frac": gbs / peak, "timing": mode,
+                                    "oracle_tokens_equal": int(np.sum(tok == o["tok"])),
+                                    "oracle_decided": int(np.sum(decided)),
+                                    "oracle_decided_equal": int(np.sum((tok == o["tok"]) & decided))}
+        del R
+        torch.cuda.empty_cache()
+    print(json.dumps({"pc_sweep": points, "peak": peak, "peak_kind": peak_kind,
+                      "workload": "llama-3.2-1b-shaped vocabulary v=128256 d=2048, batch-1 greedy",
+                      "queries_checked_per_point": 16}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -529,12 +570,18 @@ def main():
                          "exit: the case the committed ncu captures use")
     ap.add_argument("--ncu-what", default="greedy", choices=["greedy", "dense", "sample"],
                     help="with --ncu-case: which head (at --batch queries) to call")
+    ap.add_argument("--pc-sweep", action="store_true",
+                    help="time the batch-1 greedy head of the Llama-shaped vocabulary at "
+                         "c in {4008, 8016, 16032} x p in {128, 256, 512} (with oracle token checks), "
+                         "print one JSON line and exit")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         return run_reference(args)
     if args.ncu_case:
         return ncu_case(args)
+    if args.pc_sweep:
+        return pc_sweep(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

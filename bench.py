@@ -10,10 +10,13 @@ before each call are reported alongside.
 
 The sweep (on by default) times the other rows of the path at their own shapes: batches 4/16/64,
 the in-run dense head, sampling, the Gemma-shaped INT4 Stage 1 and the Qwen-shaped Monte Carlo
-marginal.  `--impl reference` times the CPU oracle (fp64, host cores) on the same workload.
+marginal.  With the CPU leg on (default) the line also carries the oracle's throughput on the host
+cores and GPU-vs-oracle token counts on the oracle's sample.  `--impl reference` times the CPU oracle (fp64, host cores) on the same workload.
 
 Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under torch.distributed.run,
-one independent replica per GPU (the head does not shard), time = max over ranks.
+one independent replica per GPU (the whole index fits one GPU and a vocabulary split would add two
+collective latencies per call, so the head does not shard), time = max over ranks.  Other modes:
+--ncu-case (untimed calls for ncu captures) and --pc-sweep (the p/c trade-off at batch 1).
 """
 
 import argparse

@@ -674,8 +674,8 @@ def main():
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": B * cfg.d * 2,
                 "d2h_bytes_per_step": B * 4, "us_per_call": 1e3 * e2e_ms / args.steps},
         # our kernels per call: batch 1 = the one persistent kernel; batches on the tensor cores =
-        # Stage 1, selection, masks, work list, Stage 2; below 8 queries = Stage 1, selection, Stage 2
-        "gpu_launches": calls * (1 if B == 1 else (5 if B >= 8 else 3)),
+        # Stage 1, selection, masks, work list, Stage 2; below 12 queries = Stage 1, selection, Stage 2
+        "gpu_launches": calls * (1 if B == 1 else (5 if B >= 12 else 3)),
         "clocks": sampler.summary(),
     }
     if not args.no_sweep and rank == 0:

@@ -155,7 +155,7 @@ const char* fh_last_error(void);
    For each query q: S_q = the p clusters with the largest s_q = C·h_q; candidates = the p·b tokens of
    S_q through C2T; out_tok[q] = argmax of their exact logits z_t = E[t]·h_q (fp32 accumulation).
    out_tok: device, B int32.  dbg: optional intermediate outputs, or NULL.
-   Execution (all paths compute the same thing): B = 1 runs one persistent kernel; BF16 batches of 8
+   Execution (all paths compute the same thing): B = 1 runs one persistent kernel; BF16 batches of 12
    or more run Stage 1 and Stage 2 on the tensor cores, reading each needed E row once for the whole
    batch (debug outputs force the per-query Stage 2 instead); other batches run per-query CUDA-core
    kernels.  The paths sum the fp32 logits in different orders, so their tokens can differ only where

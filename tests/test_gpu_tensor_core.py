@@ -1,7 +1,7 @@
 """Parity of the tensor-core (tcgen05) path with the fp64 oracle.
 
-Batches of 2..64 queries on a BF16 index take the tensor-core kernel: the dense head for every such
-batch, FlashHead Stage 2 when no debug outputs are requested.  Sizes span several 128-row tiles with a
+Batches of 2..64 queries on a BF16 index take the tensor-core kernel for the dense head; FlashHead
+takes it from 12 queries on when no debug outputs are requested.  Sizes span several 128-row tiles with a
 ragged tail (v = 32064), batches that are not a multiple of the 16-query MMA width, and a d that is
 not a multiple of the 64-element K-block.  Logits are compared element by element (|Δ| <= 2e-3);
 token ids must be identical wherever the oracle's margins decide them (parity.MARGIN)."""
@@ -77,9 +77,9 @@ def small(fh):
 @pytest.mark.parametrize("sample", [False, True])
 def test_flashhead_batched_without_debug(fh, orc, small, B, sample):
     """Tokens equal the oracle's wherever its set and token margins decide them; every other token
-    comes from a cluster the oracle selected or one within the margin of its threshold.  B = 4 runs on
-    CUDA cores, B = 8 and 12 gather the selected clusters into tensor-core tiles, B >= 16 streams
-    the tiles that hold a selected cluster."""
+    comes from a cluster the oracle selected or one within the margin of its threshold.  B = 4 and 8
+    run the per-query CUDA-core Stage 2, B = 12 gathers the selected clusters into tensor-core tiles,
+    B >= 16 streams the tiles that hold a selected cluster."""
     idx, H, I = small
     cfg = idx.cfg
     Hd = dev(H[:B], "bf16")

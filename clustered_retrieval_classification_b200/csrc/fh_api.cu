@@ -309,6 +309,17 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
 
 }  // namespace
 
+namespace fh {
+// The error reporter of the other C ABI files (the k-means builder): sets fh_last_error().
+fh_status report(fh_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return st;
+}
+}  // namespace fh
+
 // Used by fh_static.cu to report its own errors through fh_last_error().
 fh_status fh_internal_set_error(fh_status st, const char* msg) { return fail(st, "%s", msg); }
 

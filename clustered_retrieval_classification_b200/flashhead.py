@@ -43,6 +43,16 @@ class DebugOut(ct.Structure):
     _fields_ = [("sel", ct.c_void_p), ("cand_tok", ct.c_void_p), ("cand_logit", ct.c_void_p)]
 
 
+class KmeansArgs(ct.Structure):
+    """fh_kmeans_args (include/fh_kmeans.h)."""
+    _fields_ = [("E", ct.c_void_p), ("dtype", ct.c_int32), ("v", ct.c_int64), ("d", ct.c_int64),
+                ("c", ct.c_int64), ("iters", ct.c_int32), ("eps", ct.c_float),
+                ("max_rounds", ct.c_int64), ("init_tokens", ct.c_void_p), ("C_in", ct.c_void_p),
+                ("labels_in", ct.c_void_p), ("labels", ct.c_void_p), ("C2T", ct.c_void_p),
+                ("C", ct.c_void_p), ("C_bf16", ct.c_void_p), ("objective", ct.c_void_p),
+                ("prices", ct.c_void_p), ("iters_done", ct.c_int32), ("rounds", ct.c_int64)]
+
+
 _lib = None
 _p, _i, _i64, _u32, _u64, _f, _sz = (ct.c_void_p, ct.c_int, ct.c_int64, ct.c_uint32, ct.c_uint64,
                                       ct.c_float, ct.c_size_t)
@@ -65,6 +75,10 @@ SIGNATURES = {
     "fh_candidate_logits": (_i, [_p, _p, _i, _p, _i64, _p, _p]),
     "fh_philox_u32": (_i, [_u64, _u64, _u32, _u32, _i64, _p, _p]),
     "fh_head_greedy_static": (_i, [_p, _p, _i, _p, _p]),
+    "fh_kmeans_ws_bytes": (_sz, [_i64, _i64, _i64]),
+    "fh_kmeans_build": (_i, [_p, _p, _sz, _p]),
+    "fh_kmeans_assign": (_i, [_p, _p, _sz, _p]),
+    "fh_kmeans_update": (_i, [_p, _p, _sz, _p]),
 }
 
 
@@ -324,3 +338,80 @@ def index_from_host(E, C, C2T, dtype: str, C_q4=None, C_scales=None, int4=False,
     q4 = device_array(C_q4, "u8", device) if C_q4 is not None else None
     sc = device_array(C_scales, "bf16", device) if C_scales is not None else None
     return Index(Ed, Cd, C2Td, q4, sc, int4=int4, cluster_major=cluster_major)
+
+
+# ----------------------------------------------------------------------------- index builder
+
+
+def _kmeans_call(fn_name, E, c, stream, **fields):
+    _need(E, "E")
+    if E.dtype != torch.bfloat16 or E.dim() != 2:
+        raise TypeError("E must be a v x d torch.bfloat16 matrix")
+    v, d = E.shape
+    L = load()
+    nbytes = L.fh_kmeans_ws_bytes(v, d, c)
+    if nbytes == 0:
+        raise FlashHeadError(2, f"invalid builder sizes v={v} d={d} c={c}")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=E.device)
+    keep = []
+    args = KmeansArgs()
+    args.E = E.data_ptr()
+    args.dtype = FH_BF16
+    args.v, args.d, args.c = v, d, c
+    for name, value in fields.items():
+        if isinstance(value, torch.Tensor):
+            _need(value, name)
+            keep.append(value)
+            setattr(args, name, value.data_ptr())
+        elif value is not None:
+            setattr(args, name, value)
+    _check(getattr(L, fn_name)(ct.byref(args), _ptr(ws), nbytes, _stream(stream)))
+    return args
+
+
+def kmeans_build(E, c, init_tokens, iters, eps=1e-4, max_rounds=0, stream=None):
+    """Equal-size spherical k-means of the rows of E (v x d BF16) into c clusters, starting from
+    the unit rows of init_tokens (c distinct ids, int32 on the device).  Returns a dict with labels
+    (v), C2T (c x v/c), C (c x d fp32), C_bf16, objective (one Eq.4 value per update), prices
+    (last auction), iters and rounds.  Synchronises the stream."""
+    v, d = E.shape
+    dev = E.device
+    out = dict(labels=torch.empty(v, dtype=torch.int32, device=dev),
+               C2T=torch.empty((c, v // c), dtype=torch.int32, device=dev),
+               C=torch.empty((c, d), dtype=torch.float32, device=dev),
+               C_bf16=torch.empty((c, d), dtype=torch.bfloat16, device=dev),
+               objective=torch.zeros(iters, dtype=torch.float64, device=dev),
+               prices=torch.empty(c, dtype=torch.float32, device=dev))
+    a = _kmeans_call("fh_kmeans_build", E, c, stream, iters=iters, eps=eps, max_rounds=max_rounds,
+                     init_tokens=init_tokens, **out)
+    out["objective"] = out["objective"][:a.iters_done]
+    out["iters"], out["rounds"] = a.iters_done, a.rounds
+    return out
+
+
+def kmeans_assign(E, C_bf16, eps=1e-4, max_rounds=0, stream=None):
+    """The equal-size assignment of the rows of E to the BF16 centres C_bf16 (c x d), within
+    v * eps of the optimum.  Returns labels, C2T, prices and rounds.  Synchronises the stream."""
+    v, d = E.shape
+    c = C_bf16.shape[0]
+    dev = E.device
+    out = dict(labels=torch.empty(v, dtype=torch.int32, device=dev),
+               C2T=torch.empty((c, v // c), dtype=torch.int32, device=dev),
+               prices=torch.empty(c, dtype=torch.float32, device=dev))
+    a = _kmeans_call("fh_kmeans_assign", E, c, stream, eps=eps, max_rounds=max_rounds,
+                     C_in=C_bf16, **out)
+    out["rounds"] = a.rounds
+    return out
+
+
+def kmeans_update(E, labels, c, stream=None):
+    """Eq.5 for an equal-size labeling: returns C2T, C (fp32 unit rows), C_bf16 and the objective
+    of Eq.4 (one value).  Synchronises the stream."""
+    v, d = E.shape
+    dev = E.device
+    out = dict(C2T=torch.empty((c, v // c), dtype=torch.int32, device=dev),
+               C=torch.empty((c, d), dtype=torch.float32, device=dev),
+               C_bf16=torch.empty((c, d), dtype=torch.bfloat16, device=dev),
+               objective=torch.zeros(1, dtype=torch.float64, device=dev))
+    _kmeans_call("fh_kmeans_update", E, c, stream, eps=1e-4, labels_in=labels, **out)
+    return out

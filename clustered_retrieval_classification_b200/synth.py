@@ -259,3 +259,28 @@ def random_index(v: int, d: int, c: int, seed: int, dtype: str = "f32") -> Index
                      heavy_frac=0.0, heavy_mult=1.0, h_scale=1.0, data_seed=seed,
                      query_seed=seed + 1)
     return Index(cfg, E, C, C2T)
+
+
+# ----------------------------------------------------------------------------- index-builder inputs
+
+KMEANS_SEED = 6000
+
+
+def planted_embeddings(c: int, b: int, d: int, spread: float, seed: int = KMEANS_SEED):
+    """Inputs for the equal-size k-means builder: v = c*b BF16 rows around c random directions,
+    exactly b per direction (noise N(0, spread^2/d) per column, norms from U(0.5, 2)), token ids
+    shuffled.  Returns (E as BF16 patterns [v, d], the generating direction of each token [v])."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    dirs = rng.standard_normal((c, d))
+    dirs /= np.linalg.norm(dirs, axis=1, keepdims=True)
+    lab = np.repeat(np.arange(c), b)
+    X = dirs[lab] + spread * rng.standard_normal((c * b, d)) / math.sqrt(d)
+    X *= rng.uniform(0.5, 2.0, size=(c * b, 1))
+    perm = rng.permutation(c * b)
+    return bf16_from_f32(X[perm].astype(np.float32)), lab[perm].astype(np.int32)
+
+
+def init_tokens(v: int, c: int, seed: int = KMEANS_SEED + 1) -> np.ndarray:
+    """c distinct token ids drawn by a seeded permutation: the builder's initial centres."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    return rng.permutation(v)[:c].astype(np.int32)

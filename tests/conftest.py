@@ -12,6 +12,12 @@ def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
 
 
+def pytest_collection_modifyitems(config, items):
+    """The index builder's device tests run after every head test (a stable sort keeps the rest in
+    file order), so that under -x a builder failure cannot hide a head result."""
+    items.sort(key=lambda item: os.path.basename(str(item.fspath)) == "test_kmeans_gpu.py")
+
+
 @pytest.fixture(scope="session")
 def orc():
     import oracle

@@ -1,8 +1,9 @@
-"""The C ABI library: it loads without a GPU, exports every function include/flashhead.h declares,
+"""The C ABI library: it loads without a GPU, exports every function include/*.h declares,
 the binding declares a signature for each, and host-side argument checks reject bad calls before
 any device work."""
 
 import ctypes as ct
+import glob
 import os
 import re
 
@@ -11,13 +12,15 @@ import pytest
 from clustered_retrieval_classification_b200 import _build
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "flashhead.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(fh_[a-z0-9_]+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names.update(re.findall(r"\b(fh_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -31,7 +34,8 @@ def test_header_declares_the_boundary():
     for required in ["fh_index_load", "fh_index_free", "fh_workspace_bytes", "fh_head_greedy",
                      "fh_head_sample", "fh_mc_token_prob", "fh_dense_head", "fh_last_error",
                      "fh_ws_status", "fh_stage1_scores", "fh_select_topp",
-                     "fh_gather_candidates", "fh_candidate_logits", "fh_philox_u32"]:
+                     "fh_gather_candidates", "fh_candidate_logits", "fh_philox_u32",
+                     "fh_kmeans_ws_bytes", "fh_kmeans_build", "fh_kmeans_assign", "fh_kmeans_update"]:
         assert required in names
 
 
@@ -65,3 +69,25 @@ def test_host_side_argument_checks(lib):
     assert L.fh_workspace_bytes(None, 0, 1, 1, 1, 1) == 0
     assert L.fh_select_topp(None, 1, 8, 2, None, None) == 1
     assert L.fh_philox_u32(0, 0, 0, 0, 0, None, None) == 1
+
+
+def test_builder_host_side_argument_checks(lib):
+    """Index builder (include/fh_kmeans.h): sizes and arguments are checked before any CUDA call."""
+    from clustered_retrieval_classification_b200 import flashhead as F
+    L = F.load()
+    assert L.fh_kmeans_ws_bytes(100, 64, 7) == 0          # c does not divide v
+    assert L.fh_kmeans_ws_bytes(112, 64, 7) >= 112 * 7 * 4
+    assert L.fh_kmeans_build(None, None, 0, None) == 1    # FH_ERR_ARG
+    a = F.KmeansArgs()
+    a.E, a.dtype, a.v, a.d, a.c, a.iters, a.eps = 16, F.FH_F32, 112, 64, 7, 1, 1e-4
+    assert L.fh_kmeans_build(ct.byref(a), None, 0, None) == 7   # FP32 E: FH_ERR_UNSUPPORTED
+    a.dtype = F.FH_BF16
+    a.v = 100
+    assert L.fh_kmeans_build(ct.byref(a), None, 0, None) == 2   # v % c
+    a.v, a.d = 112, 60
+    assert L.fh_kmeans_build(ct.byref(a), None, 0, None) == 2   # d % 8
+    a.d = 64
+    assert L.fh_kmeans_build(ct.byref(a), None, 0, None) == 1   # init_tokens NULL
+    assert b"init_tokens" in L.fh_last_error()
+    assert L.fh_kmeans_assign(ct.byref(a), None, 0, None) == 1  # C_in NULL
+    assert L.fh_kmeans_update(ct.byref(a), None, 0, None) == 1  # labels_in NULL

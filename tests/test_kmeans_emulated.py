@@ -1,0 +1,142 @@
+"""The index builder's steps (equal-size spherical k-means; FlashHead notes, Module 1, Eq.4/Eq.5)
+run on the CPU through a host build of the same per-item functions and iteration loop the device
+kernels use (tests/kmeans_emu.cpp), checked against the float64 oracle.  This covers the auction,
+C2T, Eq.5 and the loop's control flow, indexing included, without a GPU; the device build is
+checked the same way by the GPU tests."""
+
+import ctypes as ct
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+from clustered_retrieval_classification_b200 import synth
+from kmeans_checks import check_assignment, check_run, check_update
+from oracle import kmeans_oracle as K
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+DONE, BAD_INIT, ZERO_ROW, DEGENERATE, ROUND_LIMIT = 0, 1, 2, 3, 4
+
+
+@pytest.fixture(scope="module")
+def emu(tmp_path_factory):
+    out = str(tmp_path_factory.mktemp("kmemu") / "kmemu.so")
+    subprocess.run(["g++", "-O2", "-std=c++17", "-ffp-contract=off", "-fPIC", "-shared", "-o", out,
+                    os.path.join(HERE, "kmeans_emu.cpp")], check=True)
+    L = ct.CDLL(out)
+    L.emu_kmeans.restype = ct.c_int
+    p = ct.c_void_p
+    L.emu_kmeans.argtypes = [ct.c_int, p, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_int, ct.c_float,
+                             ct.c_int64, p, p, p, p, p, p, p, p, p, p, p]
+    return L
+
+
+def ptr(a):
+    return None if a is None else a.ctypes.data_as(ct.c_void_p)
+
+
+def call(L, op, E, c, iters=1, eps=1e-4, max_rounds=0, init=None, C_in=None, labels_in=None):
+    v, d = E.shape
+    b = v // c
+    labels = np.full(v, -1, dtype=np.int32)
+    C2T = np.zeros((c, b), dtype=np.int32)
+    C = np.zeros((c, d), dtype=np.float32)
+    Cb = np.zeros((c, d), dtype=np.uint16)
+    obj = np.zeros(max(iters, 1), dtype=np.float64)
+    prices = np.zeros(c, dtype=np.float32)
+    it = ct.c_int32(0)
+    rounds = ct.c_int64(0)
+    st = L.emu_kmeans(op, ptr(np.ascontiguousarray(E)), v, d, c, iters, eps, max_rounds,
+                      ptr(init), ptr(C_in), ptr(labels_in), ptr(labels), ptr(C2T), ptr(C), ptr(Cb),
+                      ptr(obj), ptr(prices), ct.byref(it), ct.byref(rounds))
+    return dict(status=st, labels=labels, C2T=C2T, C=C, C_bf16=Cb, objective=obj[:it.value],
+                prices=prices, iters=it.value, rounds=rounds.value)
+
+
+def random_centres(c, d, seed):
+    rng = np.random.default_rng(seed)
+    C = rng.standard_normal((c, d))
+    C /= np.linalg.norm(C, axis=1, keepdims=True)
+    return synth.bf16_from_f32(C.astype(np.float32))
+
+
+@pytest.mark.parametrize("c,b,d,spread", [(16, 32, 64, 1.0), (8, 40, 72, 3.0), (5, 13, 24, 0.5),
+                                            (96, 8, 32, 1.0), (200, 3, 16, 2.0)])
+def test_assignment_is_certified_and_near_optimal(emu, c, b, d, spread):
+    """c > 32 puts several clusters on each of the 32 lanes that scan a token's row."""
+    E, _ = synth.planted_embeddings(c, b, d, spread, seed=c * 100 + b)
+    C_in = random_centres(c, d, seed=b)
+    r = call(emu, 1, E, c, C_in=C_in, eps=1e-4)
+    assert r["status"] == DONE and r["rounds"] > 0
+    got, best = check_assignment(E, C_in, c, 1e-4, r["labels"], r["C2T"], r["prices"])
+    assert got <= best + 1e-9
+
+
+def test_assignment_degenerate_shapes(emu):
+    E, _ = synth.planted_embeddings(1, 40, 16, 1.0, seed=3)
+    r = call(emu, 1, E, 1, C_in=random_centres(1, 16, 1))  # one cluster holds every token
+    assert r["status"] == DONE and np.all(r["labels"] == 0)
+    assert np.array_equal(r["C2T"][0], np.arange(40))
+    E, _ = synth.planted_embeddings(12, 1, 16, 1.0, seed=4)  # b = 1: a permutation
+    C_in = random_centres(12, 16, 2)
+    r = call(emu, 1, E, 12, C_in=C_in)
+    assert r["status"] == DONE
+    check_assignment(E, C_in, 12, 1e-4, r["labels"], r["C2T"], r["prices"])
+
+
+def test_assignment_tolerance_bounds_the_loss(emu):
+    """A coarse eps still returns a valid labeling whose loss stays within v * eps."""
+    E, _ = synth.planted_embeddings(10, 30, 32, 2.0, seed=8)
+    C_in = random_centres(10, 32, 9)
+    for eps in (0.25, 0.01):
+        r = call(emu, 1, E, 10, C_in=C_in, eps=eps)
+        assert r["status"] == DONE
+        check_assignment(E, C_in, 10, eps, r["labels"], r["C2T"], r["prices"])
+
+
+def test_update_matches_eq5(emu):
+    E, _ = synth.planted_embeddings(9, 24, 40, 1.5, seed=10)
+    labels = np.random.default_rng(1).permutation(np.repeat(np.arange(9), 24)).astype(np.int32)
+    r = call(emu, 2, E, 9, labels_in=labels)
+    assert r["status"] == DONE and r["iters"] == 1
+    assert np.array_equal(r["C2T"], K.c2t_from_labels(labels, 9, 24))
+    check_update(E, labels, 9, r["C"], r["C_bf16"], r["objective"][0])
+
+
+def test_build_recovers_planted_clusters(emu):
+    c, b = 8, 64
+    E, gen = synth.planted_embeddings(c, b, 72, 0.3, seed=11)
+    init = np.array([np.nonzero(gen == k)[0][0] for k in range(c)], dtype=np.int32)
+    r = call(emu, 0, E, c, iters=20, init=init)
+    assert r["status"] == DONE
+    assert 1 <= r["iters"] < 20  # stopped at a fixed point
+    assert np.array_equal(r["labels"], gen)
+    check_run(E, c, r["labels"], r["C2T"], r["C"], r["C_bf16"], r["objective"], 1e-4)
+    o_lab, o_C, o_hist = K.kmeans(E, c, init, iters=20)
+    assert np.array_equal(o_lab, gen)
+    assert r["objective"][-1] == pytest.approx(o_hist[-1], rel=1e-5)
+
+
+def test_build_on_overlapping_clusters(emu):
+    c, b = 16, 32
+    E, _ = synth.planted_embeddings(c, b, 64, 3.0, seed=12)
+    init = synth.init_tokens(c * b, c)
+    r = call(emu, 0, E, c, iters=30, init=init)
+    assert r["status"] == DONE and r["iters"] >= 2
+    # no comparison with the oracle's own run: an eps-optimal assignment may break ties of the
+    # exact one differently, and from there the two runs reach different local optima
+    check_run(E, c, r["labels"], r["C2T"], r["C"], r["C_bf16"], r["objective"], 1e-4)
+
+
+def test_rejected_inputs(emu):
+    E, gen = synth.planted_embeddings(4, 8, 16, 0.5, seed=13)
+    Ez = E.copy()
+    Ez[5] = 0
+    assert call(emu, 0, Ez, 4, iters=3, init=np.arange(4, dtype=np.int32))["status"] == ZERO_ROW
+    assert call(emu, 0, E, 4, iters=3, init=np.array([0, 1, 1, 2], dtype=np.int32))["status"] == BAD_INIT
+    assert call(emu, 0, E, 4, iters=3, init=np.array([0, 1, 2, 32], dtype=np.int32))["status"] == BAD_INIT
+    bad = gen.copy()
+    bad[0] = (bad[0] + 1) % 4
+    assert call(emu, 2, E, 4, labels_in=bad)["status"] == BAD_INIT
+    assert call(emu, 1, E, 4, C_in=random_centres(4, 16, 3), max_rounds=1)["status"] == ROUND_LIMIT

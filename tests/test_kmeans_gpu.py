@@ -1,0 +1,114 @@
+"""The index builder on the device (include/fh_kmeans.h: equal-size spherical k-means, FlashHead
+notes Module 1, Eq.4/Eq.5) against the float64 oracle, through the C ABI.  The same checks as the
+CPU tests of the host build (tests/kmeans_checks.py): certified near-optimal equal-size
+assignments, Eq.5 element by element, and whole runs whose centres are Eq.5 of their labels with
+an objective that does not rise.  Sizes span several 64-token tensor-core launches with a ragged
+last launch, more clusters than the 32 lanes of a bid warp, and d past one 64-column K-block."""
+
+import numpy as np
+import pytest
+import torch
+
+from clustered_retrieval_classification_b200 import synth
+from kmeans_checks import check_assignment, check_run, check_update
+from oracle import kmeans_oracle as K
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def dev(a, kind):
+    from clustered_retrieval_classification_b200 import flashhead as F
+    return F.device_array(a, kind, DEV)
+
+
+def host_bf16(t):
+    return t.cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def random_centres(c, d, seed):
+    rng = np.random.default_rng(seed)
+    C = rng.standard_normal((c, d))
+    C /= np.linalg.norm(C, axis=1, keepdims=True)
+    return synth.bf16_from_f32(C.astype(np.float32))
+
+
+@pytest.mark.parametrize("c,b,d,spread", [(16, 32, 64, 1.0), (8, 40, 72, 3.0), (96, 8, 128, 1.0),
+                                          (76, 34, 256, 2.0), (200, 3, 200, 2.0)])
+def test_assignment_is_certified_and_near_optimal(fh, c, b, d, spread):
+    E, _ = synth.planted_embeddings(c, b, d, spread, seed=c * 100 + b)
+    C_in = random_centres(c, d, seed=b)
+    r = fh.kmeans_assign(dev(E, "bf16"), dev(C_in, "bf16"), eps=1e-4)
+    assert r["rounds"] > 0
+    check_assignment(E, C_in, c, 1e-4, r["labels"].cpu().numpy(), r["C2T"].cpu().numpy(),
+                     r["prices"].cpu().numpy())
+
+
+def test_assignment_one_cluster_and_permutation(fh):
+    E, _ = synth.planted_embeddings(1, 40, 64, 1.0, seed=3)
+    r = fh.kmeans_assign(dev(E, "bf16"), dev(random_centres(1, 64, 1), "bf16"))
+    assert np.all(r["labels"].cpu().numpy() == 0)
+    assert np.array_equal(r["C2T"].cpu().numpy()[0], np.arange(40))
+    E, _ = synth.planted_embeddings(12, 1, 64, 1.0, seed=4)
+    C_in = random_centres(12, 64, 2)
+    r = fh.kmeans_assign(dev(E, "bf16"), dev(C_in, "bf16"))
+    check_assignment(E, C_in, 12, 1e-4, r["labels"].cpu().numpy(), r["C2T"].cpu().numpy(),
+                     r["prices"].cpu().numpy())
+
+
+def test_update_matches_eq5(fh):
+    E, _ = synth.planted_embeddings(9, 24, 136, 1.5, seed=10)
+    labels = np.random.default_rng(1).permutation(np.repeat(np.arange(9), 24)).astype(np.int32)
+    r = fh.kmeans_update(dev(E, "bf16"), dev(labels, "i32"), 9)
+    assert np.array_equal(r["C2T"].cpu().numpy(), K.c2t_from_labels(labels, 9, 24))
+    check_update(E, labels, 9, r["C"].cpu().numpy(), host_bf16(r["C_bf16"]),
+                 float(r["objective"].cpu()[0]))
+
+
+def test_build_recovers_planted_clusters(fh):
+    c, b = 8, 64
+    E, gen = synth.planted_embeddings(c, b, 72, 0.3, seed=11)
+    init = np.array([np.nonzero(gen == k)[0][0] for k in range(c)], dtype=np.int32)
+    r = fh.kmeans_build(dev(E, "bf16"), c, dev(init, "i32"), iters=20)
+    assert 1 <= r["iters"] < 20
+    labels = r["labels"].cpu().numpy()
+    assert np.array_equal(labels, gen)
+    check_run(E, c, labels, r["C2T"].cpu().numpy(), r["C"].cpu().numpy(), host_bf16(r["C_bf16"]),
+              r["objective"].cpu().numpy(), 1e-4)
+
+
+def test_build_on_overlapping_clusters(fh):
+    c, b = 48, 40
+    E, _ = synth.planted_embeddings(c, b, 256, 3.0, seed=12)
+    init = synth.init_tokens(c * b, c)
+    r = fh.kmeans_build(dev(E, "bf16"), c, dev(init, "i32"), iters=30)
+    assert r["iters"] >= 2
+    hist = r["objective"].cpu().numpy()
+    check_run(E, c, r["labels"].cpu().numpy(), r["C2T"].cpu().numpy(), r["C"].cpu().numpy(),
+              host_bf16(r["C_bf16"]), hist, 1e-4)
+    # no comparison with the oracle's own run: an eps-optimal assignment may break ties of the
+    # exact one differently, and from there the two runs reach different local optima
+
+
+def test_rejected_inputs(fh):
+    E, gen = synth.planted_embeddings(4, 16, 64, 0.5, seed=13)
+    Ez = E.copy()
+    Ez[5] = 0
+    with pytest.raises(fh.FlashHeadError) as e:
+        fh.kmeans_build(dev(Ez, "bf16"), 4, dev(np.arange(4, dtype=np.int32), "i32"), iters=3)
+    assert e.value.status == 1
+    with pytest.raises(fh.FlashHeadError) as e:
+        fh.kmeans_build(dev(E, "bf16"), 4, dev(np.array([0, 1, 1, 2], dtype=np.int32), "i32"), iters=3)
+    assert e.value.status == 1
+    bad = gen.copy()
+    bad[0] = (bad[0] + 1) % 4
+    with pytest.raises(fh.FlashHeadError) as e:
+        fh.kmeans_update(dev(E, "bf16"), dev(bad, "i32"), 4)
+    assert e.value.status == 1
+    with pytest.raises(fh.FlashHeadError) as e:
+        fh.kmeans_assign(dev(E, "bf16"), dev(random_centres(4, 64, 3), "bf16"), max_rounds=1)
+    assert e.value.status == 6
+    # the workspace and the context stay usable after every rejection
+    r = fh.kmeans_assign(dev(E, "bf16"), dev(random_centres(4, 64, 3), "bf16"))
+    assert K.is_equal_size(r["labels"].cpu().numpy(), 4, 16)

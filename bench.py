@@ -16,7 +16,8 @@ cores and GPU-vs-oracle token counts on the oracle's sample.  `--impl reference`
 Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under torch.distributed.run,
 one independent replica per GPU (the whole index fits one GPU and a vocabulary split would add two
 collective latencies per call, so the head does not shard), time = max over ranks.  Other modes:
---ncu-case (untimed calls for ncu captures) and --pc-sweep (the p/c trade-off at batch 1).
+--ncu-case (untimed calls for ncu captures), --pc-sweep (the p/c trade-off at batch 1) and
+--kmeans (the equal-size k-means index builder on the Llama-shaped embeddings).
 """
 
 import argparse
@@ -559,6 +560,41 @@ def pc_sweep(args):
     return 0
 
 
+def kmeans_bench(args):
+    """The index builder (equal-size spherical k-means, FlashHead notes Module 1) on the
+    Llama-shaped embedding matrix (v = 128256, d = 2048, BF16) into c = 8016 clusters of 16:
+    --kmeans-iters iterations from seeded initial tokens, timed with CUDA events around the call
+    (which synchronises after every auction round).  The line carries the library's own outputs
+    (iterations, auction rounds, the objective per iteration) and two validity checks of the
+    result: every cluster holds exactly b tokens and C2T lists each token once.  Parity with the
+    oracle is the tests' job (tests/test_kmeans_gpu.py)."""
+    from clustered_retrieval_classification_b200 import flashhead as F
+    F.load()
+    cfg = synth.CONFIGS["llama"]
+    idx = synth.make_index(cfg)
+    v, d, c, b = cfg.v, cfg.d, cfg.c, cfg.b
+    E = F.device_array(idx.E, "bf16")
+    init = F.device_array(synth.init_tokens(v, c), "i32")
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    r = F.kmeans_build(E, c, init, iters=args.kmeans_iters, eps=1e-4)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    labels = r["labels"].cpu().numpy()
+    C2T = r["C2T"].cpu().numpy()
+    it = max(r["iters"], 1)
+    print(json.dumps({"kmeans": {
+        "workload": "llama-3.2-1b-shaped embeddings v=128256 d=2048 bf16, c=8016 (b=16)",
+        "iters": r["iters"], "rounds": r["rounds"], "ms_total": ms, "ms_per_iter": ms / it,
+        "similarity_tflop_per_iter": 2.0 * v * c * d / 1e12,
+        "objective": r["objective"].cpu().numpy().tolist(),
+        "equal_size": bool(np.all(np.bincount(labels, minlength=c) == b)),
+        "c2t_is_permutation": bool(np.array_equal(np.sort(C2T.ravel()), np.arange(v)))}}),
+        flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -577,6 +613,10 @@ def main():
                     help="time the batch-1 greedy head of the Llama-shaped vocabulary at "
                          "c in {4008, 8016, 16032} x p in {128, 256, 512} (with oracle token checks), "
                          "print one JSON line and exit")
+    ap.add_argument("--kmeans", action="store_true",
+                    help="run the index builder on the Llama-shaped embeddings (c=8016), print one "
+                         "JSON line with its timing and validity checks, and exit")
+    ap.add_argument("--kmeans-iters", type=int, default=5)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -585,6 +625,8 @@ def main():
         return ncu_case(args)
     if args.pc_sweep:
         return pc_sweep(args)
+    if args.kmeans:
+        return kmeans_bench(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

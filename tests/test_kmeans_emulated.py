@@ -113,6 +113,8 @@ def test_build_recovers_planted_clusters(emu):
     assert 1 <= r["iters"] < 20  # stopped at a fixed point
     assert np.array_equal(r["labels"], gen)
     check_run(E, c, r["labels"], r["C2T"], r["C"], r["C_bf16"], r["objective"], 1e-4)
+    # at a fixed point the last auction scored the returned BF16 centres: its prices certify it
+    check_assignment(E, r["C_bf16"], c, 1e-4, r["labels"], r["C2T"], r["prices"])
     o_lab, o_C, o_hist = K.kmeans(E, c, init, iters=20)
     assert np.array_equal(o_lab, gen)
     assert r["objective"][-1] == pytest.approx(o_hist[-1], rel=1e-5)
@@ -127,6 +129,8 @@ def test_build_on_overlapping_clusters(emu):
     # no comparison with the oracle's own run: an eps-optimal assignment may break ties of the
     # exact one differently, and from there the two runs reach different local optima
     check_run(E, c, r["labels"], r["C2T"], r["C"], r["C_bf16"], r["objective"], 1e-4)
+    if r["iters"] < 30:  # stopped at a fixed point: the prices certify the final labels
+        check_assignment(E, r["C_bf16"], c, 1e-4, r["labels"], r["C2T"], r["prices"])
 
 
 def test_rejected_inputs(emu):

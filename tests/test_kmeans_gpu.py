@@ -76,6 +76,9 @@ def test_build_recovers_planted_clusters(fh):
     assert np.array_equal(labels, gen)
     check_run(E, c, labels, r["C2T"].cpu().numpy(), r["C"].cpu().numpy(), host_bf16(r["C_bf16"]),
               r["objective"].cpu().numpy(), 1e-4)
+    # at a fixed point the last auction scored the returned BF16 centres: its prices certify it
+    check_assignment(E, host_bf16(r["C_bf16"]), c, 1e-4, labels, r["C2T"].cpu().numpy(),
+                     r["prices"].cpu().numpy())
 
 
 def test_build_on_overlapping_clusters(fh):
@@ -87,6 +90,9 @@ def test_build_on_overlapping_clusters(fh):
     hist = r["objective"].cpu().numpy()
     check_run(E, c, r["labels"].cpu().numpy(), r["C2T"].cpu().numpy(), r["C"].cpu().numpy(),
               host_bf16(r["C_bf16"]), hist, 1e-4)
+    if r["iters"] < 30:  # stopped at a fixed point: the prices certify the final labels
+        check_assignment(E, host_bf16(r["C_bf16"]), c, 1e-4, r["labels"].cpu().numpy(),
+                         r["C2T"].cpu().numpy(), r["prices"].cpu().numpy())
     # no comparison with the oracle's own run: an eps-optimal assignment may break ties of the
     # exact one differently, and from there the two runs reach different local optima
 

@@ -118,3 +118,27 @@ def test_rejected_inputs(fh):
     # the workspace and the context stay usable after every rejection
     r = fh.kmeans_assign(dev(E, "bf16"), dev(random_centres(4, 64, 3), "bf16"))
     assert K.is_equal_size(r["labels"].cpu().numpy(), 4, 16)
+
+
+def test_built_index_serves_the_head(fh, orc):
+    """The builder's outputs load as a FlashHead index (fh_index_load checks that C2T is a
+    permutation): with p = c the head returns the dense arg-max (the candidates are the whole
+    vocabulary), and with p < c the oracle's token wherever its set and token margins decide it."""
+    c, b, d = 1024, 8, 64
+    E, _ = synth.planted_embeddings(c, b, d, 1.0, seed=21)
+    Ed = dev(E, "bf16")
+    r = fh.kmeans_build(Ed, c, dev(synth.init_tokens(c * b, c), "i32"), iters=3)
+    I = fh.Index(Ed, r["C_bf16"], r["C2T"])
+    rng = np.random.default_rng(4)
+    H = synth.store((rng.standard_normal((4, d)) * 2).astype(np.float32), "bf16")
+    Hd = dev(H, "bf16")
+    for q in range(4):
+        assert int(fh.head_greedy(I, Hd[q:q + 1], c).item()) == int(fh.dense_head(I, Hd[q:q + 1]).item())
+    cfg = synth.HeadConfig("built-index", v=c * b, d=d, c=c, p=100, dtype="bf16", noise=0.0,
+                           heavy_frac=0.0, heavy_mult=1.0, h_scale=1.0, data_seed=21, query_seed=22)
+    idx = synth.Index(cfg, E, host_bf16(r["C_bf16"]), r["C2T"].cpu().numpy())
+    for q in range(4):
+        tok = int(fh.head_greedy(I, Hd[q:q + 1], 100).item())
+        o = orc.head(idx, H[q:q + 1], 100)
+        if o["set_margin"][0] > 4e-3 and o["tok_margin"][0] > 4e-3:
+            assert tok == int(o["tok"][0]), q

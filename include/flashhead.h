@@ -15,6 +15,7 @@
  * "selective quantization").  A Monte Carlo driver estimates the marginal token probability
  * p̂(t|h) = (1/N) Σ_i p(t|h,S_i) over N independent Stage-1 draws S_i (FlashHead notes,
  * Module 4 and Eq. 7).  A dense head over all v rows is provided as the in-run comparison.
+ * The index (C and C2T) is built offline from E by equal-size spherical k-means: see fh_kmeans.h.
  *
  * Citation names used in this header:
  *   "FlashHead notes"   — the reading-notes page "FlashHead: Efficient Drop-In Replacement for the

@@ -91,3 +91,26 @@ def test_builder_host_side_argument_checks(lib):
     assert b"init_tokens" in L.fh_last_error()
     assert L.fh_kmeans_assign(ct.byref(a), None, 0, None) == 1  # C_in NULL
     assert L.fh_kmeans_update(ct.byref(a), None, 0, None) == 1  # labels_in NULL
+
+
+@pytest.mark.parametrize("struct,pyname", [("fh_index_desc", "IndexDesc"), ("fh_debug_out", "DebugOut"),
+                                           ("fh_kmeans_args", "KmeansArgs")])
+def test_binding_structs_match_the_headers(tmp_path, struct, pyname):
+    """Every field of the binding's ctypes structures sits at the offset the C compiler gives it."""
+    import subprocess
+    from clustered_retrieval_classification_b200 import flashhead as F
+    py = getattr(F, pyname)
+    fields = [f[0] for f in py._fields_]
+    src = tmp_path / "layout.c"
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fh_kmeans.h"', "int main(void) {",
+             f'  printf("%zu\\n", sizeof({struct}));']
+    lines += [f'  printf("%zu\\n", offsetof({struct}, {f}));' for f in fields]
+    lines += ["  return 0;", "}"]
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)],
+                   check=True)
+    out = [int(x) for x in subprocess.run([str(exe)], capture_output=True, text=True,
+                                          check=True).stdout.split()]
+    assert out[0] == ct.sizeof(py)
+    assert out[1:] == [getattr(py, f).offset for f in fields]

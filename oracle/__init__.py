@@ -11,7 +11,6 @@ Arrays are passed as stored: float32 values for dtype "f32", uint16 BF16 bit pat
 from __future__ import annotations
 
 import ctypes as ct
-import os
 
 import numpy as np
 

@@ -142,3 +142,25 @@ def test_built_index_serves_the_head(fh, orc):
         o = orc.head(idx, H[q:q + 1], 100)
         if o["set_margin"][0] > 4e-3 and o["tok_margin"][0] > 4e-3:
             assert tok == int(o["tok"][0]), q
+
+
+def test_assignment_at_the_llama_shape_sampled(fh):
+    """Full size (v = 128256, d = 2048, c = 8016 centres of the synthetic Llama-shaped index): the
+    assignment is equal-size and C2T lists it, and the prices certify eps-complementary slackness
+    on 256 sampled tokens against the oracle's float64 similarities (the exact optimum is out of
+    the oracle's reach at this size; the certificate bounds the loss by v * eps)."""
+    cfg = synth.CONFIGS["llama"]
+    idx = synth.make_index(cfg)
+    r = fh.kmeans_assign(dev(idx.E, "bf16"), dev(idx.C, "bf16"), eps=1e-4)
+    labels = r["labels"].cpu().numpy()
+    assert K.is_equal_size(labels, cfg.c, cfg.b)
+    assert np.array_equal(r["C2T"].cpu().numpy(), K.c2t_from_labels(labels, cfg.c, cfg.b))
+    # every generated token is far nearer its own centroid than any other, b to a centroid: the
+    # optimum is the generator's own table, which the first round of each phase already reaches
+    assert np.array_equal(r["C2T"].cpu().numpy(), idx.C2T)
+    toks = np.random.default_rng(9).choice(cfg.v, 256, replace=False)
+    A = K.unit_rows(idx.E[toks]) @ K.stored_to_f64(idx.C).T
+    prices = r["prices"].cpu().numpy().astype(np.float64)
+    net = A - prices[None, :]
+    gap = (net.max(axis=1) - net[np.arange(256), labels[toks]]).max()
+    assert gap <= 1e-4 + 4e-5, gap

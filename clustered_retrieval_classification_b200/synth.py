@@ -232,6 +232,79 @@ def shift_centroids(C: np.ndarray, t: float) -> np.ndarray:
     return C - t * C.mean(axis=0, keepdims=True)
 
 
+def anisotropic_centroids(c: int, d: int, common: float, seed: int) -> np.ndarray:
+    """Unit centroids normalise(u + common·sqrt(d)·m) with u ~ N(0, I) and one fixed unit direction m
+    (float64): stand-ins for real head centroids, which share a dominant mean component, for the
+    centroid-shift study of INT4 Stage 1."""
+    rng = np.random.Generator(np.random.PCG64(seed))
+    m = rng.standard_normal(d)
+    m /= np.linalg.norm(m)
+    u = rng.standard_normal((c, d)) + common * math.sqrt(d) * m[None, :]
+    return u / np.linalg.norm(u, axis=1, keepdims=True)
+
+
+# ----------------------------------------------------------------------------- coarse-fine head inputs
+# The coarse-fine head (page "Fast LM Head via Coarse-Fine Decomposition and Tile-Wise Weight
+# Clustering", abstract) reads E through a per-tile codebook and an index map.  These helpers build
+# that offline index for a synthetic E; the head's own arithmetic (look-up tables, coarse scores,
+# selection, exact logits) is not here.
+
+CF_TILE_W = 8        # columns per tile
+CF_CODES = 16        # codebook entries per tile (4-bit codes)
+CF_TOPK = 1024       # candidates that get exact logits
+
+
+def cf_pack_codes(codes: np.ndarray) -> np.ndarray:
+    """Pack a (v, T) array of 4-bit codes (T % 8 == 0) into the index-map layout the library reads:
+    uint32 words [T/8, v], word (g, u) holding the codes of tiles 8g..8g+7 of token u, tile 8g+j in
+    bits 4j..4j+3."""
+    codes = np.asarray(codes, dtype=np.uint32)
+    v, T = codes.shape
+    if T % 8:
+        raise ValueError("the number of tiles must be a multiple of 8")
+    g = codes.reshape(v, T // 8, 8)
+    words = np.zeros((v, T // 8), dtype=np.uint32)
+    for j in range(8):
+        words |= (g[:, :, j] & 0xF) << np.uint32(4 * j)
+    return np.ascontiguousarray(words.T)
+
+
+def cf_index(E: np.ndarray, dtype: str, w: int = CF_TILE_W, K: int = CF_CODES, iters: int = 3,
+             seed: int = 7000, chunk: int = 8192):
+    """Offline tile-wise k-means of the embedding rows: E's columns are cut into T = d/w tiles; per
+    tile, K centres are fitted to the v sub-rows by `iters` Lloyd iterations (float32, starting from
+    K distinct sub-rows chosen by a seeded permutation; an empty centre keeps its old value).
+    Returns (codebooks float32 [T, K, w], packed codes uint32 [T/8, v]), the codes nearest to the
+    returned centres."""
+    X = stored_to_f64(E, dtype).astype(np.float32)
+    v, d = X.shape
+    if d % (8 * w):
+        raise ValueError("d must be a multiple of 8 tiles")
+    T = d // w
+    rng = np.random.Generator(np.random.PCG64(seed))
+    Xt = np.ascontiguousarray(X.reshape(v, T, w).transpose(1, 0, 2))          # (T, v, w)
+    cb = np.ascontiguousarray(Xt[:, rng.permutation(v)[:K], :])               # (T, K, w)
+
+    def assign(cb):
+        codes = np.empty((T, v), dtype=np.int64)
+        cc = (cb.astype(np.float32) ** 2).sum(-1)[:, None, :]                 # (T, 1, K)
+        for u0 in range(0, v, chunk):
+            dot = np.matmul(Xt[:, u0:u0 + chunk, :], cb.transpose(0, 2, 1))   # (T, n, K)
+            codes[:, u0:u0 + chunk] = np.argmin(cc - 2.0 * dot, axis=2)
+        return codes
+
+    for _ in range(iters):
+        codes = assign(cb)
+        for t in range(T):
+            cnt = np.bincount(codes[t], minlength=K)
+            nz = cnt > 0
+            for i in range(w):
+                sums = np.bincount(codes[t], weights=Xt[t, :, i], minlength=K)
+                cb[t, nz, i] = (sums[nz] / cnt[nz]).astype(np.float32)
+    cb32 = np.ascontiguousarray(cb.astype(np.float32))
+    return cb32, cf_pack_codes(assign(cb32).T)
+
+
 def make_queries(cfg: HeadConfig, n: int, seed: int | None = None) -> np.ndarray:
     """n hidden vectors h ~ N(0, I/d) * h_scale, rounded to the storage dtype."""
     rng = np.random.Generator(np.random.PCG64(cfg.query_seed if seed is None else seed))

@@ -11,6 +11,7 @@
 #include "../../include/flashhead.h"
 #include "fh_device.cuh"
 #include "fh_kernels.cuh"
+#include "fh_nvtx.cuh"
 
 struct fh_index {
   fh_index_desc desc;
@@ -37,6 +38,8 @@ fh_status cuda_fail(cudaError_t e, const char* what) {
 constexpr size_t kHeaderBytes = 1024 + 4096;  // control words, then the score histogram
 constexpr size_t kGenOffset = 536;             // batch-1 head: tag of the last completed call
 constexpr size_t kTcTicketOffset = 544;        // tensor-core head: arrival ticket (zero between calls)
+constexpr size_t kKeysReadyOffset = 552;       // batch-1 head: arrivals before its full selection
+constexpr size_t kArriveOffset = 556;          // batch-1 head: arrivals at its final reduction
 constexpr size_t kAlign = 256;
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -45,7 +48,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Workspace regions of one call; offsets from the workspace base.
 struct Layout {
-  size_t keys = 0, sel = 0, part = 0, list = 0, bnd = 0, qmask = 0, best = 0, tiles = 0, z = 0, s = 0,
+  size_t keys = 0, sel = 0, part = 0, bucket = 0, slots = 0, qmask = 0, best = 0, tiles = 0, z = 0, s = 0,
          zmax = 0, Z = 0,
          cluster_of = 0, per_draw = 0;
   size_t total = 0;
@@ -71,9 +74,9 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
       L.best = take((size_t)B * 8);
       L.tiles = take((size_t)(std::max<int64_t>(D.c, (D.v + 127) / 128) + 1) * 4);
     }
-    if (B == 1) {  // the persistent batch-1 kernel's tagged selection entries
-      L.list = take((size_t)p * 8);
-      L.bnd = take((size_t)fh::kHead1BndMax * 8);
+    if (B == 1 && fh::head1_threads(D.c) != 0) {  // the persistent batch-1 kernel's word table
+      L.bucket = take((size_t)fh::kHead1Bins * fh::kHead1BucketCap * 8);
+      L.slots = take((size_t)idx->num_sms * 8);    // and its per-block maxima
     }
   } else if (op == FH_OP_DENSE) {
     const int G = fh::stage2_blocks(D.v, B, idx->num_sms);
@@ -104,10 +107,12 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 // Workspace header (first kHeaderBytes): status word at 0, per-query tickets at 16 (64 x 4 bytes),
-// the persistent head's 64-bit final-reduction ticket at 520, its packed arg-max at 528 and its call
-// generation at 536 (the tag of the last completed call); bytes [1024, 5120) hold its 1024-bin score
-// histogram in every layout, so no other call ever writes there.  The ticket and the generation only
-// grow; the arg-max, the histogram and the selection entries return to zero at the end of every call.
+// the persistent head's call generation at 536 (the tag of the last completed call), its key-arrival
+// count at 552 and its final-reduction arrival count at 556; bytes
+// [1024, 5120) hold its 1024-bin score histogram in every layout, so no other call ever writes there.
+// The tickets, the arrival counts and the generation only grow; the histogram returns to zero at the
+// end of every call, the word table is tagged with the call generation, and the per-block maxima
+// (the `slots` region) are rewritten by every call.
 // A new workspace must start zeroed (fh_ws_status re-zeroes the header after a device-side error,
 // keeping the generation moving).
 uint32_t* status_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
@@ -189,12 +194,12 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     h.tau = tau;
     h.seed = seed;
     h.step = step;
-    h.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, 520));
-    h.best = reinterpret_cast<unsigned long long*>(word_at(ws, 528));
+    h.arrive = word_at(ws, kArriveOffset);
+    h.slots = reinterpret_cast<unsigned long long*>(base + L.slots);
     h.hist = word_at(ws, 1024);
     h.gen = word_at(ws, kGenOffset);
-    h.order = reinterpret_cast<unsigned long long*>(base + L.list);
-    h.bnd = reinterpret_cast<unsigned long long*>(base + L.bnd);
+    h.keys_ready = word_at(ws, kKeysReadyOffset);
+    h.bucket = reinterpret_cast<unsigned long long*>(base + L.bucket);
     h.out_tok = out_tok;
     h.dbg_sel = dbg ? dbg->sel : nullptr;
     h.dbg_tok = dbg ? dbg->cand_tok : nullptr;
@@ -205,7 +210,10 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     return FH_OK;
   }
   const bool fused = false;
-  const bool tc = tc_eligible(idx, B, kTcMinBatchHead) && !dbg && D.E_perm != nullptr;
+  // The tensor-core Stage 2 produces no per-candidate outputs: asking for them takes the CUDA-core
+  // Stage 2 instead; the probe sets alone can come from either.
+  const bool per_cand = dbg && (dbg->cand_tok || dbg->cand_logit);
+  const bool tc = tc_eligible(idx, B, kTcMinBatchHead) && !per_cand && D.E_perm != nullptr;
   if (tc && s1fmt(idx) == FH_STAGE1_DENSE) {
     // Stage 1 on the tensor cores too: keys[q][k] = C[k]·h_q (+ the Gumbel term when sampling)
     fh::TcParams tp = {};
@@ -223,6 +231,10 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
       return cuda_fail(e, "tensor-core stage-1 launch");
     if ((e = fh::launch_select(keys, sel, B, D.c, p, st)) != cudaSuccess)
       return cuda_fail(e, "select launch");
+    if (dbg && dbg->sel &&
+        (e = cudaMemcpyAsync(dbg->sel, sel, (size_t)B * p * 4, cudaMemcpyDeviceToDevice, st)) !=
+            cudaSuccess)
+      return cuda_fail(e, "debug copy");
   } else {
     fh::Stage1Params s1 = stage1_params(idx, H, B, keys, ws);
     s1.sample = sample;
@@ -323,6 +335,15 @@ fh_status report(fh_status st, const char* fmt, ...) {
 // Used by fh_static.cu to report its own errors through fh_last_error().
 fh_status fh_internal_set_error(fh_status st, const char* msg) { return fail(st, "%s", msg); }
 
+// Used by fh_static.cu: the host-side argument checks of a head call (nothing is launched).
+fh_status fh_internal_check_head(const fh_index* idx, const void* H, int B, int p, const int32_t* out_tok) {
+  fh_status r = check_batch(idx, H, B);
+  if (r != FH_OK) return r;
+  if (!out_tok) return fail(FH_ERR_ARG, "out_tok is NULL");
+  if (p < 1 || p > idx->desc.c) return fail(FH_ERR_ARG, "p=%d outside [1, c=%lld]", p, (long long)idx->desc.c);
+  return FH_OK;
+}
+
 extern "C" {
 
 const char* fh_last_error(void) { return g_err; }
@@ -334,6 +355,7 @@ size_t fh_index_load_ws_bytes(const fh_index_desc* desc) {
 
 fh_status fh_index_load(const fh_index_desc* desc, void* ws, size_t ws_bytes, fh_stream stream,
                         fh_index** out) {
+  FH_NVTX_RANGE("fh_index_load");
   if (out) *out = nullptr;
   if (!desc || !out) return fail(FH_ERR_ARG, "desc or out is NULL");
   const fh_index_desc& D = *desc;
@@ -403,6 +425,7 @@ size_t fh_workspace_bytes(const fh_index* idx, int op, int B, int p, int T, int6
 }
 
 fh_status fh_ws_status(void* ws, fh_stream stream) {
+  FH_NVTX_RANGE("fh_ws_status");
   if (!ws) return fail(FH_ERR_WORKSPACE, "workspace is NULL");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint32_t status = 0;
@@ -430,6 +453,7 @@ fh_status fh_ws_status(void* ws, fh_stream stream) {
 
 fh_status fh_head_greedy(const fh_index* idx, const void* H, int B, int p, int32_t* out_tok,
                          void* ws, size_t ws_bytes, fh_stream stream, const fh_debug_out* dbg) {
+  FH_NVTX_RANGE("fh_head_greedy");
   return run_head(idx, H, B, p, 0, 1.0f, 0, 0, out_tok, ws, ws_bytes,
                   static_cast<cudaStream_t>(stream), dbg);
 }
@@ -437,6 +461,7 @@ fh_status fh_head_greedy(const fh_index* idx, const void* H, int B, int p, int32
 fh_status fh_head_sample(const fh_index* idx, const void* H, int B, int p, float tau, uint64_t seed,
                          uint64_t step, int32_t* out_tok, void* ws, size_t ws_bytes,
                          fh_stream stream, const fh_debug_out* dbg) {
+  FH_NVTX_RANGE("fh_head_sample");
   return run_head(idx, H, B, p, 1, tau, seed, step, out_tok, ws, ws_bytes,
                   static_cast<cudaStream_t>(stream), dbg);
 }
@@ -444,6 +469,7 @@ fh_status fh_head_sample(const fh_index* idx, const void* H, int B, int p, float
 fh_status fh_dense_head(const fh_index* idx, const void* H, int B, int sample, float tau,
                         uint64_t seed, uint64_t step, int32_t* out_tok, float* out_logits,
                         void* ws, size_t ws_bytes, fh_stream stream) {
+  FH_NVTX_RANGE("fh_dense_head");
   fh_status r = check_batch(idx, H, B);
   if (r != FH_OK) return r;
   if (!out_tok && !out_logits) return fail(FH_ERR_ARG, "out_tok and out_logits are both NULL");
@@ -497,6 +523,17 @@ fh_status fh_dense_head(const fh_index* idx, const void* H, int B, int sample, f
 fh_status fh_mc_token_prob(const fh_index* idx, const void* H, int B, const int32_t* targets, int T,
                            int p, float tau, int64_t N, uint64_t seed, double* out_mean,
                            double* out_se, void* ws, size_t ws_bytes, fh_stream stream) {
+  FH_NVTX_RANGE("fh_mc_token_prob");
+  return fh_mc_token_prob_range(idx, H, B, targets, T, p, tau, 0, N, seed, out_mean, out_se, ws,
+                                ws_bytes, stream);
+}
+
+fh_status fh_mc_token_prob_range(const fh_index* idx, const void* H, int B, const int32_t* targets,
+                                 int T, int p, float tau, int64_t i0, int64_t N, uint64_t seed,
+                                 double* out_mean, double* out_se, void* ws, size_t ws_bytes,
+                                 fh_stream stream) {
+  FH_NVTX_RANGE("fh_mc_token_prob_range");
+  if (i0 < 0 || i0 > (int64_t{1} << 40)) return fail(FH_ERR_ARG, "i0 outside [0, 2^40]");
   fh_status r = check_batch(idx, H, B);
   if (r != FH_OK) return r;
   const fh_index_desc& D = idx->desc;
@@ -560,6 +597,7 @@ fh_status fh_mc_token_prob(const fh_index* idx, const void* H, int B, const int3
   mp.c = D.c;
   mp.b = D.b;
   mp.N = N;
+  mp.i0 = i0;
   mp.B = B;
   mp.T = T;
   mp.p = p;
@@ -572,19 +610,36 @@ fh_status fh_mc_token_prob(const fh_index* idx, const void* H, int B, const int3
 
 fh_status fh_stage1_scores(const fh_index* idx, const void* H, int B, float* out_s, void* ws,
                            size_t ws_bytes, fh_stream stream) {
+  FH_NVTX_RANGE("fh_stage1_scores");
   fh_status r = check_batch(idx, H, B);
   if (r != FH_OK) return r;
   if (!out_s) return fail(FH_ERR_ARG, "out_s is NULL");
   if ((r = check_ws(ws, ws_bytes, kHeaderBytes)) != FH_OK) return r;
+  cudaError_t e;
+  if (tc_eligible(idx, B, kTcMinBatchHead) && s1fmt(idx) == FH_STAGE1_DENSE) {
+    // the kernel the fused head runs at these batches: keys mode of the tensor-core head
+    fh::TcParams tp = {};
+    tp.rows = idx->desc.c;
+    tp.d = idx->desc.d;
+    tp.B = B;
+    tp.b = 1;
+    tp.out_keys = out_s;
+    tp.status = status_of(ws);
+    if ((e = fh::launch_tc_head(idx->desc.C, H, tp, idx->num_sms, static_cast<cudaStream_t>(stream))) !=
+        cudaSuccess)
+      return cuda_fail(e, "tensor-core stage-1 launch");
+    return FH_OK;
+  }
   fh::Stage1Params s1 = stage1_params(idx, H, B, out_s, ws);
-  cudaError_t e = fh::launch_stage1(s1, idx->desc.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32,
-                                    idx->num_sms, static_cast<cudaStream_t>(stream), false);
+  e = fh::launch_stage1(s1, idx->desc.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms,
+                        static_cast<cudaStream_t>(stream), false);
   if (e != cudaSuccess) return cuda_fail(e, "stage-1 launch");
   return FH_OK;
 }
 
 fh_status fh_gumbel_keys(const float* s, int B, int64_t c, float tau, uint64_t seed, uint64_t step,
                          uint32_t rng_stream, float* out_keys, fh_stream stream) {
+  FH_NVTX_RANGE("fh_gumbel_keys");
   if (!s || !out_keys) return fail(FH_ERR_ARG, "s or out_keys is NULL");
   if (B < 1 || c < 1) return fail(FH_ERR_ARG, "empty input");
   if (!(tau > 0.0f)) return fail(FH_ERR_ARG, "tau must be > 0");
@@ -596,6 +651,7 @@ fh_status fh_gumbel_keys(const float* s, int B, int64_t c, float tau, uint64_t s
 
 fh_status fh_select_topp(const float* keys, int B, int64_t c, int p, int32_t* out_sel,
                          fh_stream stream) {
+  FH_NVTX_RANGE("fh_select_topp");
   if (!keys || !out_sel) return fail(FH_ERR_ARG, "keys or out_sel is NULL");
   if (B < 1 || B > 65535) return fail(FH_ERR_ARG, "B outside [1, 65535]");
   if (c < 1 || c > FH_MAX_C) return fail(FH_ERR_SHAPE, "c outside [1, %d]", FH_MAX_C);
@@ -607,6 +663,7 @@ fh_status fh_select_topp(const float* keys, int B, int64_t c, int p, int32_t* ou
 
 fh_status fh_gather_candidates(const fh_index* idx, const int32_t* sel, int B, int p,
                                int32_t* out_cand, fh_stream stream) {
+  FH_NVTX_RANGE("fh_gather_candidates");
   if (!idx || !sel || !out_cand) return fail(FH_ERR_ARG, "NULL argument");
   if (B < 1 || p < 1 || p > idx->desc.c) return fail(FH_ERR_ARG, "bad B or p");
   cudaError_t e = fh::launch_gather(idx->desc.C2T, idx->desc.b, sel, B, p, out_cand,
@@ -617,6 +674,7 @@ fh_status fh_gather_candidates(const fh_index* idx, const int32_t* sel, int B, i
 
 fh_status fh_candidate_logits(const fh_index* idx, const void* H, int B, const int32_t* cand,
                               int64_t P, float* out_z, fh_stream stream) {
+  FH_NVTX_RANGE("fh_candidate_logits");
   fh_status r = check_batch(idx, H, B);
   if (r != FH_OK) return r;
   if (!cand || !out_z) return fail(FH_ERR_ARG, "cand or out_z is NULL");
@@ -629,6 +687,7 @@ fh_status fh_candidate_logits(const fh_index* idx, const void* H, int B, const i
 
 fh_status fh_philox_u32(uint64_t seed, uint64_t step, uint32_t row, uint32_t rng_stream, int64_t n,
                         uint32_t* out, fh_stream stream) {
+  FH_NVTX_RANGE("fh_philox_u32");
   if (!out || n < 1) return fail(FH_ERR_ARG, "out is NULL or n < 1");
   if (n > (1LL << 32)) return fail(FH_ERR_ARG, "n > 2^32");
   cudaError_t e = fh::launch_philox(seed, step, row, rng_stream, n, out,

@@ -1,35 +1,42 @@
-// fh_head1.cu — the batch-1 FlashHead head as one persistent cooperative kernel (one block per SM).
+// fh_head1.cu — the batch-1 FlashHead head as one persistent kernel (one block per SM).
 //
 // At batch 1 the whole call moves ~66 MB (Llama-shaped head), about 10 µs of HBM time on a B200, so
 // every launch boundary and every serial step between the two bandwidth phases shows.  One kernel
-// therefore runs the whole path (FlashHead notes, overall architecture and Figure 1):
+// runs the whole path (FlashHead notes, overall architecture and Figure 1):
 //
-//   1. Stage 1: each block loads h, then bulk-copies its share of centroid rows (C, or the INT4
-//      nibbles) into its shared-memory ring at once, computes s = C·h (or the Gumbel key s/τ + G),
-//      writes the keys, and counts each key in a 1024-bin block histogram.  The bins cover a range
-//      fixed in advance from ‖h‖ (unit centroids give |s| <= ‖h‖; the Gumbel term lies in
-//      [-2.9, 16.7]); keys outside are clamped into the end bins, so the binning is monotone for any
-//      input and only its resolution depends on the range.  The block adds its counts to the global
-//      histogram with returning release adds, which give every key a distinct position in its bin.
-//   2. Grid barrier = histogram poll: every block polls the summed histogram until its counts reach c
-//      (bounded wait); the last poll holds the counts, the boundary bin follows by a block scan.
-//   3. Selection without a global list (FlashHead notes, Module 2): a certain cluster's rank in the
-//      Stage-2 list is (keys in higher bins) + (its position in its bin); the block that scored it
-//      writes its id at that rank as one 64-bit word tagged with the call's generation, and the
-//      boundary bin's (key, id) pairs likewise.  Block 0 ranks the boundary bin exactly (warp rank,
-//      or radix passes when crowded — then every block selects on all keys) and writes the ids it
-//      selects at the remaining ranks.  Each block polls only the words of its own rows, all before
-//      it issues any Stage-2 copy.
-//   4. Stage 2 (FlashHead notes, Module 1 and Figure 1): the block streams its slice of the p·b
-//      candidate rows, each together with the 16-byte C2T chunk holding its token id, computes the
-//      exact logits and keeps the arg-max of z (greedy, Eq. 2) or of z/τ + G' (sampling, Eq. 3).
-//   5. Each block folds its best (value, token) into one 64-bit atomicMax; the last block to arrive
-//      writes the token and clears the histogram, the selection words and the maximum.
+//   0. Prologue: one Stage-1 copy per warp (index data only) is issued at once; the kernel then waits
+//      for the preceding kernel of the stream (programmatic dependent launch) before it reads h or
+//      touches the workspace, so the centroid stream starts during the predecessor's tail; h is
+//      requested before the rest of the first copies (a small load queues behind the bulk copies in
+//      flight on its SM).
+//   1. Stage 1: each block streams its share of centroid rows (C, or the INT4 nibbles) through
+//      per-warp shared-memory rings, computes s = C·h (or the Gumbel key s/τ + G), and counts each key
+//      in a block histogram.  The bins are a monotone integer function of the exactly scaled key
+//      (key·2^-e with 2^e above the bound ‖h‖ of unit centroids, or ‖h‖/τ + 17 with the Gumbel term):
+//      64 bins per binade of |key·2^-e| in [2^-8, 1) on each side of zero, so a key's bin and its
+//      order inside the bin come from its bit pattern.
+//   2. Exchange: the block adds its counts to the global histogram (one returning add per non-empty
+//      bin, all in flight together), which gives every key a distinct position in its bin, and writes
+//      one tagged word (call tag, cluster id, order inside the bin) per key at (bin, position).
+//   3. Grid barrier = histogram poll: every block polls the summed histogram until its counts reach c
+//      (bounded wait).  The scan of the counts gives the boundary bin d* holding the p-th key, the
+//      number of keys above it, and for every rank of the Stage-2 list (bins from the top, positions
+//      inside a bin, then the boundary bin's taken keys) the word that names its cluster.
+//   4. Selection (FlashHead notes, Module 2): each block reads the words of the ranks its Stage-2
+//      rows need — one round of loads — and, when it has boundary ranks, the boundary bin's words,
+//      which it ranks exactly under (key desc, id asc).  A bin too full for the word table, or a
+//      boundary bin that is not a fine bin, sends every block to the full selection instead (all keys
+//      loaded, exact radix passes).
+//   5. Stage 2 (FlashHead notes, Module 1 and Figure 1): the block streams its slice of the p·b
+//      candidate rows (the cluster-major copy: a cluster is b contiguous rows), with the C2T rows of
+//      its clusters copied first for the token ids, computes the exact logits and keeps the arg-max of
+//      z (greedy, Eq. 2) or of z/τ + G' (sampling, Eq. 3).
+//   6. Each block posts its best (value, token) as one packed 64-bit word to its slot and counts itself
+//      in with a release add; block 0 waits for the G arrivals, reduces the slots, writes the token
+//      and clears the histogram.
 //
-// No small global load waits behind the bulk copies: h and the INT4 scales are loaded before the
-// Stage-1 copies, the rank words are polled before the Stage-2 copies, and token ids arrive inside the
-// row copies.  Stage-2 slots follow the rank order; the arg-max does not depend on it, and the
-// optional debug outputs are written in the canonical ascending order.
+// Stage-2 slots follow the rank order; the arg-max does not depend on it, and the optional debug
+// outputs are written in the canonical ascending order.
 #include "fh_device.cuh"
 #include "fh_kernels.cuh"
 #include "fh_select.cuh"
@@ -37,50 +44,83 @@
 
 namespace fh {
 
-constexpr int kHistBins = 1024;
-static_assert(kHead1BndMax == kSelCandMax, "boundary entries = ranked candidates");
+// Phase stamps for profiling builds (compile with -DFH_PHASE_TIMING; off in the library): thread 0 of
+// every block records %globaltimer at the phase boundaries of the batch-1 head.
+#ifdef FH_PHASE_TIMING
+__device__ unsigned long long g_h1_stamps[512 * 16];
+#define H1_STAMP(i)                                                                \
+  do {                                                                             \
+    if (threadIdx.x == 0) g_h1_stamps[blockIdx.x * 16 + (i)] = global_timer_ns();  \
+  } while (0)
+#else
+#define H1_STAMP(i) \
+  do {              \
+  } while (0)
+#endif
 
-struct Head1Layout {
-  uint32_t bars1, bars2, hs, sc, sel, hist, ownk, ownp, rank_cl, asc, tokc, ring, total;
-};
+constexpr int kHistBins = kHead1Bins;
+// Stage-1 rows each warp requests before the wait for the preceding kernel (the rest follow h).
+#ifndef FH_H1_PRE_ROWS
+#define FH_H1_PRE_ROWS 1
+#endif
+constexpr int kHead1PreRows = FH_H1_PRE_ROWS;
+#ifndef FH_H1_TOUCH
+#define FH_H1_TOUCH 0
+#endif
+constexpr int kCap = kHead1BucketCap;
+static_assert(kCap % 32 == 0 && kCap <= kSelCandMax, "bucket words are ranked by warps");
 
-__host__ __device__ inline uint32_t h1_align(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+// ------------------------------------------------------------------ key binning
+// x = key·scale with scale a power of two (exact for every |x| >= 2^-126), then, on each side of zero,
+// 64 bins per binade of |x| over [2^-8, 2^(-8 + 510/64)): the fine bins 1..510 (negative keys) and
+// 513..1022 (positive keys).  |x| < 2^-8 falls into the central bins 511 (negative) and 512 (zero and
+// positive; -0 and +0 alike), larger |x| into the end bins 0 and 1023.  Every step is an integer
+// operation on the bit pattern of x, so the bin is monotone in the key; inside a fine bin the low 17
+// bits of |x|'s pattern order the keys exactly (distinct keys have distinct x).
+constexpr uint32_t kFineLo = 0x3B800000u;  // bit pattern of 2^-8
+constexpr uint32_t kFineBins = 510u;
 
-template <int NT>
-__host__ __device__ inline Head1Layout head1_layout(uint32_t row2, int rows1_max, int nch4, int rmax,
-                                                    int slots2, uint32_t ring_bytes) {
-  // rows1_max: Stage-1 rows of the largest block (its own keys are kept); nch4: INT4 groups per row
-  const int sc_rows = nch4 ? rows1_max : 0;
-  Head1Layout L;
-  L.bars1 = 0;
-  L.bars2 = 1024;
-  L.hs = 2048;
-  L.sc = h1_align(L.hs + row2, 128);
-  L.sel = h1_align(L.sc + (uint32_t)sc_rows * nch4 * 2u + 4u, 128);
-  L.hist = h1_align(L.sel + (uint32_t)sizeof(SelectSmem<NT>), 16);
-  L.ownk = h1_align(L.hist + kHistBins * 4u, 16);
-  L.ownp = h1_align(L.ownk + (uint32_t)rows1_max * 4u, 16);
-  L.rank_cl = h1_align(L.ownp + (uint32_t)rows1_max * 4u, 16);
-  L.asc = h1_align(L.rank_cl + 2u * (uint32_t)rmax * 4u, 16);
-  L.tokc = h1_align(L.asc + 2u * (uint32_t)rmax * 4u, 16);
-  L.ring = h1_align(L.tokc + (uint32_t)slots2 * 16u, 128);
-  L.total = L.ring + ring_bytes;
-  return L;
-}
-
-// Monotone binning of a key into [0, kHistBins): the same function in Stage 1 and in the selection.
 struct Binning {
-  float lo, scale;
-  __device__ __forceinline__ uint32_t operator()(float x) const {
-    const float t = (x - lo) * scale;
-    return (uint32_t)min(kHistBins - 1, max(0, (int)t));
+  float scale;
+  __device__ __forceinline__ uint32_t operator()(float key) const {
+    const uint32_t u = __float_as_uint(key * scale);
+    const uint32_t a = u & 0x7FFFFFFFu;
+    const bool neg = (u >> 31) != 0u;
+    if (a < kFineLo) return (neg && a != 0u) ? 511u : 512u;
+    const uint32_t t = (a - kFineLo) >> 17;
+    if (neg) return t >= kFineBins ? 0u : 510u - t;
+    return t >= kFineBins ? 1023u : 513u + t;
+  }
+  // The order of a key inside its fine bin (17 bits; larger = larger key).
+  __device__ __forceinline__ uint32_t order_bits(float key) const {
+    const uint32_t u = __float_as_uint(key * scale);
+    const uint32_t off = ((u & 0x7FFFFFFFu) - kFineLo) & 0x1FFFFu;
+    return (u >> 31) ? 0x1FFFFu - off : off;
   }
 };
+
+__device__ __forceinline__ bool fine_bin(uint32_t d) {
+  return (d >= 1u && d <= 510u) || (d >= 513u && d <= 1022u);
+}
+
+// Every block computes the same ‖h‖ (same data, same reduction order) and from it the scale: the power
+// of two 2^-e with 2^e > R, R bounding |key| (unit centroids: |s| <= ‖h‖, with a 1/16 margin for INT4
+// centroids; sampling adds the Gumbel term, |G| <= 16.7 for the 23-bit uniforms).
+__device__ __forceinline__ Binning make_binning(const float hnorm, int sample, float tau) {
+  float r = hnorm * 1.0625f + 1e-30f;
+  if (sample) r = r / tau + 17.0f;
+  int e = 0;
+  frexpf(r, &e);  // r = m·2^e, m in [0.5, 1)
+  Binning bn;
+  bn.scale = ldexpf(1.0f, -e);
+  if (!(isfinite(bn.scale) && bn.scale > 0.0f)) bn.scale = 1.0f;
+  return bn;
+}
 
 // Smallest order-preserving key image u with bin(value of u) >= d (d in [1, kHistBins)), found by a
 // warp-wide 32-ary search over the images of finite floats; bin is monotone in u there, so a key is in
 // a bin >= d exactly when its image is >= the returned edge.  Called by a whole warp.
-__device__ __forceinline__ uint32_t bin_edge_image(const Binning& bin, uint32_t d) {
+__device__ __forceinline__ uint32_t bin_edge(const Binning& bin, uint32_t d) {
   const int lane = threadIdx.x & 31;
   uint32_t lo = 0x007FFFFFu, hi = 0xFF800000u;  // images of -inf and +inf
   if (bin(key_float(hi)) < d) return 0xFFFFFFFFu;  // no finite key reaches bin d
@@ -100,42 +140,6 @@ __device__ __forceinline__ uint32_t bin_edge_image(const Binning& bin, uint32_t 
   return hi;
 }
 
-// The same edge from the inverse of the binning, corrected by a few one-image steps; falls back to
-// the warp search when the correction does not settle.  Called by a whole warp.
-__device__ __forceinline__ uint32_t bin_edge(const Binning& bin, uint32_t d) {
-  bool ok = false;
-  uint32_t u = 0;
-  if (bin.scale > 0.0f) {
-    const float x0 = bin.lo + (float)d / bin.scale;
-    if (isfinite(x0)) {
-      u = float_key(x0);
-      for (int it = 0; it < 16 && u < 0xFF800000u && bin(key_float(u)) < d; ++it) ++u;
-      for (int it = 0; it < 16 && u > 0x00800000u && bin(key_float(u - 1u)) >= d; ++it) --u;
-      ok = u > 0x00800000u && u <= 0xFF800000u && bin(key_float(u)) >= d &&
-           bin(key_float(u - 1u)) < d;
-    }
-  }
-  return ok ? u : bin_edge_image(bin, d);
-}
-
-// Every block computes the same ‖h‖ (same data, same reduction order) and from it the binning.
-__device__ __forceinline__ Binning make_binning(const float hnorm, int sample, float tau) {
-  Binning bn;
-  const float r = hnorm * 1.0625f + 1e-30f;
-  const float lo = sample ? -r / tau - 3.0f : -r;
-  const float hi = sample ? r / tau + 17.0f : r;
-  bn.lo = lo;
-  bn.scale = (float)kHistBins / (hi - lo);
-  if (!(isfinite(bn.scale) && bn.scale > 0.0f)) bn.scale = 0.0f;  // everything in bin 0
-  return bn;
-}
-
-__device__ __forceinline__ uint32_t atom_add_release_u32(uint32_t* p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.release.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-  return old;
-}
-
 // HPT consecutive histogram bins (16- or 8-byte aligned) with one relaxed gpu-scope vector load.
 template <int HPT>
 __device__ __forceinline__ void load_bins_relaxed(const uint32_t* p, uint32_t (&hb)[HPT]) {
@@ -145,12 +149,6 @@ __device__ __forceinline__ void load_bins_relaxed(const uint32_t* p, uint32_t (&
   } else {
     asm volatile("ld.relaxed.gpu.global.v2.u32 {%0, %1}, [%2];" : "=r"(hb[0]), "=r"(hb[1]) : "l"(p) : "memory");
   }
-}
-
-__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
 }
 
 __device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
@@ -174,19 +172,21 @@ __device__ __forceinline__ unsigned long long poll_tagged(const unsigned long lo
   }
 }
 
+// Payload of a word: cluster id (bits 17..30) and the order inside the bin (bits 0..16).
+__device__ __forceinline__ int word_id(unsigned long long w) { return (int)((uint32_t)(w >> 17) & 0x3FFFu); }
+
 // Rank the m (<= 32*KP) boundary candidates under (key desc, id asc) and write the ids of the `need`
-// best into bsel_rank in rank order.  Every lane keeps KP candidates in registers (absent ones as
-// image 0, below every key); each warp ranks four candidates per pass, branch-free.
+// best into out in rank order.  Every lane keeps KP candidates in registers (absent ones as 0, below
+// every key); each warp ranks four candidates per pass, branch-free.
 template <int KP>
-__device__ __forceinline__ void rank_boundary(const float* cand_key, const int* cand_id, uint32_t m,
-                                              uint32_t need, int* bsel_rank, int lane, int warp,
-                                              int nwarps) {
+__device__ __forceinline__ void rank_boundary(const uint32_t* cand_key, const int* cand_id, uint32_t m,
+                                              uint32_t need, int* out, int lane, int warp, int nwarps) {
   uint32_t ck[KP];
   int cid[KP];
 #pragma unroll
   for (int u = 0; u < KP; ++u) {
     const uint32_t q = (uint32_t)(lane + 32 * u);
-    ck[u] = q < m ? __float_as_uint(cand_key[q]) : 0u;
+    ck[u] = q < m ? cand_key[q] : 0u;
     cid[u] = q < m ? cand_id[q] : 0x7FFFFFFF;
   }
   for (uint32_t i0 = (uint32_t)warp * 4u; i0 < m; i0 += (uint32_t)nwarps * 4u) {
@@ -195,7 +195,7 @@ __device__ __forceinline__ void rank_boundary(const float* cand_key, const int* 
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const uint32_t i = i0 + t;
-      ki[t] = i < m ? __float_as_uint(cand_key[i]) : 0xFFFFFFFFu;
+      ki[t] = i < m ? cand_key[i] : 0xFFFFFFFFu;
       ii[t] = i < m ? cand_id[i] : 0;
       rk[t] = 0u;
     }
@@ -207,19 +207,58 @@ __device__ __forceinline__ void rank_boundary(const float* cand_key, const int* 
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
       const uint32_t r = __reduce_add_sync(0xFFFFFFFFu, rk[t]);
-      if (lane == 0 && i0 + t < m && r < need) bsel_rank[r] = ii[t];
+      if (lane == 0 && i0 + t < m && r < need) out[r] = ii[t];
     }
   }
 }
+
+// ------------------------------------------------------------------ shared-memory layout
+
+struct Head1Layout {
+  uint32_t bars1, bars2, hs, sc, sel, hist, histg, ownk, ownp, rkid, asc, tokr, ring, total;
+};
+
+__host__ __device__ inline uint32_t h1_align(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+
+// Words of C2T copied per touched cluster: its b ids, widened to whole 16-byte chunks.
+__host__ __device__ inline int h1_tok_words(int b) { return (b + 6 + 3) / 4 * 4; }
+
+template <int NT>
+__host__ __device__ inline Head1Layout head1_layout(uint32_t row2, int rows1_max, int nch4, int rmax,
+                                                    int b, uint32_t ring_bytes) {
+  // rows1_max: Stage-1 rows of the largest block (its own keys are kept); nch4: INT4 groups per row;
+  // rmax: Stage-2 ranks (clusters) a block touches at most
+  const int sc_rows = nch4 ? rows1_max : 0;
+  Head1Layout L;
+  L.bars1 = 0;
+  L.bars2 = 1024;
+  L.hs = 2048;
+  L.sc = h1_align(L.hs + row2, 128);
+  L.sel = h1_align(L.sc + (uint32_t)sc_rows * nch4 * 2u + 4u, 128);
+  L.hist = h1_align(L.sel + (uint32_t)sizeof(SelectSmem<NT>), 16);
+  L.histg = h1_align(L.hist + kHistBins * 4u, 16);
+  L.ownk = h1_align(L.histg + kHistBins * 4u, 16);
+  L.ownp = h1_align(L.ownk + (uint32_t)rows1_max * 4u, 16);
+  L.rkid = h1_align(L.ownp + (uint32_t)rows1_max * 4u, 16);
+  L.asc = h1_align(L.rkid + (uint32_t)rmax * 4u, 16);
+  L.tokr = h1_align(L.asc + (uint32_t)rmax * 4u, 16);
+  L.ring = h1_align(L.tokr + (uint32_t)rmax * (uint32_t)h1_tok_words(b) * 4u, 128);
+  L.total = L.ring + ring_bytes;
+  return L;
+}
+
+// ------------------------------------------------------------------ the kernel
 
 template <int ELEM, int INT4_MCH, int NT, int KPT>
 __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int W = NT / 32;
+  constexpr int HPT = kHistBins / NT;  // histogram bins per thread
+  static_assert(HPT == 2 || HPT == 4, "bins per thread");
   __shared__ unsigned long long warp_best[W];
   __shared__ float red_s[W];
-  __shared__ bool abort_s, last_s;
-  __shared__ uint32_t dstar_s, above_s, total_s, edge_lo_s, edge_hi_s, m_s;
+  __shared__ bool abort_s;
+  __shared__ uint32_t dstar_s, above_s, total_s, m_s, edge_lo_s, edge_hi_s;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int G = gridDim.x, bid = blockIdx.x;
   const int64_t c = prm.c, d = prm.d;
@@ -235,34 +274,31 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   const int rows1_max = (int)((uc + uG - 1u) / uG);
   const int rows2_max = (int)(((uint32_t)P + uG - 1u) / uG);
   const int rmax = (int)(rows2_max / b) + 2;
+  const int tsw = h1_tok_words(b);
   const int K1 = prm.k1, K2 = prm.k2;
-  const Head1Layout L = head1_layout<NT>(row2, rows1_max, nch4, rmax, W * K2, prm.ring_bytes);
+  const Head1Layout L = head1_layout<NT>(row2, rows1_max, nch4, rmax, b, prm.ring_bytes);
   uint64_t* bars1 = reinterpret_cast<uint64_t*>(smem + L.bars1);
   uint64_t* bars2 = reinterpret_cast<uint64_t*>(smem + L.bars2);
+  uint64_t* tok_bar = &bars2[126];  // the C2T rows of the touched clusters
+  uint64_t* key_bar = &bars2[127];  // the key copy of the full selection
   uint8_t* hs = smem + L.hs;
   uint16_t* sc_s = reinterpret_cast<uint16_t*>(smem + L.sc);
   SelectSmem<NT>& sm = *reinterpret_cast<SelectSmem<NT>*>(smem + L.sel);
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(smem + L.hist);
+  uint32_t* histg_s = reinterpret_cast<uint32_t*>(smem + L.histg);  // keys in bins above each bin
   float* own_keys = reinterpret_cast<float*>(smem + L.ownk);
   uint32_t* own_pos = reinterpret_cast<uint32_t*>(smem + L.ownp);
-  int* rank_cl = reinterpret_cast<int*>(smem + L.rank_cl);
-  int* asc_of = reinterpret_cast<int*>(smem + L.asc);
-  uint4* tokc = reinterpret_cast<uint4*>(smem + L.tokc);
+  int* rk_id = reinterpret_cast<int*>(smem + L.rkid);   // cluster of each touched rank
+  int* asc_of = reinterpret_cast<int*>(smem + L.asc);   // its ascending position (debug outputs)
+  int32_t* tokr = reinterpret_cast<int32_t*>(smem + L.tokr);
   uint8_t* ring = smem + L.ring;
+  H1_STAMP(0);
 
-  // ------------------------------------------------------------------ prologue: h before any copy
-  uint4 hv[4];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int ch = tid + u * NT;
-    if (ch < nch2) hv[u] = __ldg(reinterpret_cast<const uint4*>(prm.H) + ch);
-  }
+  // ------------------------------------------------------------------ prologue
   const int64_t lo1 = uc * (uint32_t)bid / uG, hi1 = uc * (uint32_t)(bid + 1) / uG;
-  // this call's tags on its selection entries: 32 bits on the certain ranks, 18 on the boundary bin
-  const uint32_t tag = __ldcg(prm.gen) + 1u;
-  const uint32_t tag_b = (tag & 0x3FFFFu) | (uint32_t)((tag & 0x3FFFFu) == 0u);
-  uint32_t scv[4];  // INT4: this block's group scales, two per 32-bit word
-  const int nsc = INT4_MCH ? (int)((hi1 - lo1) * nch4) : 0;
+  const int nk = (int)(hi1 - lo1);
+  uint32_t scv[4];  // INT4: this block's group scales, two per 32-bit word (loaded before any copy)
+  const int nsc = INT4_MCH ? nk * nch4 : 0;
   const int sc_words = (nsc + 1) / 2;
   if constexpr (INT4_MCH > 0) {
 #pragma unroll
@@ -278,19 +314,41 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   }
   if (tid < W * K1) mbar_init(&bars1[tid], 1);
   if (tid < W * K2) mbar_init(&bars2[tid], 1);
-  uint64_t* bar_keys = &bars2[127];  // key copy of the full selection
-  if (tid == 0) mbar_init(bar_keys, 1);
+  if (tid == 0) {
+    mbar_init(tok_bar, 1);
+    mbar_init(key_bar, 1);
+  }
   fence_mbar_init();
   __syncthreads();
 
-  // ------------------------------------------------------------------ Stage 1
+  // Stage-1 rows of this warp: first1, first1 + W, ...; the first K1 are requested now (index data:
+  // no dependence on the preceding kernel).
   const int64_t first1 = lo1 + warp;
   const int n1 = (first1 < hi1) ? (int)((hi1 - first1 + W - 1) / W) : 0;
   uint8_t* ring1 = ring + (size_t)warp * K1 * row1;
   uint64_t* b1 = bars1 + warp * K1;
   const uint8_t* src1 = INT4_MCH ? static_cast<const uint8_t*>(static_cast<const void*>(prm.q4))
                                  : static_cast<const uint8_t*>(prm.C);
-  if (lane < K1 && lane < n1)  // the first K1 rows of the warp, one lane each
+  const int pre = min(K1, kHead1PreRows);
+  if (lane < pre && lane < n1)
+    issue_row(ring1 + (size_t)lane * row1, src1 + (size_t)(first1 + (int64_t)W * lane) * row1, row1,
+              &b1[lane]);
+
+  // h and the workspace may be written by the preceding kernel: wait for it (a no-op unless the
+  // launch allowed programmatic overlap).  A small load queues behind the bulk copies the SM has in
+  // flight, so h is requested before the rest of the first copies.
+  pdl_wait_prior();
+  uint4 hv[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int ch = tid + u * NT;
+    if (ch < nch2) hv[u] = __ldg(reinterpret_cast<const uint4*>(prm.H) + ch);
+  }
+  uint32_t tag = __ldcg(prm.gen) + 1u;  // this call's tag on its words (never 0)
+  if (tag == 0u) tag = 1u;
+  uint32_t arrive_base = 0u;  // arrivals of earlier calls (the reducer block waits for G more)
+  if (bid == 0 && tid == 0) arrive_base = __ldcg(prm.arrive);
+  if (lane >= pre && lane < K1 && lane < n1)
     issue_row(ring1 + (size_t)lane * row1, src1 + (size_t)(first1 + (int64_t)W * lane) * row1, row1,
               &b1[lane]);
 #pragma unroll
@@ -307,6 +365,7 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   }
   for (int i = tid; i < kHistBins; i += NT) hist_s[i] = 0u;
   __syncthreads();
+  H1_STAMP(1);
   // ‖h‖ (fixed reduction order, identical in every block) and the key binning
   float hsq = 0.0f;
   for (int ch = tid; ch < nch2; ch += NT) {
@@ -331,7 +390,9 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
 #pragma unroll
   for (int w = 0; w < W; ++w) hn2 += red_s[w];
   const Binning bin = make_binning(sqrtf(hn2), prm.sample, prm.tau);
+  const bool all = prm.p >= c;
 
+  // ------------------------------------------------------------------ Stage 1
   const uint32_t hs_addr = smem_addr(hs);
   for (int n = 0, slot = 0, phase = 0; n < n1; ++n) {
     if (!mbar_wait(&b1[slot], (uint32_t)phase, prm.status)) {
@@ -369,7 +430,7 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
         key = s / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 0u, (uint32_t)k));
       prm.keys[k] = key;
       own_keys[k - (int)lo1] = key;
-      own_pos[k - (int)lo1] = atomicAdd(&hist_s[bin(key_float(float_key(key)))], 1u);
+      if (!all) own_pos[k - (int)lo1] = atomicAdd(&hist_s[bin(key)], 1u);
     }
     if (++slot == K1) {
       slot = 0;
@@ -377,28 +438,38 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     }
   }
   __syncthreads();
-  // Add the block's counts to the global histogram.  The adds are releases (whoever sees a count also
-  // sees the keys this block wrote), and each returns the block's first position in that bin, so every
-  // key gets a distinct position among the keys of its bin.
-  for (int i = tid; i < kHistBins; i += NT) {
-    const uint32_t n = hist_s[i];
-    if (n) hist_s[i] = atom_add_release_u32(&prm.hist[i], n);
-  }
+  H1_STAMP(2);
 
-  // ------------------------------------------------------------------ histogram (grid barrier)
-  // The summed histogram is complete once its counts add up to c.  Every block polls it until then:
-  // the poll is the grid barrier, and its last round already holds the counts the selection needs.
-  constexpr int HPT = kHistBins / NT;  // histogram bins per thread
-  static_assert(HPT == 2 || HPT == 4, "bins per thread");
+  // ------------------------------------------------------------------ exchange and grid barrier
   uint32_t hb[HPT];
   uint32_t htot = 0, before = 0;
-  for (int i = tid; i < 1025; i += NT) sm.selbits[i] = 0u;
-  if (tid == 0) {  // (the polling loop's barriers order these before the boundary search)
-    sm.cand_count = 0u;
-    dstar_s = 0u;
-    above_s = 0u;
-  }
-  {
+  if (!all) {
+    // The block's first position in each non-empty bin: one returning add per bin, all in flight.
+    {
+      uint32_t cnt[HPT], base[HPT];
+#pragma unroll
+      for (int u = 0; u < HPT; ++u) cnt[u] = hist_s[tid + u * NT];
+#pragma unroll
+      for (int u = 0; u < HPT; ++u) base[u] = cnt[u] ? atomicAdd(prm.hist + tid + u * NT, cnt[u]) : 0u;
+#pragma unroll
+      for (int u = 0; u < HPT; ++u) hist_s[tid + u * NT] = base[u];
+    }
+    __syncthreads();
+    // One word per key at (bin, position): (tag, cluster id, order inside the bin).
+    if (tid < nk) {
+      const float key = own_keys[tid];
+      const uint32_t bn = bin(key);
+      const uint32_t pos = hist_s[bn] + own_pos[tid];
+      if (pos < (uint32_t)kCap)
+        st_relaxed_u64(prm.bucket + (size_t)bn * kCap + pos,
+                       ((unsigned long long)tag << 32) | ((unsigned long long)(lo1 + tid) << 17) |
+                           bin.order_bits(key));
+    }
+    H1_STAMP(3);
+    // The summed histogram is complete once its counts add up to c.  Every block polls it until then:
+    // the poll is the grid barrier, and its last round already holds the counts the selection needs.
+    for (int i = tid; i < 1025; i += NT) sm.selbits[i] = 0u;
+    if (tid == 0) sm.cand_count = 0u;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
       load_bins_relaxed<HPT>(prm.hist + tid * HPT, hb);
@@ -418,16 +489,24 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       return;
     }
   }
+  // Every block of this grid is resident now: the next kernel of the stream may start its prologue
+  // as blocks leave (it waits for this grid to complete before touching h or the workspace).
+  pdl_launch_dependents();
+  H1_STAMP(4);
 
   // ------------------------------------------------------------------ boundary bin
-  uint32_t* histg_s = reinterpret_cast<uint32_t*>(ring);  // keys in bins above each bin
-  const bool all = prm.p >= c;
-  {
+  if (tid == 0) {
+    dstar_s = 0u;
+    above_s = (uint32_t)c;
+    m_s = 0u;
+  }
+  __syncthreads();
+  if (!all) {
     uint32_t cum = total_s - before - htot;  // keys in bins above this thread's bins
 #pragma unroll
     for (int u = HPT - 1; u >= 0; --u) {
-      histg_s[tid * HPT + u] = cum;  // from here on: keys in bins above bin tid*HPT+u
-      if (!all && cum < (uint32_t)prm.p && cum + hb[u] >= (uint32_t)prm.p) {
+      histg_s[tid * HPT + u] = cum;  // keys in bins above bin tid*HPT+u
+      if (cum < (uint32_t)prm.p && cum + hb[u] >= (uint32_t)prm.p) {
         dstar_s = (uint32_t)(tid * HPT + u);
         above_s = cum;
         m_s = hb[u];
@@ -436,176 +515,144 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     }
     __syncthreads();
   }
-  const uint32_t dstar = all ? 0u : dstar_s;
-  const uint32_t above_n = all ? (uint32_t)c : above_s;
-  const uint32_t need = (uint32_t)prm.p - above_n;
-  const uint32_t m_total = all ? 0u : m_s;
-  // Stage-2 rows of this block: its share of the certain rows [c0, c1) and of the boundary rows
-  // [d0, d1) (global rows in list order: rank r = row / b, certain ranks first).  Local row l is
-  // c0 + l below nc and d0 + (l - nc) above, so certain rows stream while the boundary is resolved.
-  const int CR = (int)above_n * b, BR = (int)need * b;
-  const int c0 = (int)((uint32_t)CR * (uint32_t)bid / uG), c1 = (int)((uint32_t)CR * (uint32_t)(bid + 1) / uG);
-  const int d0 = CR + (int)((uint32_t)BR * (uint32_t)bid / uG);
-  const int d1 = CR + (int)((uint32_t)BR * (uint32_t)(bid + 1) / uG);
-  const int nc = c1 - c0, nr = nc + (d1 - d0);
-  const int rc0 = c0 / b, rc1 = (c1 + b - 1) / b;  // certain ranks touched
-  const int rb0 = d0 / b, rb1 = (d1 + b - 1) / b;  // boundary ranks touched
-  int* rk_c = rank_cl;
-  int* rk_b = rank_cl + rmax;
-  int* asc_c = asc_of;
-  int* asc_b = asc_of + rmax;
-  const bool want_dbg = prm.dbg_sel || prm.dbg_tok || prm.dbg_logit;
-
+  const uint32_t dstar = dstar_s;
+  const uint32_t above_n = above_s;
+  const uint32_t need = (uint32_t)prm.p - min(above_n, (uint32_t)prm.p);
+  const uint32_t m_total = m_s;
+  bool fast = true;
+  if (!all) {
+    // every bin from d* up must fit the word table, and a partly taken boundary bin must be a fine
+    // bin (its words then order the keys exactly)
+    bool over = false;
+#pragma unroll
+    for (int u = 0; u < HPT; ++u) over |= (uint32_t)(tid * HPT + u) >= dstar && hb[u] > (uint32_t)kCap;
+    over = __syncthreads_or(over);
+    fast = !over && (need == m_total || fine_bin(dstar));
+  }
   const uint8_t* E = static_cast<const uint8_t*>(prm.E);
   const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
   const bool perm = Ep != nullptr;
-  const int n2 = (warp < nr) ? (nr - warp + W - 1) / W : 0;
-  uint8_t* ring2 = ring + (size_t)warp * K2 * row2;
-  uint64_t* b2 = bars2 + warp * K2;
-  uint4* tokc_w = tokc + warp * K2;
-  auto global_row = [&](int l) { return l < nc ? c0 + l : d0 + (l - nc); };
-  auto row_e = [&](int g) {  // flat C2T index (= row of the cluster-major copy) of global row g
-    const int r = g / b;
-    const int cl = (r < (int)above_n) ? rk_c[r - rc0] : rk_b[r - rb0];
-    return cl * b + (g - r * b);
-  };
-  auto issue2 = [&](int n) {
-    const int slot = n % K2;
-    const int e = row_e(global_row(warp + W * n));
-    const int32_t* chunk = prm.C2T + (e & ~3);  // 16-byte chunk holding the token id
-    mbar_arrive_expect_tx(&b2[slot], row2 + 16u);
-    bulk_g2s(&tokc_w[slot], chunk, 16u, &b2[slot]);
-    const uint8_t* src = perm ? Ep + (size_t)e * row2 : E + (size_t)__ldg(prm.C2T + e) * row2;
-    bulk_g2s(ring2 + (size_t)slot * row2, src, row2, &b2[slot]);
-  };
-  const bool fast = all || m_total <= (uint32_t)kSelCandMax;
+#if FH_H1_TOUCH
+  if (perm && !all && tid < nk) {  // one 16-byte L2 prefetch per own certain cluster
+    const uint32_t bn = bin(own_keys[tid]);
+    if (bn > dstar || (bn == dstar && need == m_total))
+      asm volatile("cp.async.bulk.prefetch.L2.global [%0], 16;" ::"l"(Ep + (size_t)(lo1 + tid) * (size_t)b * row2)
+                   : "memory");
+  }
+#endif
 
-  if (fast) {
-    // ---------------------------------------------------------------- distributed selection
-    // A cluster's rank in the Stage-2 list is (keys in higher bins) + (its position in its bin), known
-    // to the block that scored it as soon as the histogram is: each block writes the ids of its
-    // certain clusters at their ranks, and the (key, id) of its boundary-bin clusters at their
-    // positions, each as one 64-bit word tagged with the call's tag.  Block 0 resolves the boundary
-    // bin and writes the ranks it fills the same way.  Every block polls only the words its own rows
-    // need, so no word is read by more than a few blocks: no counters, no fences, no hot spot.
-    const int nk = (int)(hi1 - lo1);
-    if (tid < nk) {
-      const uint32_t img = float_key(own_keys[tid]);
-      const uint32_t dg = bin(key_float(img));
-      const uint32_t pos = hist_s[dg] + own_pos[tid];
-      const unsigned long long tg = (unsigned long long)tag << 32;
-      const uint32_t id = (uint32_t)(lo1 + tid);
-      if (all || dg > dstar) {
-        st_relaxed_u64(prm.order + histg_s[dg] + pos, tg | id);
-      } else if (dg == dstar) {  // (18-bit tag, 14-bit id, key image)
-        st_relaxed_u64(prm.bnd + pos, ((unsigned long long)tag_b << 46) |
-                                      ((unsigned long long)id << 32) | img);
-      }
+  // This block's Stage-2 rows [r0, r1) of the rank-ordered list (row g: rank g / b, row g % b of
+  // that cluster) and the ranks they touch.
+  const int r0 = (int)((uint32_t)P * (uint32_t)bid / uG), r1 = (int)((uint32_t)P * (uint32_t)(bid + 1) / uG);
+  const int rk0 = r0 / b, rk1 = (r1 > r0) ? (r1 - 1) / b + 1 : rk0;
+  const int nrk = rk1 - rk0;
+  const bool want_dbg = prm.dbg_sel || prm.dbg_tok || prm.dbg_logit;
+  int* tab = reinterpret_cast<int*>(ring);  // debug: the whole list (ring free until Stage 2)
+
+  if (all) {
+    // every cluster is taken: rank r is cluster r
+    if (tid < nrk) {
+      rk_id[tid] = rk0 + tid;
+      asc_of[tid] = rk0 + tid;
     }
-    // Poll tagged words (each thread at most one of `words`, all loads of a round in flight together);
-    // false if a wait gave up (status set).
-    auto poll_words = [&](const unsigned long long* words, int n, int* dst) {
-      bool ok = true;
-      for (int q = tid; q < n; q += NT) dst[q] = (int)(uint32_t)poll_tagged(words + q, tag, prm.status, ok);
-      return ok;
+    if (prm.dbg_sel && bid == 0)
+      for (int q = tid; q < prm.p; q += NT) prm.dbg_sel[q] = q;
+  } else if (fast) {
+    // ---------------------------------------------------------------- selection from the words
+    // Rank r < above_n lives in the bin t0 = the lowest t with (keys above t) <= r, at position
+    // r - (keys above t0); ranks from above_n on are the boundary bin's taken keys.
+    auto certain_word = [&](uint32_t r, bool& ok) {
+      int lo = 0, hi = kHistBins - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (histg_s[mid] <= r) hi = mid;
+        else lo = mid + 1;
+      }
+      return word_id(poll_tagged(prm.bucket + (size_t)lo * kCap + (r - histg_s[lo]), tag, prm.status, ok));
     };
-    // Every word this block needs is read before any of its Stage-2 copies is issued: a small load
-    // issued behind a block's bulk copies waits until they have drained.
-    if (need > 0u) {
-      if (bid == 0) {
-        // The resolver: reads the boundary bin's keys once, ranks them exactly, and writes the ids
-        // of the `need` best at ranks above_n .. p - 1, tagged like the certain ones.
-        bool ok = true;
-        {
-          const uint32_t qa = (uint32_t)tid, qb = (uint32_t)(tid + NT);
-          uint32_t pend = (qa < m_total ? 1u : 0u) | (qb < m_total ? 2u : 0u);
-          const uint64_t t0 = global_timer_ns();
-          for (uint32_t it = 1; pend; ++it) {
-            unsigned long long v0 = 0ull, v1 = 0ull;
-            if (pend & 1u) v0 = ld_relaxed_u64(prm.bnd + qa);
-            if (pend & 2u) v1 = ld_relaxed_u64(prm.bnd + qb);
-            if ((pend & 1u) && (uint32_t)(v0 >> 46) == tag_b) {
-              sm.cand_key[qa] = __uint_as_float((uint32_t)v0);
-              sm.cand_id[qa] = (int)((uint32_t)(v0 >> 32) & 0x3FFFu);
-              pend &= ~1u;
-            }
-            if ((pend & 2u) && (uint32_t)(v1 >> 46) == tag_b) {
-              sm.cand_key[qb] = __uint_as_float((uint32_t)v1);
-              sm.cand_id[qb] = (int)((uint32_t)(v1 >> 32) & 0x3FFFu);
-              pend &= ~2u;
-            }
-            if (pend && (it & 15u) == 0u && global_timer_ns() - t0 > 500000000ull) {
-              set_status(prm.status, kStatusTimeout);
-              ok = false;
-              break;
-            }
-          }
+    const bool bnd_ranks = want_dbg || rk1 > (int)above_n;  // does this block need the boundary bin?
+    bool ok = true;
+    if (want_dbg) {
+      for (uint32_t r = tid; r < above_n; r += NT) tab[r] = certain_word(r, ok);
+    } else if (tid < nrk && (uint32_t)(rk0 + tid) < above_n) {
+      rk_id[tid] = certain_word((uint32_t)(rk0 + tid), ok);
+    }
+    int* bsel = reinterpret_cast<int*>(sm.selbits);  // boundary ids in rank order (need <= kCap)
+    if (bnd_ranks && need > 0u) {
+      const unsigned long long* bw = prm.bucket + (size_t)dstar * kCap;
+      if (need == m_total) {  // the whole bin is taken: any order will do, take the positions
+        if (tid < (int)m_total) bsel[tid] = word_id(poll_tagged(bw + tid, tag, prm.status, ok));
+      } else {
+        uint32_t* ckey = reinterpret_cast<uint32_t*>(sm.cand_key);
+        if (tid < (int)m_total) {
+          const unsigned long long w = poll_tagged(bw + tid, tag, prm.status, ok);
+          ckey[tid] = (uint32_t)(w & 0x1FFFFull) + 1u;  // 0 stays below every key
+          sm.cand_id[tid] = word_id(w);
         }
         if (!__syncthreads_and(ok)) return;
-        int* bsel_rank = reinterpret_cast<int*>(sm.selbits);
-        if (m_total <= 128u)
-          rank_boundary<4>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
-        else
-          rank_boundary<kSelCandMax / 32>(sm.cand_key, sm.cand_id, m_total, need, bsel_rank, lane, warp, W);
-        __syncthreads();
-        const unsigned long long tg = (unsigned long long)tag << 32;
-        for (uint32_t r = tid; r < need; r += NT)
-          st_relaxed_u64(prm.order + above_n + r, tg | (uint32_t)bsel_rank[r]);
+        rank_boundary<kCap / 32>(ckey, sm.cand_id, m_total, need, bsel, lane, warp, W);
       }
     }
-    // the certain and the boundary ranks of this block's rows (the resolver reads back its own words)
-    {
-      bool ok = poll_words(prm.order + rc0, rc1 - rc0, rk_c);
-      if (rb1 > rb0) ok = poll_words(prm.order + rb0, rb1 - rb0, rk_b) && ok;
-      if (!__syncthreads_and(ok)) return;
-    }
+    if (!__syncthreads_and(ok)) return;
     if (want_dbg) {
-      // canonical (ascending) positions: count the selected clusters below each of this block's
-      bool ok = true;
-      for (int q = tid; q < prm.p; q += NT) poll_tagged(prm.order + q, tag, prm.status, ok);
-      if (!__syncthreads_and(ok)) return;
-      auto sel_at = [&](int q) { return (int)(uint32_t)__ldcg(prm.order + q); };
-      const int ncr = rc1 - rc0, nbr = rb1 - rb0;
-      for (int t = warp; t < ncr + nbr; t += W) {
-        const int x = t < ncr ? rk_c[t] : rk_b[t - ncr];
+      for (uint32_t r = above_n + tid; r < (uint32_t)prm.p; r += NT) tab[r] = bsel[r - above_n];
+      __syncthreads();
+      if (tid < nrk) rk_id[tid] = tab[rk0 + tid];
+    } else if (tid < nrk && (uint32_t)(rk0 + tid) >= above_n) {
+      rk_id[tid] = bsel[rk0 + tid - (int)above_n];
+    }
+    __syncthreads();
+    if (want_dbg) {
+      // canonical (ascending) positions of this block's clusters, and the probe set
+      for (int t = warp; t < nrk; t += W) {
+        const int x = rk_id[t];
         uint32_t cnt = 0;
-        for (int q = lane; q < prm.p; q += 32) cnt += (uint32_t)(sel_at(q) < x);
+        for (int q = lane; q < prm.p; q += 32) cnt += (uint32_t)(tab[q] < x);
         cnt = __reduce_add_sync(0xFFFFFFFFu, cnt);
-        if (lane == 0) {
-          if (t < ncr) asc_c[t] = (int)cnt;
-          else asc_b[t - ncr] = (int)cnt;
-        }
+        if (lane == 0) asc_of[t] = (int)cnt;
       }
       if (prm.dbg_sel && bid == 0) {
         for (int q = tid; q < prm.p; q += NT) {
-          const int x = sel_at(q);
+          const int x = tab[q];
           uint32_t cnt = 0;
-          for (int y = 0; y < prm.p; ++y) cnt += (uint32_t)(sel_at(y) < x);
+          for (int y = 0; y < prm.p; ++y) cnt += (uint32_t)(tab[y] < x);
           prm.dbg_sel[cnt] = x;
         }
       }
-      __syncthreads();
-    }
-    if (lane < K2 && lane < n2) {
-      fence_proxy_async_smem();  // the ring was last read by Stage 1
-      issue2(lane);
     }
   } else {
     // ---------------------------------------------------------------- full selection (crowded bin)
-    // More than kSelCandMax keys share the boundary bin: every block loads all keys and selects
-    // with the block-wide selector (exact radix passes on the boundary bin).
-    const uint32_t keys_bytes = (uint32_t)((c * 4 + 15) / 16 * 16);
-    float* keys_s = reinterpret_cast<float*>(ring + kHistBins * 4);
-    // Every thread saw some of the release adds of the histogram: its acquire fence makes the keys
-    // of those blocks visible, and the barrier passes that on to thread 0, which copies them.
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+    // A bin from d* up holds more keys than the word table, or the boundary bin cannot order its keys
+    // from the words: every block loads all keys and selects with the block-wide selector (exact radix
+    // passes on the boundary bin).  The keys are visible once every block has arrived here.
+    if (tid == 0) {
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
+      uint32_t old;
+      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(prm.keys_ready) : "memory");
+      const uint32_t target = (old / uG + 1u) * uG;
+      const uint64_t t0 = global_timer_ns();
+      abort_s = false;
+      for (uint32_t it = 1;; ++it) {
+        uint32_t v;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(prm.keys_ready) : "memory");
+        if ((int32_t)(v - target) >= 0) break;
+        if ((it & 63u) == 0 && global_timer_ns() - t0 > 500000000ull) {
+          set_status(prm.status, kStatusTimeout);
+          abort_s = true;
+          break;
+        }
+      }
+    }
     __syncthreads();
+    if (abort_s) return;
+    const uint32_t keys_bytes = (uint32_t)((c * 4 + 15) / 16 * 16);
+    float* keys_s = reinterpret_cast<float*>(ring);
     if (tid == 0) {
       asm volatile("fence.proxy.async;" ::: "memory");
-      mbar_arrive_expect_tx(bar_keys, keys_bytes);
-      bulk_g2s(keys_s, prm.keys, keys_bytes, bar_keys);
+      mbar_arrive_expect_tx(key_bar, keys_bytes);
+      bulk_g2s(keys_s, prm.keys, keys_bytes, key_bar);
     }
-    if (!mbar_wait(bar_keys, 0u, prm.status)) return;
+    if (!mbar_wait(key_bar, 0u, prm.status)) return;
     uint32_t key[KPT];
     {
       const int kb = tid * KPT;
@@ -644,58 +691,92 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       int a = (int)(exa >> 32);
       for (uint32_t bits = sel; bits; bits &= bits - 1, ++a) {
         const int j = __ffs(bits) - 1;
-        if (st.certain >> j & 1u) {
-          if (rc >= rc0 && rc < rc1) {
-            rk_c[rc - rc0] = base + j;
-            asc_c[rc - rc0] = a;
-          }
-          ++rc;
-        } else {
-          if (rb >= rb0 && rb < rb1) {
-            rk_b[rb - rb0] = base + j;
-            asc_b[rb - rb0] = a;
-          }
-          ++rb;
+        int& r = (st.certain >> j & 1u) ? rc : rb;
+        if (r >= rk0 && r < rk1) {
+          rk_id[r - rk0] = base + j;
+          asc_of[r - rk0] = a;
         }
+        ++r;
         if (prm.dbg_sel && bid == 0) prm.dbg_sel[a] = base + j;
       }
     }
     __syncthreads();
-    if (lane < K2 && lane < n2) {
-      fence_proxy_async_smem();  // the ring was last read by the key copy
-      issue2(lane);
+  }
+  H1_STAMP(5);
+
+  // ------------------------------------------------------------------ Stage 2
+  // The C2T rows of the touched clusters first (one small copy each; b ids widened to 16-byte
+  // chunks), then this warp's first K2 candidate rows.
+  const int nr = r1 - r0;
+  const int n2 = (warp < nr) ? (nr - warp + W - 1) / W : 0;
+  uint8_t* ring2 = ring + (size_t)warp * K2 * row2;
+  uint64_t* b2 = bars2 + warp * K2;
+  if (tid == 0 && nrk > 0) {
+    uint32_t bytes = 0;
+    for (int i = 0; i < nrk; ++i) {
+      const int e0 = rk_id[i] * b;
+      bytes += (uint32_t)(((e0 + b + 3) & ~3) - (e0 & ~3)) * 4u;
+    }
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(tok_bar, bytes);
+    for (int i = 0; i < nrk; ++i) {
+      const int e0 = rk_id[i] * b;
+      const int s0 = e0 & ~3;
+      bulk_g2s(tokr + i * tsw, prm.C2T + s0, (uint32_t)(((e0 + b + 3) & ~3) - s0) * 4u, tok_bar);
     }
   }
-  __syncthreads();
-  // ------------------------------------------------------------------ Stage 2
+  auto token_of = [&](int q, int j) {  // rank q (global), row j of its cluster
+    const int e0 = rk_id[q - rk0] * b;
+    return tokr[(q - rk0) * tsw + (e0 & 3) + j];
+  };
+  if (!perm) {  // the rows are addressed through their token ids: wait for the C2T rows
+    const bool ok = nrk == 0 || mbar_wait(tok_bar, 0u, prm.status);
+    if (!__syncthreads_and(ok)) return;
+  }
+  auto issue2 = [&](int n) {
+    const int slot = n % K2;
+    const int g = r0 + warp + W * n;
+    const int q = g / b, j = g - q * b;
+    mbar_arrive_expect_tx(&b2[slot], row2);
+    const uint8_t* src = perm ? Ep + ((size_t)rk_id[q - rk0] * b + j) * row2
+                              : E + (size_t)token_of(q, j) * row2;
+    bulk_g2s(ring2 + (size_t)slot * row2, src, row2, &b2[slot]);
+  };
+  if (lane < K2 && lane < n2) {
+    fence_proxy_async_smem();  // the ring was last read by Stage 1 and the selection
+    issue2(lane);
+  }
   unsigned long long best = 0ull;
-  for (int n = 0, slot = 0, phase = 0; n < n2; ++n) {
+  bool tok_ok = true;
+  if (perm && n2 > 0 && lane == 0)  // the C2T rows went out ahead of every E row
+    tok_ok = mbar_wait(tok_bar, 0u, prm.status);
+  tok_ok = __shfl_sync(0xFFFFFFFFu, tok_ok, 0);
+  H1_STAMP(10);
+  for (int n = 0, slot = 0, phase = 0; n < n2 && tok_ok; ++n) {
     if (!mbar_wait(&b2[slot], (uint32_t)phase, prm.status)) {
       for (int m = n + 1; m < n2 && m < n + K2; ++m)
         mbar_wait(&b2[m % K2], (uint32_t)((m / K2) & 1), nullptr, 50000000ull);
       break;
     }
-    const int g = global_row(warp + W * n);
+    if (n == 0) H1_STAMP(6);
+    const int g = r0 + warp + W * n;
     const float z = warp_sum(row_dot_partial<ELEM>(smem_addr(ring2 + (size_t)slot * row2), hs_addr,
                                                    nch2, lane));
     __syncwarp();
     if (lane == 0) {
-      const int q = g / b;
-      const int e = row_e(g);
-      const uint4 ch = tokc_w[slot];
-      const uint32_t q4i = (uint32_t)(e & 3);
-      const uint32_t tok = q4i == 0 ? ch.x : q4i == 1 ? ch.y : q4i == 2 ? ch.z : ch.w;
       if (n + K2 < n2) {
         fence_proxy_async_smem();
         issue2(n + K2);
       }
+      const int q = g / b, j = g - q * b;
+      const uint32_t tok = (uint32_t)token_of(q, j);
       float val = z;
       if (prm.sample)
         val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 1u, tok));
       const unsigned long long pk = pack_best(val, tok);
       best = pk > best ? pk : best;
       if (want_dbg) {
-        const int ai = ((q < (int)above_n) ? asc_c[q - rc0] : asc_b[q - rb0]) * b + (g - q * b);
+        const int ai = asc_of[q - rk0] * b + j;
         if (prm.dbg_logit) prm.dbg_logit[ai] = z;
         if (prm.dbg_tok) prm.dbg_tok[ai] = (int32_t)tok;
       }
@@ -705,42 +786,78 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       phase ^= 1;
     }
   }
+  if (!tok_ok) {  // (status recorded) the E rows already requested land before the block leaves
+    for (int m = 0; m < n2 && m < K2; ++m)
+      mbar_wait(&b2[m % K2], 0u, nullptr, 50000000ull);
+    return;
+  }
 
   // ------------------------------------------------------------------ arg-max over the grid
+  // Every block posts its best (value, ~token) to its slot and counts itself in with a release add;
+  // block 0 waits for all G arrivals of this call, reduces the slots, writes the token and returns
+  // the histogram to zero for the next call.  No other block waits for anything here.
   if (lane == 0) warp_best[warp] = best;
   __syncthreads();
+  H1_STAMP(7);
   if (tid == 0) {
     unsigned long long bb = 0ull;
     for (int w = 0; w < W; ++w) bb = warp_best[w] > bb ? warp_best[w] : bb;
-    if (bb) atomicMax(prm.best, bb);
-    __threadfence();
-    const unsigned long long t = atomicAdd(prm.ticket, 1ull);
-    last_s = ((t + 1) % (unsigned long long)G) == 0ull;
+    st_relaxed_u64(prm.slots + bid, bb);
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(prm.arrive) : "memory");
+  }
+  if (bid != 0) return;
+  if (tid == 0) {
+    const uint32_t target = arrive_base + uG;
+    const uint64_t t0 = global_timer_ns();
+    abort_s = false;
+    for (uint32_t it = 1;; ++it) {
+      uint32_t a;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(a) : "l"(prm.arrive) : "memory");
+      if ((int32_t)(a - target) >= 0) break;
+      if ((it & 63u) == 0 && global_timer_ns() - t0 > 500000000ull) {
+        set_status(prm.status, kStatusTimeout);
+        abort_s = true;
+        break;
+      }
+    }
   }
   __syncthreads();
-  if (last_s) {
-    __threadfence();
-    for (int i = tid; i < kHistBins; i += NT) prm.hist[i] = 0u;
-    if (fast) {  // the next call starts from zeroed entries (the tags already tell calls apart)
-      for (uint32_t q = tid; q < (uint32_t)prm.p; q += NT) prm.order[q] = 0ull;
-      for (uint32_t q = tid; q < m_total; q += NT) prm.bnd[q] = 0ull;
-    }
-    if (tid == 0) *prm.gen = tag;
-    if (tid == 0) {
-      const unsigned long long fin = atomicAdd(prm.best, 0ull);
-      prm.out_tok[0] = (int32_t)best_id(fin);
-      atomicExch(prm.best, 0ull);
-    }
+  H1_STAMP(8);
+  if (abort_s) return;
+  unsigned long long mine = 0ull;
+  for (int i = tid; i < G; i += NT) {
+    const unsigned long long v = __ldcg(prm.slots + i);
+    mine = v > mine ? v : mine;
   }
+  mine = warp_max_u64(mine);
+  if (lane == 0) warp_best[warp] = mine;
+  for (int i = tid; i < kHistBins; i += NT) prm.hist[i] = 0u;
+  if (tag == 0xFFFFFFFFu) {  // the tags wrap after this call: no older word may alias a new tag
+    for (int i = tid; i < kHistBins * kCap; i += NT) prm.bucket[i] = 0ull;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    unsigned long long fin = 0ull;
+    for (int w = 0; w < W; ++w) fin = warp_best[w] > fin ? warp_best[w] : fin;
+    *prm.gen = tag;
+    prm.out_tok[0] = (int32_t)best_id(fin);
+  }
+  H1_STAMP(9);
 }
 
 // ------------------------------------------------------------------ launcher
+
+#ifdef FH_PHASE_TIMING
+extern "C" int fh_probe_head1_stamps(unsigned long long* host, int n) {
+  return (int)cudaMemcpyFromSymbol(host, g_h1_stamps, (size_t)n * 8);
+}
+#endif
 
 int head1_threads(int64_t c) { return c <= 256 * 32 ? 256 : (c <= 512 * 32 ? 512 : 0); }
 
 cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaStream_t st) {
   const int NT = head1_threads(prm.c);
-  if (NT == 0) return cudaErrorInvalidValue;
+  if (NT == 0 || prm.c > (1 << 14)) return cudaErrorInvalidValue;  // cluster ids travel in 14 bits
   const int W = NT / 32;
   const int G = num_sms;
   const uint32_t row2 = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
@@ -750,16 +867,16 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
   const int64_t P = (int64_t)prm.p * prm.b;
   if ((prm.c * prm.b) * (int64_t)G >= (int64_t{1} << 31)) return cudaErrorInvalidValue;  // 32-bit splits
   const int rows1_max = (int)((prm.c + G - 1) / G);
+  if (rows1_max > NT) return cudaErrorInvalidValue;  // one thread per own key
   if (int4 && (rows1_max * nch4 + 1) / 2 > 4 * NT) return cudaErrorInvalidValue;
   const int rows2_max = (int)((P + G - 1) / G);
   const int rmax = (int)(rows2_max / prm.b) + 2;
-  auto fixed_for = [&](int k2) {
-    return (NT == 256 ? head1_layout<256>(row2, rows1_max, nch4, rmax, W * k2, 0)
-                      : head1_layout<512>(row2, rows1_max, nch4, rmax, W * k2, 0)).total;
-  };
+  if (rmax > NT) return cudaErrorInvalidValue;
+  const int b = (int)prm.b;
+  const uint32_t fixed = (NT == 256 ? head1_layout<256>(row2, rows1_max, nch4, rmax, b, 0)
+                                    : head1_layout<512>(row2, rows1_max, nch4, rmax, b, 0)).total;
   const uint32_t budget = 220u * 1024u;
-  const int kcap = (1024 / 8 - 1) / W;  // barriers per stage (the last one of bars2 is the key copy's)
-  const uint32_t fixed = fixed_for(kcap);
+  const int kcap = (1024 / 8 - 2) / W;  // barriers per stage (the last two of bars2 are reserved)
   if (fixed + (uint32_t)W * (row2 > row1 ? row2 : row1) > budget) return cudaErrorInvalidValue;
   const uint32_t ring_bytes = (budget - fixed) / 128u * 128u;
   auto slots = [&](uint32_t row, int64_t rows) {
@@ -769,20 +886,24 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
     if (k > kcap) k = kcap;
     return (int)(k < 1 ? 1 : k);
   };
-  if (ring_bytes < (uint32_t)((prm.c * 4 + 15) / 16 * 16) + 4096u) return cudaErrorInvalidValue;
+  // the crowded-bin selection copies all keys into the ring, the debug outputs list the probe set there
+  if (ring_bytes < (uint32_t)((prm.c * 4 + 15) / 16 * 16)) return cudaErrorInvalidValue;
   prm.k1 = slots(row1, rows1_max);
   prm.k2 = slots(row2, rows2_max);
   prm.ring_bytes = ring_bytes;
-  const size_t smem = fixed_for(prm.k2) + ring_bytes;
+  const size_t smem = fixed + ring_bytes;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
+  // One block per SM.  The grid barrier needs every block resident: a programmatically overlapped
+  // launch lets this grid's blocks start only as the preceding grid's blocks leave, and this grid lets
+  // the next one start only after its own barrier, when all of its blocks are resident.
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const int kpt = (int)((prm.c + NT - 1) / NT);

@@ -533,16 +533,21 @@ __global__ void k_mc_zmax(const float* z, int64_t v, float tau, float* zmax) {
   }
 }
 
+// Z[q][k] = Σ_{u in cluster k} exp(z_u/τ - zmax_q): one warp per (query, cluster), lane j takes the
+// cluster's rows j, j+32, ... and a fixed shuffle tree sums them (deterministic).
 __global__ void k_mc_partition(const float* z, const int32_t* C2T, int64_t v, int64_t c, int64_t b,
                                float tau, const float* zmax, double* Z, int B) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < (int64_t)B * c;
-       i += (int64_t)gridDim.x * blockDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  for (int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; i < (int64_t)B * c; i += nw) {
     const int64_t q = i / c, k = i % c;
     const double m = (double)zmax[q];
     double acc = 0.0;
-    for (int64_t j = 0; j < b; ++j)
+    for (int64_t j = lane; j < b; j += 32)
       acc += exp((double)z[(size_t)q * v + C2T[k * b + j]] / (double)tau - m);
-    Z[i] = acc;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, off);
+    if (lane == 0) Z[i] = acc;
   }
 }
 
@@ -584,7 +589,7 @@ __global__ void __launch_bounds__(kMcThreads) k_mc_draws(const McParams prm) {
     uint32_t key[KPT];
 #pragma unroll
     for (int g = 0; g < KPT / 4; ++g) {
-      const uint4 w = philox_block(prm.seed, (uint64_t)i, (uint32_t)q, 2u, (uint32_t)((base >> 2) + g));
+      const uint4 w = philox_block(prm.seed, (uint64_t)(prm.i0 + i), (uint32_t)q, 2u, (uint32_t)((base >> 2) + g));
       const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -846,8 +851,8 @@ cudaError_t launch_mc(const McParams& prm, int num_sms, cudaStream_t st) {
   cudaError_t e;
   k_mc_cluster_of<<<1024, 256, 0, st>>>(prm.C2T, prm.v, prm.b, const_cast<int32_t*>(prm.cluster_of));
   k_mc_zmax<<<prm.B, 1024, 0, st>>>(prm.z, prm.v, prm.tau, prm.zmax);
-  k_mc_partition<<<1024, 256, 0, st>>>(prm.z, prm.C2T, prm.v, prm.c, prm.b, prm.tau, prm.zmax, prm.Z,
-                                       prm.B);
+  k_mc_partition<<<4 * num_sms, 256, 0, st>>>(prm.z, prm.C2T, prm.v, prm.c, prm.b, prm.tau, prm.zmax,
+                                               prm.Z, prm.B);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   int64_t gd = (4 * (int64_t)num_sms + prm.B - 1) / prm.B;
   if (gd > prm.N) gd = prm.N;

@@ -85,6 +85,7 @@ struct McParams {
   double* out_mean;            // B x T
   double* out_se;              // B x T
   int64_t v, c, b, N;
+  int64_t i0;                  // first draw index (draw i uses Philox step i0 + i)
   int B, T, p;
   float tau;
   uint64_t seed;
@@ -119,7 +120,8 @@ cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long l
                                cudaStream_t st);
 
 // The batch-1 persistent head (fh_head1.cu).
-constexpr int kHead1BndMax = 512;  // boundary-bin keys the distributed selection takes
+constexpr int kHead1Bins = 1024;       // Stage-1 key histogram
+constexpr int kHead1BucketCap = 64;    // tagged (cluster, key) words kept per histogram bin
 
 struct Head1Params {
   const void* C;               // c x d (dense Stage 1) or null
@@ -135,12 +137,12 @@ struct Head1Params {
   int sample;
   float tau;
   uint64_t seed, step;
-  unsigned long long* ticket;     // final-reduction arrivals (grows by gridDim.x per call)
-  unsigned long long* best;       // packed (key, ~token) maximum (zero between calls)
-  uint32_t* hist;                 // 1024-bin key histogram (zero between calls)
-  uint32_t* gen;                  // tag of the last completed call (a call tags its entries gen+1)
-  unsigned long long* order;      // p: (tag, cluster) at the rank of each cluster above the boundary bin
-  unsigned long long* bnd;        // kHead1BndMax: (tag, cluster, key image) of the boundary bin's keys
+  uint32_t* arrive;               // final-reduction arrivals (grows by gridDim.x per call)
+  unsigned long long* slots;      // gridDim.x packed (key, ~token) maxima, one per block
+  uint32_t* hist;                 // kHead1Bins-bin key histogram (zero between calls)
+  uint32_t* gen;                  // tag of the last completed call (a call tags its words gen+1)
+  uint32_t* keys_ready;           // arrivals once the keys are written (grows by gridDim.x per use)
+  unsigned long long* bucket;     // kHead1Bins x kHead1BucketCap tagged words (tag, cluster, key)
   int32_t* out_tok;
   int32_t* dbg_sel;            // p or null
   int32_t* dbg_tok;            // p*b or null

@@ -23,6 +23,7 @@
 
 #include "../../include/fh_kmeans.h"
 #include "fh_kernels.cuh"
+#include "fh_nvtx.cuh"
 #include "fh_kmeans_core.cuh"
 
 namespace fh {
@@ -494,14 +495,17 @@ size_t fh_kmeans_ws_bytes(int64_t v, int64_t d, int64_t c) {
 }
 
 fh_status fh_kmeans_build(fh_kmeans_args* args, void* ws, size_t ws_bytes, fh_stream stream) {
+  FH_NVTX_RANGE("fh_kmeans_build");
   return run_op(args, kBuild, ws, ws_bytes, stream);
 }
 
 fh_status fh_kmeans_assign(fh_kmeans_args* args, void* ws, size_t ws_bytes, fh_stream stream) {
+  FH_NVTX_RANGE("fh_kmeans_assign");
   return run_op(args, kAssign, ws, ws_bytes, stream);
 }
 
 fh_status fh_kmeans_update(fh_kmeans_args* args, void* ws, size_t ws_bytes, fh_stream stream) {
+  FH_NVTX_RANGE("fh_kmeans_update");
   return run_op(args, kUpdate, ws, ws_bytes, stream);
 }
 

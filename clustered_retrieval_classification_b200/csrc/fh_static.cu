@@ -10,6 +10,13 @@
 // Host code cannot use the array's name as a device address (in host code it is only a host-side
 // stand-in), so the address is looked up with cudaGetSymbolAddress, once per device with that device
 // current, and passed to the kernels as an ordinary workspace pointer.
+//
+// The array is used exactly like a workspace: it starts zeroed (a static device array is
+// zero-initialised when the module loads), every call returns the words that must start at zero
+// (histogram, arg-max, tickets) to zero before it ends and tags everything else with its call
+// generation, and a device-side error stays in the array's status word until fh_static_status reads
+// it and zeroes the control block again.  A call writes -1 to out_tok before it launches, so a call
+// that fails on the device leaves -1 there instead of a plausible token.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -27,31 +34,38 @@ void* g_scratch_addr[kMaxDevices] = {};
 
 }  // namespace
 
-// Defined in fh_api.cu: records the message returned by fh_last_error().
+// Defined in fh_api.cu: records the message returned by fh_last_error(), and the host-side argument
+// checks of a head call.
 fh_status fh_internal_set_error(fh_status st, const char* msg);
+fh_status fh_internal_check_head(const fh_index* idx, const void* H, int B, int p, const int32_t* out_tok);
 
-extern "C" fh_status fh_head_greedy_static(const fh_index* idx, const void* H, int p,
-                                           int32_t* out_tok, fh_stream stream) {
+// The array's device address on the current device (looked up on first use there).
+static fh_status static_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fh_internal_set_error(FH_ERR_CUDA, cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fh_internal_set_error(FH_ERR_UNSUPPORTED, "device ordinal too large");
-  void* scratch = nullptr;
-  {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!g_scratch_addr[dev]) {
-      void* addr = nullptr;
-      e = cudaGetSymbolAddress(&addr, g_static_scratch);
-      if (e != cudaSuccess || !addr) {
-        char msg[160];
-        snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch failed: %s",
-                 cudaGetErrorString(e));
-        return fh_internal_set_error(FH_ERR_CUDA, msg);
-      }
-      g_scratch_addr[dev] = addr;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* addr = nullptr;
+    e = cudaGetSymbolAddress(&addr, g_static_scratch);
+    if (e != cudaSuccess || !addr) {
+      char msg[160];
+      snprintf(msg, sizeof msg, "cudaGetSymbolAddress of the static scratch failed: %s",
+               cudaGetErrorString(e));
+      return fh_internal_set_error(FH_ERR_CUDA, msg);
     }
-    scratch = g_scratch_addr[dev];
+    g_scratch_addr[dev] = addr;
   }
+  *out = g_scratch_addr[dev];
+  return FH_OK;
+}
+
+extern "C" fh_status fh_head_greedy_static(const fh_index* idx, const void* H, int p,
+                                           int32_t* out_tok, fh_stream stream) {
+  // argument errors are found before anything is queued on the stream
+  fh_status r = fh_internal_check_head(idx, H, 1, p, out_tok);
+  if (r != FH_OK) return r;
   const size_t need = fh_workspace_bytes(idx, FH_OP_GREEDY, 1, p, 0, 0);
   if (need == 0) return fh_internal_set_error(FH_ERR_ARG, "invalid index handle or p");
   if (need > (size_t)FH_STATIC_SCRATCH_BYTES) {
@@ -60,10 +74,26 @@ extern "C" fh_status fh_head_greedy_static(const fh_index* idx, const void* H, i
              "holds %d bytes", need, p, (int)FH_STATIC_SCRATCH_BYTES);
     return fh_internal_set_error(FH_ERR_WORKSPACE, msg);
   }
-  // Every call shares the array and it keeps the previous call's contents: clear the part this call
-  // uses (its counters and histogram must start at zero).
-  e = cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream));
+  void* scratch = nullptr;
+  if ((r = static_scratch(&scratch)) != FH_OK) return r;
+  // A call that fails on the device (a bounded wait that gave up) never writes its token: it leaves
+  // this -1, and the error waits in the status word for fh_static_status.
+  cudaError_t e = cudaMemsetAsync(out_tok, 0xFF, sizeof(int32_t), static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fh_internal_set_error(FH_ERR_CUDA, cudaGetErrorString(e));
   return fh_head_greedy(idx, H, 1, p, out_tok, scratch, (size_t)FH_STATIC_SCRATCH_BYTES, stream,
                         nullptr);
+}
+
+extern "C" fh_status fh_static_status(fh_stream stream) {
+  void* scratch = nullptr;
+  const fh_status r = static_scratch(&scratch);
+  if (r != FH_OK) return r;
+  return fh_ws_status(scratch, stream);
+}
+
+extern "C" fh_status fh_static_scratch(void** dev_ptr, size_t* bytes) {
+  if (!dev_ptr || !bytes) return fh_internal_set_error(FH_ERR_ARG, "dev_ptr or bytes is NULL");
+  const fh_status r = static_scratch(dev_ptr);
+  if (r == FH_OK) *bytes = (size_t)FH_STATIC_SCRATCH_BYTES;
+  return r;
 }

@@ -43,6 +43,12 @@ class DebugOut(ct.Structure):
     _fields_ = [("sel", ct.c_void_p), ("cand_tok", ct.c_void_p), ("cand_logit", ct.c_void_p)]
 
 
+class CfDesc(ct.Structure):
+    """fh_cf_desc (include/fh_cfhead.h)."""
+    _fields_ = [("v", ct.c_int64), ("d", ct.c_int64), ("w", ct.c_int32), ("K", ct.c_int32),
+                ("E", ct.c_void_p), ("codebooks", ct.c_void_p), ("codes", ct.c_void_p)]
+
+
 class KmeansArgs(ct.Structure):
     """fh_kmeans_args (include/fh_kmeans.h)."""
     _fields_ = [("E", ct.c_void_p), ("dtype", ct.c_int32), ("v", ct.c_int64), ("d", ct.c_int64),
@@ -67,6 +73,7 @@ SIGNATURES = {
     "fh_head_greedy": (_i, [_p, _p, _i, _i, _p, _p, _sz, _p, _p]),
     "fh_head_sample": (_i, [_p, _p, _i, _i, _f, _u64, _u64, _p, _p, _sz, _p, _p]),
     "fh_mc_token_prob": (_i, [_p, _p, _i, _p, _i, _i, _f, _i64, _u64, _p, _p, _p, _sz, _p]),
+    "fh_mc_token_prob_range": (_i, [_p, _p, _i, _p, _i, _i, _f, _i64, _i64, _u64, _p, _p, _p, _sz, _p]),
     "fh_dense_head": (_i, [_p, _p, _i, _i, _f, _u64, _u64, _p, _p, _p, _sz, _p]),
     "fh_stage1_scores": (_i, [_p, _p, _i, _p, _p, _sz, _p]),
     "fh_gumbel_keys": (_i, [_p, _i, _i64, _f, _u64, _u64, _u32, _p, _p]),
@@ -75,6 +82,13 @@ SIGNATURES = {
     "fh_candidate_logits": (_i, [_p, _p, _i, _p, _i64, _p, _p]),
     "fh_philox_u32": (_i, [_u64, _u64, _u32, _u32, _i64, _p, _p]),
     "fh_head_greedy_static": (_i, [_p, _p, _i, _p, _p]),
+    "fh_static_status": (_i, [_p]),
+    "fh_static_scratch": (_i, [_p, _p]),
+    "fh_cf_load": (_i, [_p, _p]),
+    "fh_cf_free": (None, [_p]),
+    "fh_cf_workspace_bytes": (_sz, [_p, _i, _i]),
+    "fh_cf_head": (_i, [_p, _p, _i, _i, _i, _f, _u64, _u64, _p, _p, _sz, _p, _p, _p]),
+    "fh_cf_coarse_scores": (_i, [_p, _p, _i, _p, _p, _sz, _p]),
     "fh_kmeans_ws_bytes": (_sz, [_i64, _i64, _i64]),
     "fh_kmeans_build": (_i, [_p, _p, _sz, _p]),
     "fh_kmeans_assign": (_i, [_p, _p, _sz, _p]),
@@ -230,17 +244,23 @@ def dense_head(index: Index, H, sample=False, tau=1.0, seed=0, step=0, out=None,
     return out
 
 
-def mc_token_prob(index: Index, H, targets, p, tau, N, seed, ws=None, stream=None):
-    """Monte Carlo marginal probabilities: (mean [B, T] fp64, se [B, T] fp64)."""
+def mc_token_prob(index: Index, H, targets, p, tau, N, seed, ws=None, stream=None, i0=None):
+    """Monte Carlo marginal probabilities: (mean [B, T] fp64, se [B, T] fp64) over draws
+    [0, N), or [i0, i0 + N) when i0 is given."""
     _need(H, "H")
     _need(targets, "targets")
     B, T = targets.shape
     mean = torch.empty((B, T), dtype=torch.float64, device=H.device)
     se = torch.empty((B, T), dtype=torch.float64, device=H.device)
     ws = ws if ws is not None else index.workspace(FH_OP_MC, B, p, T, N)
-    _check(load().fh_mc_token_prob(index.handle, _ptr(H), B, _ptr(targets), T, p, float(tau), N,
-                                   seed, _ptr(mean), _ptr(se), _ptr(ws), ws.numel(),
-                                   _stream(stream)))
+    if i0 is None:
+        _check(load().fh_mc_token_prob(index.handle, _ptr(H), B, _ptr(targets), T, p, float(tau), N,
+                                       seed, _ptr(mean), _ptr(se), _ptr(ws), ws.numel(),
+                                       _stream(stream)))
+    else:
+        _check(load().fh_mc_token_prob_range(index.handle, _ptr(H), B, _ptr(targets), T, p, float(tau),
+                                             i0, N, seed, _ptr(mean), _ptr(se), _ptr(ws), ws.numel(),
+                                             _stream(stream)))
     return mean, se
 
 
@@ -306,6 +326,19 @@ def head_greedy_static(index: Index, H, p, out=None, stream=None):
     return out
 
 
+def static_status(stream=None):
+    """Raise if an allocation-free call recorded a device-side error in the static scratch (and zero
+    its control block, so that the next call starts clean)."""
+    _check(load().fh_static_status(_stream(stream)))
+
+
+def static_scratch():
+    """(device address, bytes) of the static scratch on the current device."""
+    ptr, n = ct.c_void_p(), ct.c_size_t()
+    _check(load().fh_static_scratch(ct.byref(ptr), ct.byref(n)))
+    return ptr.value, n.value
+
+
 def ws_status(ws, stream=None):
     """Raise if a previous call recorded a device-side error in this workspace."""
     _check(load().fh_ws_status(_ptr(ws), _stream(stream)))
@@ -338,6 +371,80 @@ def index_from_host(E, C, C2T, dtype: str, C_q4=None, C_scales=None, int4=False,
     q4 = device_array(C_q4, "u8", device) if C_q4 is not None else None
     sc = device_array(C_scales, "bf16", device) if C_scales is not None else None
     return Index(Ed, Cd, C2Td, q4, sc, int4=int4, cluster_major=cluster_major)
+
+
+# ----------------------------------------------------------------------------- coarse-fine head
+
+
+class CfIndex:
+    """A coarse-fine head index (include/fh_cfhead.h): E [v, d] bf16, codebooks [T, K, w] float32,
+    codes [T/8, v] int32 (the packed 4-bit index map, uint32 bit patterns).  Keeps them alive."""
+
+    def __init__(self, E, codebooks, codes):
+        for t, n in ((E, "E"), (codebooks, "codebooks"), (codes, "codes")):
+            _need(t, n)
+        if E.dtype != torch.bfloat16 or codebooks.dtype != torch.float32:
+            raise TypeError("E must be bfloat16 and codebooks float32")
+        self.E, self.codebooks, self.codes = E, codebooks, codes
+        self.v, self.d = E.shape
+        T, self.K, self.w = codebooks.shape
+        self.desc = CfDesc(self.v, self.d, self.w, self.K, E.data_ptr(), codebooks.data_ptr(),
+                           codes.data_ptr())
+        h = ct.c_void_p()
+        _check(load().fh_cf_load(ct.byref(self.desc), ct.byref(h)))
+        self.handle = h
+
+    def workspace_bytes(self, B, k) -> int:
+        n = load().fh_cf_workspace_bytes(self.handle, B, k)
+        if n == 0:
+            raise FlashHeadError(1, "invalid workspace request")
+        return n
+
+    def close(self):
+        if getattr(self, "handle", None):
+            load().fh_cf_free(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def cf_index_from_host(E, codebooks, codes, device="cuda") -> CfIndex:
+    """Upload a bf16 E (uint16 patterns), float32 codebooks and the packed uint32 index map."""
+    import numpy as np
+    cw = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint32).view(np.int32)).to(device)
+    return CfIndex(device_array(E, "bf16", device), device_array(codebooks, "f32", device), cw)
+
+
+def cf_head(index: CfIndex, H, k, sample=False, tau=1.0, seed=0, step=0, out=None, ws=None,
+            stream=None, debug=None):
+    """Coarse-fine head: int32 token ids [B].  debug: dict with optional "cand" (int32 [B, k]) and
+    "coarse" (float32 [B, v]) device tensors to fill."""
+    _need(H, "H")
+    B = H.shape[0]
+    out = out if out is not None else torch.empty(B, dtype=torch.int32, device=H.device)
+    if ws is None:
+        ws = torch.zeros(index.workspace_bytes(B, k), dtype=torch.uint8, device=H.device)
+    debug = debug or {}
+    _check(load().fh_cf_head(index.handle, _ptr(H), B, k, 1 if sample else 0, float(tau), seed, step,
+                             _ptr(out), _ptr(ws), ws.numel(), _stream(stream), _ptr(debug.get("cand")),
+                             _ptr(debug.get("coarse"))))
+    return out
+
+
+def cf_coarse_scores(index: CfIndex, H, ws=None, stream=None):
+    """Coarse scores float32 [B, v] (the first step of cf_head)."""
+    _need(H, "H")
+    B = H.shape[0]
+    if ws is None:
+        ws = torch.zeros(index.workspace_bytes(B, 1), dtype=torch.uint8, device=H.device)
+    out = torch.empty((B, index.v), dtype=torch.float32, device=H.device)
+    _check(load().fh_cf_coarse_scores(index.handle, _ptr(H), B, _ptr(out), _ptr(ws), ws.numel(),
+                                      _stream(stream)))
+    return out
 
 
 # ----------------------------------------------------------------------------- index builder

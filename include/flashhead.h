@@ -38,6 +38,8 @@
  *     returns a thread-local message describing the last non-FH_OK status of the calling thread.
  *   - Allocation.  No compute entry point allocates device memory: scratch space is the caller's
  *     workspace buffer, sized by fh_workspace_bytes.
+ *   - Profiling.  Every entry point marks its host-side extent with an NVTX range of its own name
+ *     (header-only NVTX v3: without an attached profiler a push or pop is a no-op call).
  *   - Tie rules.  Clusters are ordered by (score desc, cluster id asc), tokens by
  *     (logit desc, token id asc); -0.0 is treated as +0.0.  Inputs must be finite.
  *   - Random numbers.  Sampling uses Philox4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel random
@@ -158,7 +160,8 @@ const char* fh_last_error(void);
    out_tok: device, B int32.  dbg: optional intermediate outputs, or NULL.
    Execution (all paths compute the same thing): B = 1 runs one persistent kernel; BF16 batches of 12
    or more run Stage 1 and Stage 2 on the tensor cores, reading each needed E row once for the whole
-   batch (debug outputs force the per-query Stage 2 instead); other batches run per-query CUDA-core
+   batch (dbg->cand_tok or dbg->cand_logit force the per-query Stage 2 instead; dbg->sel alone does
+   not); other batches run per-query CUDA-core
    kernels.  The paths sum the fp32 logits in different orders, so their tokens can differ only where
    two candidates' logits are within that rounding (~1e-6 relative); each path is deterministic. */
 fh_status fh_head_greedy(const fh_index* idx, const void* H, int B, int p, int32_t* out_tok,
@@ -183,6 +186,16 @@ fh_status fh_mc_token_prob(const fh_index* idx, const void* H, int B, const int3
                            int p, float tau, int64_t N, uint64_t seed, double* out_mean,
                            double* out_se, void* ws, size_t ws_bytes, fh_stream stream);
 
+/* The same estimate over the draws i0 .. i0 + N - 1 (draw i uses step i of the FH_RNG_MC stream), so
+   that a long run can be split into ranges — on one device over time, or over several devices — and
+   recomputed bit for bit: the sum over consecutive ranges of N_r·mean_r equals N·mean of the whole
+   range (up to the rounding of the sums).  0 <= i0 <= 2^40; other arguments as fh_mc_token_prob,
+   which is this call with i0 = 0. */
+fh_status fh_mc_token_prob_range(const fh_index* idx, const void* H, int B, const int32_t* targets,
+                                 int T, int p, float tau, int64_t i0, int64_t N, uint64_t seed,
+                                 double* out_mean, double* out_se, void* ws, size_t ws_bytes,
+                                 fh_stream stream);
+
 /* Dense head over the whole vocabulary (FlashHead notes, Eq. 1–3): z = E·h_q for every token.
    sample == 0: out_tok[q] = argmax z; sample != 0: argmax of z_t/τ + G(seed, step, q, FH_RNG_STAGE2, t).
    out_logits: device B x v fp32 logits z, or NULL.  BF16 batches of 2 or more run on the tensor
@@ -195,7 +208,9 @@ fh_status fh_dense_head(const fh_index* idx, const void* H, int B, int sample, f
 /* Each runs one step of the path on its own, for step-by-step checking; the fused calls above
    run the same device code. */
 
-/* Stage-1 scores s = C·h_q (FlashHead notes, Figure 1 Stage 1), fp32.  out_s: device, B x c. */
+/* Stage-1 scores s = C·h_q (FlashHead notes, Figure 1 Stage 1), fp32.  out_s: device, B x c.
+   Runs the kernel the fused heads run at batch B: BF16 batches of 12 or more on the tensor cores,
+   the CUDA-core Stage-1 kernel otherwise. */
 fh_status fh_stage1_scores(const fh_index* idx, const void* H, int B, float* out_s,
                            void* ws, size_t ws_bytes, fh_stream stream);
 
@@ -233,15 +248,30 @@ fh_status fh_philox_u32(uint64_t seed, uint64_t step, uint32_t row, uint32_t rng
    implicit device synchronisation.  The call's scratch lives in a file-scope device array of
    FH_STATIC_SCRATCH_BYTES bytes that every GPU loading the library keeps until process exit.
    H: device, 1 x d; out_tok: device, 1 int32.  Allocates nothing: it calls no cudaMalloc/cudaFree
-   and no allocating library routine; it clears the part of the array it uses with cudaMemsetAsync.
+   and no allocating library routine.  Argument errors return before anything is queued.
+   The array is used like a workspace: it starts zeroed, and every call leaves the words that must
+   start at zero (histogram, arg-max, tickets) at zero again and tags the rest with its call
+   generation.  The call first writes -1 to out_tok, so a call that fails on the device (a bounded
+   wait that gave up) leaves -1 there; its error stays in the array's status word until
+   fh_static_status reports it and zeroes the control block (until then later calls fail too).
    The first call on a device looks up the array's device address (cudaGetSymbolAddress, with that
    device current); make that first call before any stream capture.  Calls share the one array, so
    calls that overlap in time on the GPU (on different streams) race; serialise them.
-   Returns FH_ERR_WORKSPACE with a message when the index needs more scratch than the array holds
-   (about 4*c + 12*p + 15 KiB bytes: every c up to FH_MAX_C at p = 512, about 15,000 at p = c). */
-enum { FH_STATIC_SCRATCH_BYTES = 262144 };
+   Returns FH_ERR_WORKSPACE with a message when the index needs more scratch than the array holds:
+   4·(c + p) bytes plus about 530 KiB for c <= 16384 (the batch-1 kernel's word table), plus about
+   7 KiB above; every index with c + p up to about 31,000 fits. */
+enum { FH_STATIC_SCRATCH_BYTES = 655360 };
 fh_status fh_head_greedy_static(const fh_index* idx, const void* H, int p, int32_t* out_tok,
                                 fh_stream stream);
+
+/* Read and clear the status word of the current device's static scratch (synchronises `stream`):
+   FH_OK, or the device-side error of an earlier fh_head_greedy_static call (FH_ERR_TIMEOUT), after
+   which the array's control block is zeroed again, as fh_ws_status does for a workspace. */
+fh_status fh_static_status(fh_stream stream);
+
+/* The device address and size of the current device's static scratch, for diagnostics and tests
+   (writing to it while calls run races with them). */
+fh_status fh_static_scratch(void** dev_ptr, size_t* bytes);
 
 #ifdef __cplusplus
 }

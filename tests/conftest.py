@@ -36,3 +36,21 @@ def fh():
     from clustered_retrieval_classification_b200 import flashhead
     flashhead.load()
     return flashhead
+
+
+@pytest.fixture(scope="session")
+def llama_host():
+    """The Llama-3.2-1B-shaped synthetic index (v=128256, d=2048, c=8016, p=512) and 64 queries,
+    built once per session on the host."""
+    from clustered_retrieval_classification_b200 import synth
+    cfg = synth.CONFIGS["llama"]
+    return synth.make_index(cfg), synth.make_queries(cfg, 64)
+
+
+@pytest.fixture(scope="session")
+def gemma_host():
+    """The Gemma-3-1B-shaped synthetic index with INT4 Stage-1 centroids (v=262144, d=1152,
+    c=16384, p=1024) and 32 queries, built once per session on the host."""
+    from clustered_retrieval_classification_b200 import synth
+    cfg = synth.CONFIGS["gemma"]
+    return synth.make_index(cfg), synth.make_queries(cfg, 32)

@@ -8,7 +8,11 @@ Tolerances (fp32 accumulation of BF16 products against float64):
     the clusters that differ must lie within 4e-3 of the threshold;
   * a token id must be identical whenever the sets agree and the oracle's top-1 margin exceeds 4e-3;
     otherwise the token must be a near-maximum (within 4e-3) of the oracle's decision keys over the
-    candidates the GPU used.
+    candidates the GPU used;
+  * Monte Carlo means (same Philox draws on both sides) within max(1e-9, 1e-3·mean, 0.1·se) and
+    standard errors within max(1e-12, 1e-2·se): relative bounds, so that a target of probability
+    ~1/v is checked as closely as a likely one.  The slack covers draws whose probe sets differ
+    because the GPU forms the keys in fp32 (a near-tie at the p-th key).
 """
 
 import numpy as np
@@ -48,3 +52,10 @@ def check_tokens(gpu_tok, orc_tok, tok_margin, same_set, valid_fn, tol=MARGIN):
         best, mine = valid_fn(q, int(gpu_tok[q]))
         assert mine >= best - tol, f"query {q}: GPU token is not a near-maximum"
     return differ
+
+
+def check_mc(mean, se, o):
+    """GPU Monte Carlo estimates against the oracle's on the same draws (see the module docstring)."""
+    tol = np.maximum(np.maximum(1e-9, 1e-3 * np.abs(o["mean"])), 0.1 * o["se"])
+    assert np.all(np.abs(mean - o["mean"]) <= tol), (mean, o["mean"], tol)
+    assert np.all(np.abs(se - o["se"]) <= np.maximum(1e-12, 1e-2 * o["se"])), (se, o["se"])

@@ -8,7 +8,8 @@ import pytest
 import torch
 
 from clustered_retrieval_classification_b200 import synth
-from parity import LOGIT_TOL, MARGIN, check_sets, check_tokens
+from headcheck import check_head as _check_head, dev, load
+from parity import LOGIT_TOL, MARGIN, check_mc
 
 pytestmark = pytest.mark.gpu
 
@@ -17,16 +18,6 @@ DEV = "cuda"
 
 def widen(a, dtype):
     return synth.stored_to_f64(a, dtype)
-
-
-def dev(a, kind):
-    from clustered_retrieval_classification_b200 import flashhead as F
-    return F.device_array(a, kind, DEV)
-
-
-def load(fh, idx, int4=False, cluster_major=True):
-    return fh.index_from_host(idx.E, idx.C, idx.C2T, idx.cfg.dtype, idx.C_q4, idx.C_scales,
-                              int4=int4, cluster_major=cluster_major)
 
 
 # ----------------------------------------------------------------------------- fixtures
@@ -143,49 +134,6 @@ def test_gather_and_candidate_logits(fh, orc, mid):
 # ----------------------------------------------------------------------------- fused head
 
 
-def _run_head(fh, I, Hd, p, sample, tau, seed, step, P, B):
-    dbg = dict(sel=torch.empty((B, p), dtype=torch.int32, device=DEV),
-               cand_tok=torch.empty((B, P), dtype=torch.int32, device=DEV),
-               cand_logit=torch.empty((B, P), dtype=torch.float32, device=DEV))
-    if sample:
-        tok = fh.head_sample(I, Hd, p, tau, seed, step, debug=dbg)
-    else:
-        tok = fh.head_greedy(I, Hd, p, debug=dbg)
-    torch.cuda.synchronize()
-    return tok.cpu().numpy(), {k: v.cpu().numpy() for k, v in dbg.items()}
-
-
-def _check_head(fh, orc, idx, H, p, sample=False, tau=1.0, seed=0, step=0, batch=None,
-                cluster_major=True, int4=False):
-    cfg = idx.cfg
-    I = load(fh, idx, int4=int4, cluster_major=cluster_major)
-    B = batch or H.shape[0]
-    Hq = H[:B]
-    P = p * cfg.b
-    tok, dbg = _run_head(fh, I, dev(Hq, cfg.dtype), p, sample, tau, seed, step, P, B)
-    o = orc.head(idx, Hq, p, sample=sample, tau=tau, seed=seed, step=step, use_int4=int4)
-    s = orc.stage1_scores(idx.C if not int4 else None, cfg.dtype, Hq, cfg.c, cfg.d,
-                          q4=idx.C_q4 if int4 else None, scales=idx.C_scales if int4 else None)
-    keys = orc.gumbel_keys(s, tau, seed, step, 0) if sample else s
-    n_set = check_sets(dbg["sel"], o["sel"], keys, o["set_margin"])
-    same = [set(dbg["sel"][q]) == set(o["sel"][q]) for q in range(B)]
-    for q in range(B):
-        if same[q]:
-            assert np.array_equal(dbg["cand_tok"][q], o["cand"][q])
-            assert np.abs(dbg["cand_logit"][q] - o["z"][q]).max() <= LOGIT_TOL
-
-    def valid(q, t):
-        cand = dbg["cand_tok"][q:q + 1]
-        z = orc.logits(idx.E, cfg.dtype, Hq[q:q + 1], cand)[0]
-        if sample:
-            g = np.array([orc.gumbel(orc.draw_u32(seed, step, q, 1, int(u))) for u in cand[0]])
-            z = z / tau + g
-        return z.max(), z[list(cand[0]).index(t)]
-
-    n_tok = check_tokens(tok, o["tok"], o["tok_margin"], same, valid)
-    return n_set, n_tok
-
-
 def test_greedy_tiny_fp32_batch1(fh, orc, tiny):
     idx, H = tiny
     for q in range(0, 64, 3):
@@ -283,9 +231,7 @@ def test_mc_matches_oracle(fh, orc):
     mean, se = fh.mc_token_prob(I, dev(H, "bf16"), dev(targets, "i32"), cfg.p, 1.0, N, synth.MC_SEED)
     mean, se = mean.cpu().numpy(), se.cpu().numpy()
     o = orc.mc(idx, H, targets, cfg.p, 1.0, synth.MC_SEED, n_draws=N)
-    tol = np.maximum(1e-4, 0.1 * o["se"])
-    assert np.all(np.abs(mean - o["mean"]) <= tol), (mean, o["mean"])
-    assert np.all(np.abs(se - o["se"]) <= np.maximum(1e-5, 0.1 * o["se"]))
+    check_mc(mean, se, o)
 
 
 def test_mc_p_equals_c_is_dense_softmax(fh):
@@ -400,9 +346,9 @@ def test_workspace_status_clean(fh, mid):
 
 
 @pytest.fixture(scope="module")
-def llama():
-    cfg = synth.CONFIGS["llama"]
-    return synth.make_index(cfg), synth.make_queries(cfg, 4)
+def llama(llama_host):
+    idx, H = llama_host
+    return idx, H[:4]
 
 
 def test_llama_full_size_batch1_sampled(fh, orc, llama):

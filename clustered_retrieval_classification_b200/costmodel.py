@@ -45,3 +45,12 @@ def dense_bytes(v: int, d: int, B: int, elem_bytes: int) -> int:
 def head_flops(d: int, c: int, p: int, b: int, B: int) -> int:
     """Multiply-adds ×2 of the method proper: B·(c + p·b)·d."""
     return 2 * B * (c + p * b) * d
+
+
+def cf_bytes(v: int, d: int, w: int, K: int, k: int, B: int, unique_candidates: int) -> int:
+    """Coarse-fine head (page "Fast LM Head via Coarse-Fine Decomposition and Tile-Wise Weight
+    Clustering"): the 4-bit index map once (d/w codes per token, half a byte each), the fp32
+    codebooks once, the E rows of the distinct candidates of the batch once (BF16), the B hidden
+    vectors and the B token ids."""
+    T = d // w
+    return v * T // 2 + T * K * w * 4 + unique_candidates * d * 2 + B * d * 2 + B * 4

@@ -71,6 +71,22 @@ def test_host_side_argument_checks(lib):
     assert L.fh_philox_u32(0, 0, 0, 0, 0, None, None) == 1
 
 
+def test_cfhead_host_side_argument_checks(lib):
+    """Coarse-fine head (include/fh_cfhead.h): shapes and arguments are checked before any CUDA call."""
+    from clustered_retrieval_classification_b200 import flashhead as F
+    L = F.load()
+    out = ct.c_void_p()
+    d = F.CfDesc(1000, 72, 8, 16, 16, 16, 16)
+    assert L.fh_cf_load(ct.byref(d), ct.byref(out)) == 2        # d not a multiple of 8 tiles
+    d = F.CfDesc(1000, 64, 8, 17, 16, 16, 16)
+    assert L.fh_cf_load(ct.byref(d), ct.byref(out)) == 2        # K > 16: codes are 4 bits
+    d = F.CfDesc(1000, 64, 8, 16, 16, None, 16)
+    assert L.fh_cf_load(ct.byref(d), ct.byref(out)) == 1        # codebooks missing
+    assert b"codebooks" in L.fh_last_error()
+    assert L.fh_cf_workspace_bytes(None, 1, 1) == 0
+    assert L.fh_cf_head(None, None, 1, 1, 0, 1.0, 0, 0, None, None, 0, None, None, None) == 1
+
+
 def test_builder_host_side_argument_checks(lib):
     """Index builder (include/fh_kmeans.h): sizes and arguments are checked before any CUDA call."""
     from clustered_retrieval_classification_b200 import flashhead as F
@@ -94,7 +110,7 @@ def test_builder_host_side_argument_checks(lib):
 
 
 @pytest.mark.parametrize("struct,pyname", [("fh_index_desc", "IndexDesc"), ("fh_debug_out", "DebugOut"),
-                                           ("fh_kmeans_args", "KmeansArgs")])
+                                           ("fh_kmeans_args", "KmeansArgs"), ("fh_cf_desc", "CfDesc")])
 def test_binding_structs_match_the_headers(tmp_path, struct, pyname):
     """Every field of the binding's ctypes structures sits at the offset the C compiler gives it."""
     import subprocess
@@ -102,7 +118,8 @@ def test_binding_structs_match_the_headers(tmp_path, struct, pyname):
     py = getattr(F, pyname)
     fields = [f[0] for f in py._fields_]
     src = tmp_path / "layout.c"
-    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fh_kmeans.h"', "int main(void) {",
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fh_kmeans.h"', '#include "fh_cfhead.h"',
+             "int main(void) {",
              f'  printf("%zu\\n", sizeof({struct}));']
     lines += [f'  printf("%zu\\n", offsetof({struct}, {f}));' for f in fields]
     lines += ["  return 0;", "}"]

@@ -41,12 +41,10 @@ from clustered_retrieval_classification_b200 import costmodel, synth  # noqa: E4
 # Llama-3.2-1B with c=8016, p=512, batch 1) -> 2500 tokens/s.  Context from other hardware.
 PAGES_TOKENS_PER_S = 1.0 / 0.40e-3
 
-# DRAM traffic per launch from the committed ncu captures (profiles/), valid only for the kernel
-# sources they were taken on (sha1 of the csrc files); null otherwise.
-TRAFFIC = {
-    # profiles/k_head1_llama_batch1.md: dram__bytes_read.sum + dram__bytes_write.sum of one launch
-    (1, "2d156eb1e20e"): 66_547_456 + 565_760,
-}
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum of one ncu-captured launch
+# of the batch-1 kernel), valid only for the kernel sources it was taken on (sha1 of their code);
+# null otherwise.
+TRAFFIC = {}
 
 L2_FLUSH_BYTES = 256 << 20
 
@@ -173,47 +171,58 @@ class Timer:
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
-    def b2b(self, step_fn, K, W, sampler=None, graph_calls=8):
-        """step_fn(k) issues call k.  Calls are captured in a CUDA graph of `graph_calls` calls when
-        possible (else run eagerly).  Returns (total ms for K calls, mode)."""
-        g = None
+    def b2b(self, step_fn, K, W, sampler=None, graph_calls=8, repeats=1):
+        """step_fn(k) issues call k.  Exactly K calls are timed per repeat: K // graph_calls replays of
+        a CUDA graph of `graph_calls` calls plus one replay of a graph of the remaining K % graph_calls
+        (eager calls when capture fails).  Returns (list of total ms per repeat, K, mode)."""
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
+        reps, rem = divmod(K, graph_calls)
+        graphs = []
         try:
             with torch.cuda.stream(s):
                 for k in range(graph_calls):
                     step_fn(k)
             torch.cuda.synchronize()
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=s):
-                for k in range(graph_calls):
-                    step_fn(k)
+            for n, k0 in ((graph_calls, 0), (rem, graph_calls)):
+                if n == 0:
+                    graphs.append(None)
+                    continue
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s):
+                    for k in range(n):
+                        step_fn(k0 + k)
+                graphs.append(g)
             torch.cuda.synchronize()
         except Exception:
-            g = None
+            graphs = []
             torch.cuda.synchronize()
-        reps = max(1, K // graph_calls) if g is not None else K
-        if g is not None:
-            for _ in range(max(1, W // graph_calls)):
-                g.replay()
+        if graphs:
+            for _ in range(max(1, -(-W // graph_calls))):
+                graphs[0].replay()
         else:
             for k in range(W):
                 step_fn(k)
         self.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        times = []
         ctx = sampler if sampler is not None else _Null()
         with ctx:
-            e0.record()
-            if g is not None:
-                for _ in range(reps):
-                    g.replay()
-            else:
-                for k in range(K):
-                    step_fn(W + k)
-            e1.record()
-            self.barrier()
-        calls = reps * graph_calls if g is not None else K
-        return e0.elapsed_time(e1), calls, ("cuda-graph" if g is not None else "eager")
+            for _ in range(repeats):
+                self.barrier()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                if graphs:
+                    for _ in range(reps):
+                        graphs[0].replay()
+                    if graphs[1] is not None:
+                        graphs[1].replay()
+                else:
+                    for k in range(K):
+                        step_fn(W + k)
+                e1.record()
+                self.barrier()
+                times.append(e0.elapsed_time(e1))
+        return times, K, ("cuda-graph" if graphs else "eager")
 
     def isolated(self, step_fn, K, W):
         for k in range(W):
@@ -364,15 +373,18 @@ def sweep(F, T, R, cfg, idx, Hd, Hh, args, peak):
         out[name] = r
 
     for B in (1, 4, 16, 64):
-        t, n, _ = T.b2b(head_step(F, R, Hd, B, cfg.p), K, W)
+        t, n, _ = T.b2b(head_step(F, R, Hd, B, cfg.p), K, W, repeats=3)
+        t = statistics.median(t)
         U = cfg.p if B == 1 else unique_clusters(F, R[0], Hd, cfg.p, B)
         rec(f"greedy_b{B}", t, n, B, costmodel.head_bytes(cfg.v, cfg.d, cfg.c, cfg.p, B, int(round(U)), 2),
             {"unique_clusters": U})
     for B in (1, 64):
-        t, n, _ = T.b2b(dense_step(F, R, Hd, B), min(K, 32), W)
+        t, n, _ = T.b2b(dense_step(F, R, Hd, B), min(K, 32), W, repeats=3)
+        t = statistics.median(t)
         rec(f"dense_b{B}", t, n, B, costmodel.dense_bytes(cfg.v, cfg.d, B, 2))
     for B in (1, 4, 16, 64):
-        t, n, _ = T.b2b(head_step(F, R, Hd, B, cfg.p, mode="sample"), K, W)
+        t, n, _ = T.b2b(head_step(F, R, Hd, B, cfg.p, mode="sample"), K, W, repeats=3)
+        t = statistics.median(t)
         rec(f"sample_b{B}", t, n, B)
     g = F.head_greedy(R[0], Hd[:64], cfg.p).cpu().numpy()
     d = F.dense_head(R[0], Hd[:64]).cpu().numpy()
@@ -385,7 +397,8 @@ def sweep(F, T, R, cfg, idx, Hd, Hh, args, peak):
     GR = Replicated(F, gidx, int4=True)
     GH = F.device_array(synth.make_queries(gcfg, 1024), "bf16")
     for B in (1, 8, 32):
-        t, n, _ = T.b2b(head_step(F, GR, GH, B, gcfg.p), K, W)
+        t, n, _ = T.b2b(head_step(F, GR, GH, B, gcfg.p), K, W, repeats=3)
+        t = statistics.median(t)
         U = gcfg.p if B == 1 else unique_clusters(F, GR[0], GH, gcfg.p, B)
         rec(f"int4_b{B}", t, n, B,
             costmodel.head_bytes(gcfg.v, gcfg.d, gcfg.c, gcfg.p, B, int(round(U)), 2, int4=True),
@@ -399,6 +412,11 @@ def sweep(F, T, R, cfg, idx, Hd, Hh, args, peak):
     out["int4_agreement_with_bf16_stage1"] = same / GH.shape[0]
     out["int4_agreement_queries"] = int(GH.shape[0])
     del GR, GB
+    out["int4_shift"] = int4_shift_recall(F, gcfg, gidx, GH[:64])
+    torch.cuda.empty_cache()
+    # coarse-fine head on the Llama-shaped vocabulary (v=128256, d=2048; 256 tiles of 8 columns,
+    # 16 codes each; k = 1024 candidates)
+    out["cfhead"] = cf_sweep(F, T, cfg, idx, Hd, K, W, peak)
     torch.cuda.empty_cache()
     # Qwen-shaped Monte Carlo marginal: 16 h x 8 targets, N = 10000 draws each
     qcfg = synth.CONFIGS["qwen"]
@@ -411,10 +429,87 @@ def sweep(F, T, R, cfg, idx, Hd, Hh, args, peak):
     ms = T.isolated(lambda k: F.mc_token_prob(QI, QH, tg, qcfg.p, 1.0, N, synth.MC_SEED, ws=ws), 3, 1)
     mean, se = F.mc_token_prob(QI, QH, tg, qcfg.p, 1.0, N, synth.MC_SEED, ws=ws)
     t = statistics.fmean(ms) * 1e-3
-    out["mc_qwen"] = {"ms_per_call": t * 1e3, "draws_per_s": 16 * N / t,
-                      "keys_per_s": 16 * N * qcfg.c / t, "max_se": float(se.max().item()),
-                      "B": 16, "T": 8, "N": N}
+    keys_per_s = 16 * N * qcfg.c / t
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    clk = ClockSampler(0).max_mhz or 1965
+    # ALU ceiling: every Gumbel key costs two MUFU logarithms (G = -log(-log u)); the SFU returns 16
+    # results per clock per SM, so keys/s <= SMs x 8 x clock
+    mufu_peak = sms * 8 * clk * 1e6
+    out["mc_qwen"] = {"ms_per_call": t * 1e3, "draws_per_s": 16 * N / t, "keys_per_s": keys_per_s,
+                      "max_se": float(se.max().item()), "B": 16, "T": 8, "N": N,
+                      "roofline": {"bound": "alu", "achieved": keys_per_s, "peak": mufu_peak,
+                                   "unit": "Gumbel keys/s", "frac": keys_per_s / mufu_peak,
+                                   "peak_kind": f"derived: {sms} SMs x 16 MUFU results/clock / 2 "
+                                                f"logarithms per key x {clk} MHz"}}
     return out
+
+
+def cf_sweep(F, T, cfg, idx, Hd, K, W, peak):
+    """The coarse-fine head at batches 1, 4, 16 (greedy) and 1 (sampling), timed like the headline,
+    with its algorithmic bytes, and the top-1 agreement with the in-run dense head over 64 queries."""
+    cb, words = synth.cf_index(idx.E, "bf16")
+    base = F.cf_index_from_host(idx.E, cb, words)
+    reps = [base] + [F.CfIndex(base.E, base.codebooks.clone(), base.codes.clone())
+                     for _ in range(REPLICAS - 1)]
+    k = synth.CF_TOPK
+    res = {"w": synth.CF_TILE_W, "K": synth.CF_CODES, "k": k}
+    pool = Hd.shape[0]
+    for B, sample in ((1, False), (4, False), (16, False), (1, True)):
+        outs = [torch.empty(B, dtype=torch.int32, device="cuda") for _ in reps]
+        wss = [torch.zeros(r.workspace_bytes(B, k), dtype=torch.uint8, device="cuda") for r in reps]
+
+        def step(i):
+            r = i % len(reps)
+            off = (i * B) % (pool - B + 1)
+            F.cf_head(reps[r], Hd[off:off + B], k, sample=sample, tau=0.8, seed=synth.SAMPLE_SEED,
+                      step=i, out=outs[r], ws=wss[r])
+        t, n, _ = T.b2b(step, K, W, repeats=3)
+        us = 1e3 * statistics.median(t) / n
+        cand = torch.empty((B, k), dtype=torch.int32, device="cuda")
+        F.cf_head(base, Hd[:B], k, debug=dict(cand=cand))
+        U = int(torch.unique(cand).numel())  # distinct candidate rows of the batch
+        by = costmodel.cf_bytes(cfg.v, cfg.d, synth.CF_TILE_W, synth.CF_CODES, k, B, U)
+        g = by / (us * 1e-6) / 1e9
+        res[("sample" if sample else "greedy") + f"_b{B}"] = {
+            "us_per_call": us, "tokens_per_s": B / (us * 1e-6), "bytes": by, "gbs": g, "frac": g / peak,
+            "unique_candidates": U}
+    FI = F.index_from_host(idx.E, idx.C, idx.C2T, "bf16", cluster_major=False)
+    agree = 0
+    for q0 in range(0, 64, 16):
+        a = F.cf_head(base, Hd[q0:q0 + 16], k).cpu().numpy()
+        b = F.dense_head(FI, Hd[q0:q0 + 16]).cpu().numpy()
+        agree += int(np.sum(a == b))
+    res["agreement_with_dense_top1"] = agree / 64
+    return res
+
+
+def int4_shift_recall(F, cfg, idx, Hd):
+    """Reparameterised INT4 centroids (Softmax Reparameterization pages; FlashHead notes, Module 3):
+    the recall of the GPU's INT4 probe sets against its BF16 ones, |S_int4 ∩ S_bf16| / p averaged over
+    the queries, with the centroids shifted by C' = C - t·mean(C) before quantisation.  Two centroid
+    sets at the Gemma shape: the synthetic index's own (isotropic, mean ~0) and unit centroids that
+    share one direction (weight 1.0), which stand in for real head centroids."""
+    B = Hd.shape[0]
+
+    def sets(I):
+        sel = torch.empty((B, cfg.p), dtype=torch.int32, device="cuda")
+        F.head_greedy(I, Hd, cfg.p, debug=dict(sel=sel))
+        return sel.cpu().numpy()
+
+    res = {"queries": B, "p": cfg.p}
+    for name, Cf in (("synthetic", synth.stored_to_f64(idx.C, "bf16")),
+                     ("common_direction_1.0", synth.anisotropic_centroids(cfg.c, cfg.d, 1.0, 77))):
+        C = synth.store(Cf.astype(np.float32), "bf16")
+        Cb = synth.stored_to_f64(C, "bf16")
+        ref = sets(F.index_from_host(idx.E, C, idx.C2T, "bf16", cluster_major=False))
+        row = {}
+        for t in (0.0, 1.0):
+            q, sc = synth.quantize_int4_g32(synth.shift_centroids(Cb, t))
+            got = sets(F.index_from_host(idx.E, C, idx.C2T, "bf16", q, sc, int4=True, cluster_major=False))
+            row[f"t={t:g}"] = float(np.mean([len(set(got[i]) & set(ref[i])) / cfg.p for i in range(B)]))
+        res[name] = row
+        torch.cuda.empty_cache()
+    return res
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -450,16 +545,29 @@ def oracle_baseline(idx, H, p, budget_s=12.0, budget_1core_s=4.0):
 
 
 def parity_counters(F, I, Hd, out, n, p):
-    """GPU (batch-1 calls, the timed kernel) against the oracle on the oracle's sample: token ids
-    equal overall and where the oracle's set and token margins (4e-3) decide them."""
+    """GPU (batch-1 calls, the timed kernel) against the oracle on the oracle's sample.  A query is
+    decided when the GPU's probe set (from a call with the debug output) equals the oracle's and the
+    oracle's top-1 margin exceeds 4e-3; decided tokens must be equal."""
     tok = np.array([int(F.head_greedy(I, Hd[1 + q:2 + q], p).item()) for q in range(n)])
-    decided = (out["set_margin"] > 4e-3) & (out["tok_margin"] > 4e-3)
+    same_set = np.zeros(n, dtype=bool)
+    sel = torch.empty((1, p), dtype=torch.int32, device="cuda")
+    for q in range(n):
+        F.head_greedy(I, Hd[1 + q:2 + q], p, debug=dict(sel=sel))
+        same_set[q] = np.array_equal(np.sort(sel.cpu().numpy()[0]), np.sort(out["sel"][q]))
+    decided = same_set & (out["tok_margin"] > 4e-3)
     return {"queries": int(n), "tokens_equal": int(np.sum(tok == out["tok"])),
-            "decided": int(np.sum(decided)), "decided_equal": int(np.sum((tok == out["tok"]) & decided)),
-            "margin": 4e-3}
+            "sets_equal": int(np.sum(same_set)), "decided": int(np.sum(decided)),
+            "decided_equal": int(np.sum((tok == out["tok"]) & decided)), "margin": 4e-3,
+            "rule": "decided = GPU probe set equals the oracle's and the oracle's top-1 margin > 4e-3"}
 
 
 METRIC = "head tokens/s at batch 1 (µs/call and HBM GB/s alongside)"
+
+
+def workload_config(cfg, B):
+    """The `config` object of both arms' lines (identical keys and values for the same workload)."""
+    return {"workload": f"llama-3.2-1b-shaped FlashHead greedy: v={cfg.v} d={cfg.d} c={cfg.c} "
+                        f"b={cfg.b} p={cfg.p} batch {B}", "batch": B}
 
 
 def run_reference(args):
@@ -485,9 +593,8 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"llama-3.2-1b-shaped FlashHead greedy: v={cfg.v} d={cfg.d} "
-                                   f"c={cfg.c} b={cfg.b} p={cfg.p} batch {B}",
-                       "impl": "fp64 CPU oracle on the host cores"},
+            "config": workload_config(cfg, B),
+            "setup": {"impl": "fp64 CPU oracle on the host cores"},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(),
                              "kind": "oracle", "sample": f"{args.steps} timed steps of batch {B}"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -540,8 +647,8 @@ def pc_sweep(args):
         Hh = synth.make_queries(cfg, 1024)
         Hd = F.device_array(Hh, "bf16")
         for p in (128, 256, 512):
-            t, n, mode = T.b2b(head_step(F, R, Hd, 1, p), K, W)
-            us = 1e3 * t / n
+            t, n, mode = T.b2b(head_step(F, R, Hd, 1, p), K, W, repeats=3)
+            us = 1e3 * statistics.median(t) / n
             by = costmodel.head_bytes(cfg.v, cfg.d, c, p, 1, p, 2)
             gbs = by / (us * 1e-6) / 1e9
             tok = np.array([int(F.head_greedy(R[0], Hd[q:q + 1], p).item()) for q in range(16)])
@@ -601,6 +708,8 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=16)
     ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="timed repeats of --steps calls each; the line reports their median")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
@@ -652,7 +761,8 @@ def main():
     Hd = F.device_array(Hh, "bf16")
     sampler = ClockSampler(local)
     step = head_step(F, R, Hd, B, cfg.p)
-    t_ms, calls, mode = T.b2b(step, args.steps, args.warmup, sampler=sampler)
+    reps_ms, calls, mode = T.b2b(step, args.steps, args.warmup, sampler=sampler, repeats=args.repeats)
+    t_ms = statistics.median(reps_ms)
     total_ms = max_over_ranks(t_ms, dist)
     tokens = sum_over_ranks(B * calls, dist)
     value = tokens / (total_ms * 1e-3)
@@ -693,19 +803,23 @@ def main():
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": calls,
         "warmup": args.warmup, "ms_per_step": total_ms / calls,
         "us_per_call": us_call, "timing": mode,
+        "repeats_us_per_call": [1e3 * t / calls for t in reps_ms],
         "us_per_call_isolated": summarize(iso),
         "higher_is_better": True, "scaling": "weak",
         "vs_baseline": value / PAGES_TOKENS_PER_S,
         "vs_baseline_note": "vs the pages' A40 head latency TPOT^H 0.40 ms (FlashHead summary, "
                             "Table 3) = 2500 tokens/s; other hardware, context only",
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": f"llama-3.2-1b-shaped FlashHead greedy: v={cfg.v} d={cfg.d} "
-                               f"c={cfg.c} b={cfg.b} p={cfg.p} batch {B}",
-                   "batch": B, "parallelism": f"replicas x{world}" if dist else "single GPU",
-                   "l2": f"inputs larger than L2: calls rotate over {REPLICAS} replicas of C and of "
-                         "the cluster-major E, so no input byte is re-read within 7 calls; the "
-                         "isolated figure flushes L2 with a 256 MiB write before each call",
-                   "inputs": "resident in HBM; a pool of 1024 distinct h, one per call"},
+        "config": workload_config(cfg, B),
+        "setup": {"parallelism": f"replicas x{world}" if dist else "single GPU",
+                  "l2": f"inputs larger than L2: calls rotate over {REPLICAS} replicas of C and of "
+                        "the cluster-major E, so no input byte is re-read within 7 calls; the "
+                        "isolated figure flushes L2 with a 256 MiB write before each call",
+                  "inputs": "resident in HBM; a pool of 1024 distinct h, one per call",
+                  "timed": f"median of {args.repeats} repeats of exactly {calls} back-to-back calls "
+                           "(CUDA-graph replay; consecutive calls overlap only through programmatic "
+                           "dependent launch: a call's centroid stream starts while the previous "
+                           "call's last blocks finish)"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": TRAFFIC.get((B, csrc_hash())),

@@ -249,9 +249,10 @@ def anisotropic_centroids(c: int, d: int, common: float, seed: int) -> np.ndarra
 # that offline index for a synthetic E; the head's own arithmetic (look-up tables, coarse scores,
 # selection, exact logits) is not here.
 
-CF_TILE_W = 8        # columns per tile
+CF_TILE_W = 2        # columns per tile
 CF_CODES = 16        # codebook entries per tile (4-bit codes)
 CF_TOPK = 1024       # candidates that get exact logits
+CF_FIT_TOKENS = 16384  # tokens the codebooks are fitted on
 
 
 def cf_pack_codes(codes: np.ndarray) -> np.ndarray:
@@ -269,40 +270,52 @@ def cf_pack_codes(codes: np.ndarray) -> np.ndarray:
     return np.ascontiguousarray(words.T)
 
 
-def cf_index(E: np.ndarray, dtype: str, w: int = CF_TILE_W, K: int = CF_CODES, iters: int = 3,
-             seed: int = 7000, chunk: int = 8192):
+def cf_index(E: np.ndarray, dtype: str, w: int = CF_TILE_W, K: int = CF_CODES, iters: int = 4,
+             seed: int = 7000, fit_tokens: int = CF_FIT_TOKENS, chunk: int = 8192, device=None):
     """Offline tile-wise k-means of the embedding rows: E's columns are cut into T = d/w tiles; per
-    tile, K centres are fitted to the v sub-rows by `iters` Lloyd iterations (float32, starting from
-    K distinct sub-rows chosen by a seeded permutation; an empty centre keeps its old value).
-    Returns (codebooks float32 [T, K, w], packed codes uint32 [T/8, v]), the codes nearest to the
-    returned centres."""
-    X = stored_to_f64(E, dtype).astype(np.float32)
+    tile, K centres are fitted by `iters` Lloyd iterations (float32) on the sub-rows of `fit_tokens`
+    tokens drawn by a seeded permutation (all tokens when v is smaller), starting from K distinct
+    ones of them; an empty centre keeps its old value.  Every token then gets the code of its nearest
+    centre.  Returns (codebooks float32 [T, K, w], packed codes uint32 [T/8, v]).  The arithmetic runs
+    in torch on `device` (default: the GPU when there is one); the index it returns is an input, read
+    as stored by the library and by the oracle alike."""
+    import torch
+    if device is None:
+        device = "cuda" if torch.cuda.is_available() else "cpu"
+    X = torch.from_numpy(stored_to_f64(E, dtype).astype(np.float32)).to(device)
     v, d = X.shape
     if d % (8 * w):
         raise ValueError("d must be a multiple of 8 tiles")
     T = d // w
     rng = np.random.Generator(np.random.PCG64(seed))
-    Xt = np.ascontiguousarray(X.reshape(v, T, w).transpose(1, 0, 2))          # (T, v, w)
-    cb = np.ascontiguousarray(Xt[:, rng.permutation(v)[:K], :])               # (T, K, w)
+    Xt = X.reshape(v, T, w).permute(1, 0, 2).contiguous()                # (T, v, w)
+    fit = torch.from_numpy(rng.permutation(v)[:min(v, fit_tokens)].astype(np.int64)).to(device)
+    Xf = Xt[:, fit, :].contiguous()
+    cb = Xf[:, :K, :].clone()                                            # (T, K, w)
 
-    def assign(cb):
-        codes = np.empty((T, v), dtype=np.int64)
-        cc = (cb.astype(np.float32) ** 2).sum(-1)[:, None, :]                 # (T, 1, K)
-        for u0 in range(0, v, chunk):
-            dot = np.matmul(Xt[:, u0:u0 + chunk, :], cb.transpose(0, 2, 1))   # (T, n, K)
-            codes[:, u0:u0 + chunk] = np.argmin(cc - 2.0 * dot, axis=2)
+    def assign(Xs, cb):
+        n = Xs.shape[1]
+        codes = torch.empty((T, n), dtype=torch.int64, device=device)
+        for u0 in range(0, n, chunk):
+            x = Xs[:, u0:u0 + chunk, :]
+            dist = torch.zeros((T, x.shape[1], K), device=device)
+            for i in range(w):
+                dist += (x[:, :, None, i] - cb[:, None, :, i]) ** 2
+            codes[:, u0:u0 + chunk] = dist.argmin(-1)
         return codes
 
     for _ in range(iters):
-        codes = assign(cb)
-        for t in range(T):
-            cnt = np.bincount(codes[t], minlength=K)
-            nz = cnt > 0
-            for i in range(w):
-                sums = np.bincount(codes[t], weights=Xt[t, :, i], minlength=K)
-                cb[t, nz, i] = (sums[nz] / cnt[nz]).astype(np.float32)
-    cb32 = np.ascontiguousarray(cb.astype(np.float32))
-    return cb32, cf_pack_codes(assign(cb32).T)
+        codes = assign(Xf, cb)
+        sums = torch.zeros((T, K, w), device=device).scatter_add_(1, codes[:, :, None].expand(-1, -1, w), Xf)
+        cnt = torch.zeros((T, K), device=device).scatter_add_(1, codes, torch.ones(codes.shape, device=device))
+        nz = cnt > 0
+        cb = torch.where(nz[:, :, None], sums / cnt.clamp(min=1)[:, :, None], cb)
+    codes = assign(Xt, cb)
+    return (np.ascontiguousarray(cb.cpu().numpy().astype(np.float32)),
+            cf_pack_codes(codes.T.cpu().numpy()))
+
+
+# ----------------------------------------------------------------------------- queries
 
 
 def make_queries(cfg: HeadConfig, n: int, seed: int | None = None) -> np.ndarray:

@@ -123,8 +123,14 @@ uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(sta
 // dense head takes it from 2 queries on; FlashHead from kTcMinBatchHead, below which the union of
 // the probe sets is sparse enough that the per-query CUDA-core Stage 2 reads fewer bytes.
 constexpr int kTcMinBatchDense = 2;
-constexpr int kTcMinBatchHead = 12;  // measured: at 8 queries the per-query Stage 2 is 1.4x faster
-constexpr int kTcListTilesBatch = 16;  // from here on Stage 2 streams whole tiles instead of gathering
+#ifndef FH_TC_MIN_BATCH_HEAD
+#define FH_TC_MIN_BATCH_HEAD 12
+#endif
+#ifndef FH_TC_LIST_TILES_BATCH
+#define FH_TC_LIST_TILES_BATCH 16
+#endif
+constexpr int kTcMinBatchHead = FH_TC_MIN_BATCH_HEAD;
+constexpr int kTcListTilesBatch = FH_TC_LIST_TILES_BATCH;  // from here on Stage 2 streams whole tiles
 bool tc_eligible(const fh_index* idx, int B, int min_batch) {
   const fh_index_desc& D = idx->desc;
   return B >= min_batch && D.dtype == FH_BF16 && fh::tc_supported(fh::kBF16, D.d, B);
@@ -139,6 +145,26 @@ fh_status check_batch(const fh_index* idx, const void* H, int B) {
 }
 
 fh_stage1_fmt s1fmt(const fh_index* idx) { return (fh_stage1_fmt)idx->desc.s1_fmt; }
+
+// INT4 Stage 1 on the tensor cores from this many queries on (measured at the Gemma-3-1B shape: the
+// CUDA-core kernels take 51 µs for 2 queries and 56 µs for 8, the tensor-core kernel 18.3–18.5 µs
+// for 4 to 8; one query is the same 19 µs either way).
+#ifndef FH_TC_MIN_BATCH_INT4
+#define FH_TC_MIN_BATCH_INT4 2
+#endif
+constexpr int kTcMinBatchInt4 = FH_TC_MIN_BATCH_INT4;
+
+// Stage 1 (scores or Gumbel keys) of s1.B queries: the dequantising tensor-core kernel for INT4
+// centroids at batch, the CUDA-core kernels otherwise.
+cudaError_t launch_stage1_for(const fh_index* idx, const fh::Stage1Params& s1, cudaStream_t st) {
+  const fh_index_desc& D = idx->desc;
+  if (s1fmt(idx) == FH_STAGE1_INT4_G32 && s1.B >= kTcMinBatchInt4 &&
+      fh::tc_int4_supported(D.d, s1.B, D.C_scales))
+    return fh::launch_tc_keys_int4(D.C_q4, D.C_scales, D.c, D.d, s1.H, s1.B, s1.sample, s1.tau,
+                                   s1.seed, s1.step, s1.out, s1.status, s1.tickets_to_clear,
+                                   s1.n_tickets, idx->num_sms, st);
+  return fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st, false);
+}
 
 fh::Stage1Params stage1_params(const fh_index* idx, const void* H, int B, float* out, void* ws) {
   const fh_index_desc& D = idx->desc;
@@ -244,7 +270,7 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     s1.rng_stream = FH_RNG_STAGE1;
     s1.tickets_to_clear = tickets_of(ws);
     s1.n_tickets = B;
-    e = fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st, fused);
+    e = launch_stage1_for(idx, s1, st);
     if (e != cudaSuccess) return cuda_fail(e, "stage-1 launch");
     if (!fused) {
       if ((e = fh::launch_select(keys, sel, B, D.c, p, st)) != cudaSuccess)
@@ -579,9 +605,7 @@ fh_status fh_mc_token_prob_range(const fh_index* idx, const void* H, int B, cons
   }
   // Stage-1 scores
   fh::Stage1Params s1 = stage1_params(idx, H, B, reinterpret_cast<float*>(base + L.s), ws);
-  if ((e = fh::launch_stage1(s1, D.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms, st,
-                             false)) != cudaSuccess)
-    return cuda_fail(e, "MC stage-1 launch");
+  if ((e = launch_stage1_for(idx, s1, st)) != cudaSuccess) return cuda_fail(e, "MC stage-1 launch");
   fh::McParams mp = {};
   mp.s = reinterpret_cast<float*>(base + L.s);
   mp.z = reinterpret_cast<float*>(base + L.z);
@@ -631,8 +655,7 @@ fh_status fh_stage1_scores(const fh_index* idx, const void* H, int B, float* out
     return FH_OK;
   }
   fh::Stage1Params s1 = stage1_params(idx, H, B, out_s, ws);
-  e = fh::launch_stage1(s1, idx->desc.dtype, s1fmt(idx) == FH_STAGE1_INT4_G32, idx->num_sms,
-                        static_cast<cudaStream_t>(stream), false);
+  e = launch_stage1_for(idx, s1, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "stage-1 launch");
   return FH_OK;
 }

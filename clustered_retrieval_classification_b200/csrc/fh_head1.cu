@@ -64,9 +64,6 @@ constexpr int kHistBins = kHead1Bins;
 #define FH_H1_PRE_ROWS 1
 #endif
 constexpr int kHead1PreRows = FH_H1_PRE_ROWS;
-#ifndef FH_H1_TOUCH
-#define FH_H1_TOUCH 0
-#endif
 constexpr int kCap = kHead1BucketCap;
 static_assert(kCap % 32 == 0 && kCap <= kSelCandMax, "bucket words are ranked by warps");
 
@@ -532,14 +529,6 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   const uint8_t* E = static_cast<const uint8_t*>(prm.E);
   const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
   const bool perm = Ep != nullptr;
-#if FH_H1_TOUCH
-  if (perm && !all && tid < nk) {  // one 16-byte L2 prefetch per own certain cluster
-    const uint32_t bn = bin(own_keys[tid]);
-    if (bn > dstar || (bn == dstar && need == m_total))
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], 16;" ::"l"(Ep + (size_t)(lo1 + tid) * (size_t)b * row2)
-                   : "memory");
-  }
-#endif
 
   // This block's Stage-2 rows [r0, r1) of the rank-ordered list (row g: rank g / b, row g % b of
   // that cluster) and the ranks they touch.

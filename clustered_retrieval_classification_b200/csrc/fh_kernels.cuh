@@ -112,12 +112,20 @@ struct TcParams {
   int32_t* tile_list;              // rows/128 scratch: or stream the 128-row tiles some query takes
   int32_t* tile_count;             // 1 scratch word: their number (both lists null: every tile)
   uint32_t* status;
-  int n_tiles;                     // set by the launcher
+  int n_tiles, tile_rows, stages;  // set by the launcher
 };
 bool tc_supported(int elem, int64_t d, int B);
 cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms, cudaStream_t st);
 cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
                                cudaStream_t st);
+bool tc_int4_supported(int64_t d, int B, const void* scales);
+// INT4 Stage-1 keys on the tensor cores: out_keys[q][k] = Σ_j q4[k][j]·scale[k][j/32]·h_q[j] (or the
+// Gumbel key when sample != 0), dequantised to fp16 in shared memory (fh_tc.cu).
+cudaError_t launch_tc_keys_int4(const uint8_t* q4, const uint16_t* scales, int64_t rows, int64_t d,
+                                const void* H, int B, int sample, float tau, uint64_t seed,
+                                uint64_t step, float* out_keys, uint32_t* status,
+                                uint32_t* tickets_to_clear, int n_tickets, int num_sms,
+                                cudaStream_t st);
 
 // The batch-1 persistent head (fh_head1.cu).
 constexpr int kHead1Bins = 1024;       // Stage-1 key histogram

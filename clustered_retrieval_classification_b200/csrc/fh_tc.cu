@@ -10,16 +10,19 @@
 // (row, query) pair by whether the query selected the row's cluster.
 //
 // One persistent CTA per SM, 8 warps with fixed roles:
-//   warp 0      TMA producer: K-blocks of 64 columns of the A tile (128 rows) and of H (N rows),
-//               128-byte swizzled, into a ring of S shared-memory stages;
-//   warp 1      MMA issuer: four 128 x N x 16 tcgen05.mma per stage into one of two TMEM accumulators;
-//   warp 2      allocates and frees the tensor memory (two accumulators, each in one half);
-//   warps 4..7  epilogue: each reads its 32 TMEM lanes (rows) of the finished accumulator, applies the
-//               mask (and the Gumbel term when sampling), and reduces the arg-max of every query.
-// The two accumulators let the epilogue of one tile overlap the MMAs of the next.  Every wait is
-// bounded: on a timeout the CTA records it, drains its own copies and MMAs, frees TMEM and leaves.
+//   warp 0      TMA producer: per stage one K-block (64 columns) of H (Bpad rows) and of each A tile
+//               of the current wave (128 or 64 rows), 128-byte swizzled;
+//   warp 1      MMA issuer: four 128 x R x 16 tcgen05.mma per tile and stage into the wave's half of
+//               tensor memory;
+//   warp 2      allocates and frees the tensor memory (two halves of 256 columns);
+//   warps 4..7  epilogue: thread q reads TMEM lane q (query q) of the finished wave, applies the mask
+//               (and the Gumbel term when sampling), and reduces the query's arg-max.
+// The two halves let the epilogue of one wave overlap the MMAs of the next.  Every wait is bounded:
+// on a timeout the CTA records it, drains its own copies and MMAs, frees TMEM and leaves.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+
+#include <cuda_fp16.h>
 
 #include <mutex>  // std::call_once
 
@@ -32,7 +35,6 @@ namespace {
 
 constexpr int kTcKB = 64;          // K elements per stage: one 128-byte swizzle atom per row
 constexpr int kTcThreads = 256;
-constexpr uint32_t kTcSmemBudget = 200u * 1024u;
 
 // ------------------------------------------------------------------ tcgen05 / TMA primitives
 
@@ -115,44 +117,65 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, volatile
 
 // ------------------------------------------------------------------ the kernel
 //
-// D = H · E_tileᵀ: the MMA's M side is the queries (H padded to 128 rows with zeros), its N side the
-// 128 rows of an E tile, so tensor-memory lane q holds query q and column r row r of the tile.  Each
-// epilogue thread owns one query and reduces its arg-max along its own columns: no cross-lane work.
+// D = H · E_tileᵀ: the MMA's M side is the queries (H padded to 128 rows), its N side the rows of an
+// E tile (128; 64 for Stage-1 keys when that gives every SM a tile), so tensor-memory lane q holds
+// query q and column r row r of the tile.  Each epilogue thread owns one query and reduces its
+// arg-max along its own columns: no cross-lane work.
+//
+// Tiles go in waves of up to kTcWave whose accumulators fill one half of the 512 TMEM columns, so
+// the epilogue of one wave overlaps the MMAs of the next.  A pipeline stage holds one K-block of H
+// and the same K-block of every tile of the wave under one barrier pair, so the K-blocks in flight
+// are bounded by the number of stages alone.  A stage's H block holds only the Bpad = ⌈B/16⌉·16
+// rows the copy writes: the MMA's rows past Bpad read whatever follows in shared memory (inside the
+// allocation, see tc_layout) and only produce accumulator lanes no thread reads.
 
-constexpr int kTcRows = 128;                       // E rows per tile (the MMA's N)
-constexpr int kTcWave = 512 / kTcRows;             // tiles whose accumulators fit tensor memory
+constexpr int kTcRows = 128;                 // E rows per tile in the head modes
+constexpr int kTcWave = 2;                   // tiles per wave (2 x 128 accumulator columns)
+constexpr int kTcMaxStages = 16;
+constexpr uint32_t kTcSmemMax = 226u * 1024u;
 
-template <int S, bool SAMPLE>
-struct TcLayout {
-  static constexpr uint32_t kBlk = 128u * 128u;    // one K-block of H or of an E tile: 128 rows x 128 B
-  static constexpr uint32_t kHOff = S * kBlk;      // S stages of E blocks, then 2 of H blocks
-  static constexpr uint32_t kRowOff = kHOff + 2 * kBlk;            // tile rows: token, mask
-  static constexpr uint32_t kClOff = kRowOff + kTcRows * 12u;        // the wave's cluster ids
-  static constexpr uint32_t kGumOff = kClOff + kTcWave * 16u * 4u;  // sampling: 4 warps x 32 x 32 G
-  static constexpr uint32_t kPairOff = kGumOff + (SAMPLE ? 4u * 32u * 32u * 4u : 0u);  // and pairs
-  static constexpr uint32_t kBars = kPairOff + (SAMPLE ? 4u * 64u * 4u : 0u) + 64u;
-  static constexpr uint32_t kDyn = kBars + 1024u + 1024u;          // + barriers, + alignment slack
+// Dynamic shared memory of the kernel: `stages` stages of (H block, E blocks of the wave), the tile
+// rows (token, mask) and the wave's cluster ids, the sampling scratch, the barriers.
+struct TcLay {
+  uint32_t h_bytes, e_bytes, stage_bytes;
+  uint32_t row_off, cl_off, gum_off, pair_off, bar_off, dyn;
 };
+__host__ __device__ inline TcLay tc_layout(int B, int tile_rows, int wave, bool sample, int stages) {
+  TcLay L;
+  L.h_bytes = (uint32_t)((B + 15) / 16 * 16) * 128u;  // multiple of 2048: keeps E blocks 1024-aligned
+  L.e_bytes = (uint32_t)tile_rows * 128u;
+  L.stage_bytes = L.h_bytes + (uint32_t)wave * L.e_bytes;
+  L.row_off = (uint32_t)stages * L.stage_bytes;
+  L.cl_off = L.row_off + (uint32_t)kTcRows * 12u;
+  L.gum_off = L.cl_off + (uint32_t)kTcWave * 16u * 4u;
+  L.pair_off = L.gum_off + (sample ? 4u * 32u * 32u * 4u : 0u);
+  L.bar_off = L.pair_off + (sample ? 4u * 64u * 4u : 0u);
+  const uint32_t end = L.bar_off + (uint32_t)(2 * kTcMaxStages + 8) * 8u;
+  // the last stage's H operand is read as 128 rows of 128 B
+  const uint32_t h_end = (uint32_t)(stages > 0 ? stages - 1 : 0) * L.stage_bytes + 128u * 128u;
+  L.dyn = (end > h_end ? end : h_end) + 1024u;  // + alignment slack
+  return L;
+}
 
 // KEYS: write the products (Stage-1 keys) instead of reducing an arg-max; SAMPLE: add the Gumbel
 // term.  Separate instantiations keep each epilogue's code out of the other modes' instruction stream.
-template <int S, bool KEYS, bool SAMPLE>
+template <bool KEYS, bool SAMPLE>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_tc_head(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmH,
               const TcParams a) {
-  using Lay = TcLayout<S, SAMPLE>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
-  uint32_t* tok_s = reinterpret_cast<uint32_t*>(smem + Lay::kRowOff);                     // 128
-  unsigned long long* msk_s = reinterpret_cast<unsigned long long*>(smem + Lay::kRowOff + 512u);  // 128
-  int32_t* wave_cl = reinterpret_cast<int32_t*>(smem + Lay::kClOff);  // kTcWave x gpt
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay::kBars);
-  uint64_t* empty = full + S;
-  uint64_t* hfull = empty + S;     // H block landed
-  uint64_t* hempty = hfull + 2;    // H block no longer read
-  uint64_t* tfull = hempty + 2;    // a wave's accumulators are final (MMA -> epilogue)
-  uint64_t* tempty = tfull + 1;    // and have been read (epilogue -> MMA)
-  uint64_t* drain = tempty + 1;    // last commit of the MMA issuer
+  constexpr int WT = KEYS ? 1 : kTcWave;
+  const int R = a.tile_rows, S = a.stages;
+  const TcLay Lay = tc_layout(a.B, R, WT, SAMPLE, S);
+  uint32_t* tok_s = reinterpret_cast<uint32_t*>(smem + Lay.row_off);                     // 128
+  unsigned long long* msk_s = reinterpret_cast<unsigned long long*>(smem + Lay.row_off + 512u);  // 128
+  int32_t* wave_cl = reinterpret_cast<int32_t*>(smem + Lay.cl_off);  // kTcWave x gpt
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay.bar_off);
+  uint64_t* empty = full + kTcMaxStages;
+  uint64_t* tfull = empty + kTcMaxStages;  // [2] a wave's accumulators are final (MMA -> epilogue)
+  uint64_t* tempty = tfull + 2;            // [2] and have been read (epilogue -> MMA)
+  uint64_t* drain = tempty + 2;            // last commit of the MMA issuer
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s;
   __shared__ bool last_s;
@@ -160,15 +183,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;
   const int KB = (int)((a.d + kTcKB - 1) / kTcKB);
-  // This CTA's tiles: bid, bid + G, ..., processed in waves of kTcWave tiles whose accumulators all
-  // live in tensor memory at once, so each H block is read once per wave.  In gather mode tile t is
-  // the gpt clusters gpt*t .. gpt*t + gpt - 1 of the selected-cluster list (b rows each).
+  // This CTA's tiles: bid, bid + G, ...  In gather mode tile t is the gpt clusters gpt*t .. gpt*t +
+  // gpt - 1 of the selected-cluster list (b rows each).
   const int gpt = a.cl_list ? (int)(kTcRows / a.b) : 0;
   const int n_cl = a.cl_list ? __ldg(a.cl_count) : 0;
   // listed mode: the contiguous tiles some query takes, tile_list[0 .. *tile_count)
   const int n_list = a.cl_list ? (n_cl + gpt - 1) / gpt : (a.tile_list ? __ldg(a.tile_count) : a.n_tiles);
   const int my_tiles = n_list > (int)blockIdx.x ? (n_list - (int)blockIdx.x + G - 1) / G : 0;
-  const int n_waves = (my_tiles + kTcWave - 1) / kTcWave;
+  const int n_waves = (my_tiles + WT - 1) / WT;
   auto tile_at = [&](int j) {
     const int e = (int)blockIdx.x + j * G;
     return a.tile_list ? __ldg(a.tile_list + e) : e;
@@ -180,37 +202,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&hfull[i], 1);
-      mbar_init(&hempty[i], 1);
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], 4);
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, 4);
     mbar_init(drain, 1);
     abort_s = 0;
   }
-  if (warp == 2) {  // all 512 columns: kTcWave accumulators of 128 lanes (queries) x 128 rows, FP32
+  if (warp == 2) {  // all 512 columns: two halves of kTcWave accumulators (128 lanes x R rows, FP32)
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  ::"r"(smem_addr(&tmem_base_s)), "r"(512u) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
-  {  // H buffers: TMA writes only the first Bpad rows; the rest must read as zeros in the MMA
-    uint4* hz = reinterpret_cast<uint4*>(smem + Lay::kHOff);
-    for (int i = tid; i < (int)(2 * Lay::kBlk / 16); i += kTcThreads) hz[i] = make_uint4(0u, 0u, 0u, 0u);
-    fence_proxy_async_smem();
   }
   fence_mbar_init();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
-  const uint32_t h_bytes = (uint32_t)((a.B + 15) / 16 * 16) * 128u;  // the H box: Bpad rows
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    int it = 0, hit = 0;
+    int it = 0;
     bool ok = true;
     for (int w = 0; w < n_waves && ok; ++w) {
-      const int j0 = w * kTcWave, nt = min(kTcWave, my_tiles - j0);
+      const int j0 = w * WT, nt = min(WT, my_tiles - j0);
       if (gpt) {  // the wave's cluster ids, read once by the whole warp (no load in the issue loop)
         for (int i = lane; i < nt * gpt; i += 32) {
           const int slot = tile_at(j0 + i / gpt) * gpt + i % gpt;
@@ -219,31 +233,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
       }
       if (lane == 0) {
-        for (int kb = 0; kb < KB && ok; ++kb, ++hit) {
-          const int hs = hit & 1;
-          if (!tc_wait(&hempty[hs], (uint32_t)(((hit >> 1) & 1) ^ 1), &abort_s, a.status)) {
+        int tl[kTcWave], nc[kTcWave];
+        uint32_t bytes = Lay.h_bytes;  // H rows past B (up to Bpad) read as zeros
+        for (int j = 0; j < nt; ++j) {
+          tl[j] = tile_at(j0 + j);
+          nc[j] = gpt ? min(gpt, n_cl - tl[j] * gpt) : 0;
+          bytes += gpt ? (uint32_t)nc[j] * (uint32_t)a.b * 128u : Lay.e_bytes;
+        }
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          if (!tc_wait(&empty[s], (uint32_t)(((it / S) & 1) ^ 1), &abort_s, a.status)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&hfull[hs], h_bytes);  // rows past B (up to Bpad) read as zeros
-          tma_load_2d(smem + Lay::kHOff + hs * Lay::kBlk, &tmH, kb * kTcKB, 0, &hfull[hs]);
-          for (int j = 0; j < nt; ++j, ++it) {
-            const int s = it % S;
-            if (!tc_wait(&empty[s], (uint32_t)(((it / S) & 1) ^ 1), &abort_s, a.status)) {
-              ok = false;
-              break;
-            }
-            uint8_t* dst = smem + (size_t)s * Lay::kBlk;
-            const int t = tile_at(j0 + j);
+          uint8_t* stg = smem + (size_t)s * Lay.stage_bytes;
+          mbar_arrive_expect_tx(&full[s], bytes);
+          tma_load_2d(stg, &tmH, kb * kTcKB, 0, &full[s]);
+          for (int j = 0; j < nt; ++j) {
+            uint8_t* dst = stg + Lay.h_bytes + (size_t)j * Lay.e_bytes;
             if (gpt) {  // one box of b rows per listed cluster; the rows of absent ones stay unread
-              const int nc = min(gpt, n_cl - t * gpt);
-              mbar_arrive_expect_tx(&full[s], (uint32_t)nc * (uint32_t)a.b * 128u);
-              for (int i = 0; i < nc; ++i)
+              for (int i = 0; i < nc[j]; ++i)
                 tma_load_2d(dst + (size_t)i * a.b * 128u, &tmE, kb * kTcKB, wave_cl[j * gpt + i] * (int)a.b,
                             &full[s]);
             } else {
-              mbar_arrive_expect_tx(&full[s], Lay::kBlk);
-              tma_load_2d(dst, &tmE, kb * kTcKB, t * kTcRows, &full[s]);
+              tma_load_2d(dst, &tmE, kb * kTcKB, tl[j] * R, &full[s]);
             }
           }
         }
@@ -256,46 +269,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // leave no copy in flight: the last loads have landed (at once when all went well)
       for (int j = max(0, it - S); j < it; ++j)
         mbar_wait(&full[j % S], (uint32_t)((j / S) & 1), nullptr, 50000000ull);
-      for (int j = max(0, hit - 2); j < hit; ++j)
-        mbar_wait(&hfull[j & 1], (uint32_t)((j >> 1) & 1), nullptr, 50000000ull);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16<kTcRows>(128);  // M = 128 queries, N = 128 rows
+      // kind::f16, FP32 accumulator, BF16 A and B, both K-major, M = 128 queries, N = R rows
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(R >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
       const uint32_t sbase = smem_addr(smem);
-      int it = 0, hit = 0;
+      int it = 0;
       bool ok = true, issued = false;
       for (int w = 0; w < n_waves && ok; ++w) {
-        const int nt = min(kTcWave, my_tiles - w * kTcWave);
-        if (!tc_wait(tempty, (uint32_t)((w & 1) ^ 1), &abort_s, a.status)) break;
+        const int nt = min(WT, my_tiles - w * WT), acc = w & 1;
+        if (!tc_wait(&tempty[acc], (uint32_t)(((w >> 1) & 1) ^ 1), &abort_s, a.status)) break;
         tc_fence_after();
-        for (int kb = 0; kb < KB && ok; ++kb, ++hit) {
-          const int hs = hit & 1;
-          if (!tc_wait(&hfull[hs], (uint32_t)((hit >> 1) & 1), &abort_s, a.status)) {
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % S;
+          if (!tc_wait(&full[s], (uint32_t)((it / S) & 1), &abort_s, a.status)) {
             ok = false;
             break;
           }
-          const uint32_t ha = sbase + Lay::kHOff + (uint32_t)hs * Lay::kBlk;
-          for (int j = 0; j < nt; ++j, ++it) {
-            const int s = it % S;
-            if (!tc_wait(&full[s], (uint32_t)((it / S) & 1), &abort_s, a.status)) {
-              ok = false;
-              break;
-            }
-            // (TMA writes and MMA reads are both async-proxy operations ordered by the barrier)
-            const uint32_t ea = sbase + (uint32_t)s * Lay::kBlk;
-            const uint32_t d_tmem = tmem + (uint32_t)(j * kTcRows);
+          tc_fence_after();
+          // (TMA writes and MMA reads are both async-proxy operations ordered by the barrier)
+          const uint32_t ha = sbase + (uint32_t)s * Lay.stage_bytes;
+          for (int j = 0; j < nt; ++j) {
+            const uint32_t ea = ha + Lay.h_bytes + (uint32_t)j * Lay.e_bytes;
+            const uint32_t d_tmem = tmem + (uint32_t)(acc * 256 + j * R);
 #pragma unroll
             for (int k = 0; k < kTcKB / 16; ++k)  // 16 BF16 = 32 bytes along K per instruction
               mma_bf16(d_tmem, sw128_desc(ha + 32u * k), sw128_desc(ea + 32u * k), idesc,
                        (uint32_t)((kb | k) != 0));
-            mma_commit(&empty[s]);  // the E stage is free once these MMAs have read it
-            issued = true;
           }
-          if (ok) mma_commit(&hempty[hs]);
+          mma_commit(&empty[s]);  // the stage is free once these MMAs have read it
+          issued = true;
         }
-        if (ok) mma_commit(tfull);
+        if (ok) mma_commit(&tfull[acc]);
       }
       if (issued) {  // every MMA has completed before the tensor memory is freed
         mma_commit(drain);
@@ -310,12 +317,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t bk = 0u, bt = 0xFFFFFFFFu;   // best key image and its token
     auto group_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
     for (int w = 0; w < n_waves; ++w) {
-      const int j0 = w * kTcWave, nt = min(kTcWave, my_tiles - j0);
-      if (!tc_wait(tfull, (uint32_t)(w & 1), &abort_s, a.status)) break;
+      const int j0 = w * WT, nt = min(WT, my_tiles - j0), acc = w & 1;
+      if (!tc_wait(&tfull[acc], (uint32_t)((w >> 1) & 1), &abort_s, a.status)) break;
       tc_fence_after();
       for (int j = 0; j < nt; ++j) {
         const int t = tile_at(j0 + j);
-        {  // the tile's rows: token and query mask (0: no query takes the row, or no row)
+        if constexpr (!KEYS) {  // the tile's rows: token and query mask (0: no query takes the row, or no row)
           const int r = et;
           int64_t row, cl;
           bool valid;
@@ -331,23 +338,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           tok_s[r] = valid ? (a.row_tok ? (uint32_t)__ldg(a.row_tok + row) : (uint32_t)row) : 0u;
           msk_s[r] = valid ? (a.qmask ? __ldg(a.qmask + cl) : ~0ull) : 0ull;
+          group_sync();
         }
-        group_sync();
-        const uint32_t tbase = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(j * kTcRows);
-        const int64_t row0 = (int64_t)t * kTcRows;  // contiguous mode: first row of the tile
-        for (int c0 = 0; c0 < kTcRows; c0 += 32) {
+        const uint32_t tbase = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(acc * 256 + j * R);
+        const int64_t row0 = (int64_t)t * R;  // contiguous mode: first row of the tile
+        for (int c0 = 0; c0 < R; c0 += 32) {
           uint32_t v[32];
           tmem_ld16(tbase + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(v));
           tmem_ld16(tbase + (uint32_t)c0 + 16u, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
           tmem_ld_wait();
           if constexpr (KEYS) {  // Stage-1 keys (contiguous rows): s[q][row] or s/τ + G(q, stream 0, row)
+            if (q < a.B) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const int64_t row = row0 + c0 + i;
-              if (q < a.B && row < a.rows) {
-                const float z = __uint_as_float(v[i]);
-                a.out_keys[(int64_t)q * a.rows + row] =
-                    SAMPLE ? z / a.tau + gumbel_from_u32(philox_word(a.seed, a.step, (uint32_t)q, 0u, (uint32_t)row)) : z;
+              for (int i = 0; i < 32; ++i) {
+                const int64_t row = row0 + c0 + i;
+                if (row < a.rows) {
+                  const float z = __uint_as_float(v[i]);
+                  a.out_keys[(int64_t)q * a.rows + row] =
+                      SAMPLE ? z / a.tau + gumbel_from_u32(philox_word(a.seed, a.step, (uint32_t)q, 0u, (uint32_t)row)) : z;
+                }
               }
             }
             continue;
@@ -361,8 +370,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // spread evenly over the lanes: a row is taken by few of the warp's 32 queries, so one
             // evaluation per row and lane would leave most lanes idle.  Lane i lists row i's takers
             // (a ballot), a scan gives each row its first pair, and pair k goes to lane k % 32.
-            uint32_t* bal_s = reinterpret_cast<uint32_t*>(smem + Lay::kPairOff) + (warp & 3) * 64;
-            gum = reinterpret_cast<float*>(smem + Lay::kGumOff) + (warp & 3) * 1024;
+            uint32_t* bal_s = reinterpret_cast<uint32_t*>(smem + Lay.pair_off) + (warp & 3) * 64;
+            gum = reinterpret_cast<float*>(smem + Lay.gum_off) + (warp & 3) * 1024;
             uint32_t my_bal = 0u;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
@@ -408,11 +417,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           if constexpr (SAMPLE) __syncwarp();  // the warp's G buffer is rewritten for the next chunk
         }
-        group_sync();  // the tile rows are rewritten for the next tile
+        if constexpr (!KEYS) group_sync();  // the tile rows are rewritten for the next tile
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tempty);  // the next wave may overwrite the accumulators
+      if (lane == 0) mbar_arrive(&tempty[acc]);  // the MMAs may overwrite these accumulators
     }
     if (!KEYS && q < a.B && bk) atomicMax(a.best + q, ((unsigned long long)bk << 32) | (unsigned long long)(~bt));
   }
@@ -530,13 +539,18 @@ bool make_map(CUtensorMap* m, const void* base, int64_t d, int64_t rows, uint32_
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, const TcParams& p, int num_sms,
+cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, TcParams p, int num_sms,
                           cudaStream_t st) {
-  constexpr int S = (int)((kTcSmemBudget - 2u * 16384u - 4096u) / 16384u);
   const bool keys = p.out_keys != nullptr, sample = p.sample != 0;
-  auto kern = keys ? (sample ? k_tc_head<S, true, true> : k_tc_head<S, true, false>)
-                   : (sample ? k_tc_head<S, false, true> : k_tc_head<S, false, false>);
-  const uint32_t dyn = sample ? TcLayout<S, true>::kDyn : TcLayout<S, false>::kDyn;
+  const int wave = keys ? 1 : kTcWave;
+  int S = kTcMaxStages;
+  for (; S >= 2; --S)
+    if (tc_layout(p.B, p.tile_rows, wave, sample, S).dyn <= kTcSmemMax) break;
+  if (S < 2) return cudaErrorInvalidValue;
+  p.stages = S;
+  auto kern = keys ? (sample ? k_tc_head<true, true> : k_tc_head<true, false>)
+                   : (sample ? k_tc_head<false, true> : k_tc_head<false, false>);
+  const uint32_t dyn = tc_layout(p.B, p.tile_rows, wave, sample, S).dyn;
   cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(kern), dyn);
   if (e != cudaSuccess) return e;
   // every SM when the tiles are listed on the device; otherwise no more CTAs than tiles
@@ -545,7 +559,295 @@ cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, const Tc
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ INT4 Stage-1 keys
+//
+// Stage-1 keys from INT4 centroids (FlashHead notes, Module 3) for a batch of queries: the MMA's B
+// operand (128 centroid rows per tile) is dequantised in shared memory — q·scale for the 4-bit q and
+// the row's BF16 group scale, which is exact in fp16 (at most 11 significant bits) — and the queries
+// are converted from BF16 to fp16 in place (exact for |h_j| in [2^-17, 65504]); kind::f16 MMAs with fp16
+// operands and FP32 accumulators then give the keys.  One tile of 128 centroid rows per CTA pass.
+// Warp roles: warp 0 loads (TMA: the query block of each K-block, the 32-byte nibble rows of the
+// tile; one bulk copy for the tile's scales), warp 1 issues the MMAs, warp 2 owns 128 TMEM columns,
+// warps 4..7 dequantise (thread t: row t of the tile) and finally read the accumulators (thread t:
+// query t) and write the keys.
+
+constexpr int kI4Stages = 4;
+constexpr uint32_t kI4Blk = 128u * 128u;   // one K-block of fp16 operand: 128 rows x 128 B
+constexpr uint32_t kI4Nib = 128u * 32u;    // one K-block of nibbles: 128 rows x 32 B
+
+struct I4Layout {
+  static constexpr uint32_t kH = 0;                                  // S query blocks (SW128)
+  static constexpr uint32_t kOp = kH + kI4Stages * kI4Blk;           // S dequantised blocks (SW128)
+  static constexpr uint32_t kNib = kOp + kI4Stages * kI4Blk;         // S nibble blocks
+  static constexpr uint32_t kSc = kNib + kI4Stages * kI4Nib;         // the tile's scales
+};
+
+struct TcInt4Params {
+  int64_t rows, d;            // c centroid rows of d columns
+  int B;
+  int sample;
+  float tau;
+  uint64_t seed, step;
+  const uint16_t* scales;     // rows x d/32 BF16
+  float* out_keys;            // B x rows
+  uint32_t* status;
+  uint32_t* tickets_to_clear;  // reset to 0 by block 0 for the kernels that follow
+  int n_tickets;
+  int n_tiles;
+};
+
+__device__ __forceinline__ uint16_t f32_to_f16_bits(float x) {
+  return __half_as_ushort(__float2half_rn(x));
+}
+
+// BF16 -> fp16 for the 8 values of a 16-byte chunk (rounds to nearest when not exact).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = (uint32_t)f32_to_f16_bits(bf16_lo(w[i])) | ((uint32_t)f32_to_f16_bits(bf16_hi(w[i])) << 16);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <bool SAMPLE>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_tc_keys_int4(const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmQ,
+                   const TcInt4Params a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
+  __shared__ uint64_t full_in[kI4Stages], dq_full[kI4Stages], op_empty[kI4Stages];
+  __shared__ uint64_t sc_full, tfull, tempty, drain;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int KB = (int)((a.d + kTcKB - 1) / kTcKB);
+  const int G32 = (int)(a.d / 32);
+  const uint32_t sc_row = (uint32_t)G32 * 2u;  // scale bytes per row
+  const uint32_t h_bytes = (uint32_t)((a.B + 15) / 16 * 16) * 128u;
+  if (tid == 0) {
+    for (int s = 0; s < kI4Stages; ++s) {
+      mbar_init(&full_in[s], 1);
+      mbar_init(&dq_full[s], 4);
+      mbar_init(&op_empty[s], 1);
+    }
+    mbar_init(&sc_full, 1);
+    mbar_init(&tfull, 1);
+    mbar_init(&tempty, 4);
+    mbar_init(&drain, 1);
+    abort_s = 0;
+  }
+  if (blockIdx.x == 0 && tid < a.n_tickets) a.tickets_to_clear[tid] = 0u;
+  if (warp == 2) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_addr(&tmem_base_s)), "r"(128u) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  {  // query blocks: TMA writes only the first Bpad rows; the rest must read as zeros in the MMA
+    uint4* hz = reinterpret_cast<uint4*>(smem + I4Layout::kH);
+    for (int i = tid; i < (int)(kI4Stages * kI4Blk / 16); i += kTcThreads) hz[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();
+  }
+  fence_mbar_init();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  const int my_tiles = a.n_tiles > (int)blockIdx.x ? (a.n_tiles - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- loads
+    if (lane == 0) {
+      int it = 0, sc_n = 0;
+      bool ok = true;
+      for (int j = 0; j < my_tiles && ok; ++j) {
+        const int t = (int)blockIdx.x + j * (int)gridDim.x;
+        const int64_t r0 = (int64_t)t * 128;
+        const int nrows = (int)min((int64_t)128, a.rows - r0);
+        // the tile's scales: one bulk copy of whole 16-byte chunks (the ragged tail is read directly
+        // by the dequantising threads), once the previous tile's dequantisation is over
+        if (j > 0 && !tc_wait(&tempty, (uint32_t)((j - 1) & 1), &abort_s, a.status)) break;
+        const uint32_t sc_bytes = (uint32_t)nrows * sc_row;
+        const uint32_t sc16 = sc_bytes & ~15u;
+        mbar_arrive_expect_tx(&sc_full, sc16);
+        if (sc16) bulk_g2s(smem + I4Layout::kSc, reinterpret_cast<const uint8_t*>(a.scales) + (size_t)r0 * sc_row, sc16, &sc_full);
+        ++sc_n;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kI4Stages;
+          if (!tc_wait(&op_empty[s], (uint32_t)(((it / kI4Stages) & 1) ^ 1), &abort_s, a.status)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_in[s], h_bytes + kI4Nib);
+          tma_load_2d(smem + I4Layout::kH + s * kI4Blk, &tmH, kb * kTcKB, 0, &full_in[s]);
+          tma_load_2d(smem + I4Layout::kNib + s * kI4Nib, &tmQ, kb * 32, (int)r0, &full_in[s]);
+        }
+      }
+      // leave no copy in flight
+      for (int j = max(0, it - kI4Stages); j < it; ++j)
+        mbar_wait(&full_in[j % kI4Stages], (uint32_t)((j / kI4Stages) & 1), nullptr, 50000000ull);
+      if (sc_n) mbar_wait(&sc_full, (uint32_t)((sc_n - 1) & 1), nullptr, 50000000ull);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(128 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+      const uint32_t sbase = smem_addr(smem);
+      int it = 0;
+      bool ok = true, issued = false;
+      for (int j = 0; j < my_tiles && ok; ++j) {
+        if (j > 0 && !tc_wait(&tempty, (uint32_t)((j - 1) & 1), &abort_s, a.status)) break;
+        tc_fence_after();
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = it % kI4Stages;
+          if (!tc_wait(&dq_full[s], (uint32_t)((it / kI4Stages) & 1), &abort_s, a.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ha = sbase + I4Layout::kH + (uint32_t)s * kI4Blk;
+          const uint32_t ba = sbase + I4Layout::kOp + (uint32_t)s * kI4Blk;
+#pragma unroll
+          for (int k = 0; k < kTcKB / 16; ++k)
+            mma_bf16(tmem, sw128_desc(ha + 32u * k), sw128_desc(ba + 32u * k), idesc, (uint32_t)((kb | k) != 0));
+          mma_commit(&op_empty[s]);
+          issued = true;
+        }
+        if (ok) mma_commit(&tfull);
+      }
+      if (issued) {
+        mma_commit(&drain);
+        mbar_wait(&drain, 0u, nullptr, 50000000ull);
+      }
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- dequantise, then the keys
+    const int et = tid - 128;  // this thread's tile row (dequantisation) and query (epilogue)
+    int it = 0;
+    for (int j = 0; j < my_tiles; ++j) {
+      const int t = (int)blockIdx.x + j * (int)gridDim.x;
+      const int64_t r0 = (int64_t)t * 128;
+      const int nrows = (int)min((int64_t)128, a.rows - r0);
+      if (!tc_wait(&sc_full, (uint32_t)(j & 1), &abort_s, a.status)) break;
+      const uint16_t* sc_s = reinterpret_cast<const uint16_t*>(smem + I4Layout::kSc);
+      // the row's scales (the bytes past the bulk copy's last whole chunk straight from memory)
+      const uint32_t sc16 = ((uint32_t)nrows * sc_row) & ~15u;
+      auto scale_at = [&](int g) {
+        const uint32_t off = (uint32_t)et * sc_row + 2u * (uint32_t)g;
+        uint16_t bits = 0;
+        if (et < nrows) bits = off < sc16 ? sc_s[off / 2] : __ldg(a.scales + (size_t)(r0 + et) * G32 + g);
+        return __uint_as_float((uint32_t)bits << 16);
+      };
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const int s = it % kI4Stages;
+        if (!tc_wait(&full_in[s], (uint32_t)((it / kI4Stages) & 1), &abort_s, a.status)) {
+          ok = false;
+          break;
+        }
+        // the query block: BF16 -> fp16 in place (threads split the Bpad x 8 chunks)
+        uint8_t* hb = smem + I4Layout::kH + s * kI4Blk;
+        for (int ch = et; ch < (int)(h_bytes / 16); ch += 128) {
+          uint4* p = reinterpret_cast<uint4*>(hb + 16 * ch);
+          *p = bf16x8_to_f16x8(*p);
+        }
+        // row et of the centroid tile: 64 nibbles -> 64 fp16 values, written 128-byte swizzled
+        const uint8_t* nib = smem + I4Layout::kNib + s * kI4Nib + et * 32;
+        uint8_t* op = smem + I4Layout::kOp + s * kI4Blk + (et >> 3) * 1024 + (et & 7) * 128;
+        const int g0 = 2 * kb;
+        const float sc0 = g0 < G32 ? scale_at(g0) : 0.0f, sc1 = g0 + 1 < G32 ? scale_at(g0 + 1) : 0.0f;
+        const uint4 w0 = *reinterpret_cast<const uint4*>(nib), w1 = *reinterpret_cast<const uint4*>(nib + 16);
+        const uint32_t words[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const __half2 s2a = __half2half2(__float2half_rn(sc0)), s2b = __half2half2(__float2half_rn(sc1));
+        const __half2 bias = __half2half2(__ushort_as_half((uint16_t)0x6408u));  // 1032 = 1024 + 8
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {  // chunk c: columns 8c .. 8c+7 (one 32-bit word of nibbles)
+          // nibble n of u is q_n + 8 (two's complement -> offset binary); fp16 0x6400 | b is 1024 + b,
+          // so subtracting 1032 gives q exactly, and q times the fp16 scale is exact (<= 11 bits)
+          const uint32_t u = words[c] ^ 0x88888888u, u4 = u >> 4;
+          uint32_t out[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            // low half: the low nibble of byte e (column 2e); high half: its high nibble (column 2e+1)
+            const uint32_t t = __byte_perm(u, u4, (uint32_t)(e | (e << 4) | ((4 + e) << 8) | ((4 + e) << 12)));
+            const uint32_t x = (t & 0x000F000Fu) | 0x64006400u;
+            const __half2 q = __hsub2(*reinterpret_cast<const __half2*>(&x), bias);
+            const __half2 r = __hmul2(q, c < 4 ? s2a : s2b);
+            out[e] = *reinterpret_cast<const uint32_t*>(&r);
+          }
+          *reinterpret_cast<uint4*>(op + ((c ^ (et & 7)) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+        }
+        fence_proxy_async_smem();  // generic writes -> the tensor core's async reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dq_full[s]);
+      }
+      if (!ok) break;
+      // the accumulators of this tile: lane q of TMEM = query q
+      if (!tc_wait(&tfull, (uint32_t)(j & 1), &abort_s, a.status)) break;
+      tc_fence_after();
+      const int q = et;
+      const uint32_t tbase = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld16(tbase + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(v));
+        tmem_ld16(tbase + (uint32_t)c0 + 16u, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
+        tmem_ld_wait();
+        if (q < a.B) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int64_t row = r0 + c0 + i;
+            if (row < a.rows) {
+              const float z = __uint_as_float(v[i]);
+              a.out_keys[(int64_t)q * a.rows + row] =
+                  SAMPLE ? z / a.tau + gumbel_from_u32(philox_word(a.seed, a.step, (uint32_t)q, 0u, (uint32_t)row)) : z;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty);  // the next tile may reuse the accumulators and scales
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(128u) : "memory");
+  }
+}
+
+// 2-D maps of the INT4 Stage 1: the queries as fp16 (same bits as the BF16 map; the data is converted
+// in shared memory) and the nibble rows (uint8, 32-byte boxes of 128 rows, no swizzle).
+bool make_map_h16(CUtensorMap* m, const void* base, int64_t d, int64_t rows, uint32_t box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2u};
+  cuuint32_t box[2] = {(cuuint32_t)kTcKB, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_map_nib(CUtensorMap* m, const void* base, int64_t d, int64_t rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)(d / 2), (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(d / 2)};
+  cuuint32_t box[2] = {32u, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
+
+bool tc_int4_supported(int64_t d, int B, const void* scales) {
+  return B >= 1 && B <= 64 && d % 32 == 0 && (reinterpret_cast<uintptr_t>(scales) & 15u) == 0 &&
+         I4Layout::kSc + (size_t)128 * (d / 32) * 2 + 1024 <= 227 * 1024;
+}
 
 bool tc_supported(int elem, int64_t d, int B) {
   return elem == kBF16 && d % 8 == 0 && B >= 1 && B <= 64 && encode_fn() != nullptr;
@@ -554,8 +856,10 @@ bool tc_supported(int elem, int64_t d, int B) {
 cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms, cudaStream_t st) {
   if (p.B < 1 || p.B > 64 || p.rows < 1 || (p.qmask && p.b < 1)) return cudaErrorInvalidValue;
   if (p.out_keys && (p.qmask || p.cl_list)) return cudaErrorInvalidValue;
-  p.n_tiles = (int)((p.rows + kTcRows - 1) / kTcRows);
-  uint32_t box = kTcRows;
+  // Stage-1 keys of few rows take 64-row tiles when that gives every SM at most one
+  p.tile_rows = (p.out_keys && (p.rows + 63) / 64 <= num_sms) ? 64 : kTcRows;
+  p.n_tiles = (int)((p.rows + p.tile_rows - 1) / p.tile_rows);
+  uint32_t box = (uint32_t)p.tile_rows;
   if (p.tile_list) {  // the selected tiles, listed on the device (the kernel reads their count)
     if (!p.qmask || p.cl_list) return cudaErrorInvalidValue;
     k_selected_tiles<<<1, 1024, 0, st>>>(p.qmask, p.rows, p.b, p.n_tiles, p.tile_list, p.tile_count);
@@ -573,6 +877,40 @@ cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms
   if (!make_map(&mE, A, p.d, p.rows, box) || !make_map(&mH, H, p.d, p.B, (uint32_t)((p.B + 15) / 16 * 16)))
     return cudaErrorInvalidValue;
   return launch_kernel(mE, mH, p, num_sms, st);
+}
+
+
+cudaError_t launch_tc_keys_int4(const uint8_t* q4, const uint16_t* scales, int64_t rows, int64_t d,
+                                const void* H, int B, int sample, float tau, uint64_t seed,
+                                uint64_t step, float* out_keys, uint32_t* status,
+                                uint32_t* tickets_to_clear, int n_tickets, int num_sms,
+                                cudaStream_t st) {
+  if (B < 1 || B > 64 || rows < 1 || d % 32 != 0 || n_tickets > kTcThreads) return cudaErrorInvalidValue;
+  TcInt4Params p = {};
+  p.rows = rows;
+  p.d = d;
+  p.B = B;
+  p.sample = sample;
+  p.tau = tau;
+  p.seed = seed;
+  p.step = step;
+  p.scales = scales;
+  p.out_keys = out_keys;
+  p.status = status;
+  p.tickets_to_clear = tickets_to_clear;
+  p.n_tickets = tickets_to_clear ? n_tickets : 0;
+  p.n_tiles = (int)((rows + 127) / 128);
+  CUtensorMap mH, mQ;
+  if (!make_map_h16(&mH, H, d, B, (uint32_t)((B + 15) / 16 * 16)) || !make_map_nib(&mQ, q4, d, rows))
+    return cudaErrorInvalidValue;
+  const size_t dyn = I4Layout::kSc + (size_t)128 * (d / 32) * 2 + 1024;
+  if (dyn > 227 * 1024) return cudaErrorInvalidValue;
+  auto kern = sample ? k_tc_keys_int4<true> : k_tc_keys_int4<false>;
+  cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(kern), dyn);
+  if (e != cudaSuccess) return e;
+  const int grid = p.n_tiles < num_sms ? p.n_tiles : num_sms;
+  kern<<<grid, kTcThreads, dyn, st>>>(mH, mQ, p);
+  return cudaGetLastError();
 }
 
 }  // namespace fh

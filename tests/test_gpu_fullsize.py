@@ -1,8 +1,8 @@
 """Parity with the oracle at the full sizes the benchmark runs, in the kernels those sizes select.
 
 * Gemma-3-1B-shaped INT4 Stage 1 (v=262144, d=1152, c=16384, p=1024): batch 1 runs the persistent
-  kernel with 512 threads (more than 8192 clusters), batch 8 the INT4 multi-query Stage 1 and the
-  per-query Stage 2, batch 32 the INT4 Stage 1 and the tensor-core Stage 2.
+  kernel with 512 threads (more than 8192 clusters), batch 8 the INT4 tensor-core Stage 1 and the
+  per-query Stage 2, batch 32 the INT4 tensor-core Stage 1 and the tensor-core Stage 2.
 * The crowded boundary bin at c > 8192 (the 512-thread full-selection branch).
 * Llama-3.2-1B-shaped batches of 16 and 64 queries (d=2048: 32 K-blocks per tile) on the
   tensor-core Stage 1 and Stage 2, greedy and sampling; the tensor-core Stage-1 keys element by

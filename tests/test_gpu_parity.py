@@ -109,7 +109,8 @@ def test_stage1_scores(fh, orc, tiny, mid):
 
 @pytest.mark.parametrize("B", [1, 3, 8])
 def test_stage1_scores_int4(fh, orc, mid_int4, B):
-    """One query per block at B = 1; eight per block otherwise (a partial group at B = 3)."""
+    """The CUDA-core kernel at B = 1 (one query per block); the dequantising tensor-core kernel at
+    B = 3 (a partial 16-query block) and B = 8."""
     idx, H = mid_int4
     I = load(fh, idx, int4=True)
     g = fh.stage1_scores(I, dev(H[:B], "bf16")).cpu().numpy()

@@ -40,6 +40,7 @@ constexpr size_t kGenOffset = 536;             // batch-1 head: tag of the last 
 constexpr size_t kTcTicketOffset = 544;        // tensor-core head: arrival ticket (zero between calls)
 constexpr size_t kKeysReadyOffset = 552;       // batch-1 head: arrivals before its full selection
 constexpr size_t kArriveOffset = 556;          // batch-1 head: arrivals at its final reduction
+constexpr size_t kUnionTicketOffset = 560;     // batched union Stage 2: arrival ticket (zero between calls)
 constexpr size_t kAlign = 256;
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -107,8 +108,9 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 }
 
 // Workspace header (first kHeaderBytes): status word at 0, per-query tickets at 16 (64 x 4 bytes),
-// the persistent head's call generation at 536 (the tag of the last completed call), its key-arrival
-// count at 552 and its final-reduction arrival count at 556; bytes
+// the persistent head's call generation at 536 (the tag of the last completed call), the tensor-core
+// head's ticket at 544, the persistent head's key-arrival count at 552 and its final-reduction arrival
+// count at 556, the union Stage 2's ticket at 560; bytes
 // [1024, 5120) hold its 1024-bin score histogram in every layout, so no other call ever writes there.
 // The tickets, the arrival counts and the generation only grow; the histogram returns to zero at the
 // end of every call, the word table is tagged with the call generation, and the per-block maxima
@@ -120,17 +122,20 @@ uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<
 uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
 
 // The tensor-core path: BF16 E (and, for FlashHead, its cluster-major copy), batches up to 64.  The
-// dense head takes it from 2 queries on; FlashHead from kTcMinBatchHead, below which the union of
-// the probe sets is sparse enough that the per-query CUDA-core Stage 2 reads fewer bytes.
+// dense head takes it from 2 queries on; FlashHead's Stage 1 from kTcMinBatchHead (below it the
+// CUDA-core kernels read the centroids as fast), its Stage 2 above kUnionMaxBatch (measured at the
+// Llama-3.2-1B shape: the union kernel 70 / 103 / 124 µs a call at 4 / 12 / 16 queries against
+// 73 / 145 / 148 µs before it; at 24 and 32 queries its 8-warp form, all that fits beside the query
+// vectors, took 237 and 290 µs against the tensor cores' 155 and 158 µs).
 constexpr int kTcMinBatchDense = 2;
 #ifndef FH_TC_MIN_BATCH_HEAD
 #define FH_TC_MIN_BATCH_HEAD 12
 #endif
-#ifndef FH_TC_LIST_TILES_BATCH
-#define FH_TC_LIST_TILES_BATCH 16
-#endif
 constexpr int kTcMinBatchHead = FH_TC_MIN_BATCH_HEAD;
-constexpr int kTcListTilesBatch = FH_TC_LIST_TILES_BATCH;  // from here on Stage 2 streams whole tiles
+#ifndef FH_UNION_MAX_BATCH
+#define FH_UNION_MAX_BATCH 16
+#endif
+constexpr int kUnionMaxBatch = FH_UNION_MAX_BATCH;
 bool tc_eligible(const fh_index* idx, int B, int min_batch) {
   const fh_index_desc& D = idx->desc;
   return B >= min_batch && D.dtype == FH_BF16 && fh::tc_supported(fh::kBF16, D.d, B);
@@ -236,11 +241,16 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     return FH_OK;
   }
   const bool fused = false;
-  // The tensor-core Stage 2 produces no per-candidate outputs: asking for them takes the CUDA-core
-  // Stage 2 instead; the probe sets alone can come from either.
+  // Stage 2 of a batch: the union of the probe sets streamed once on the CUDA cores (up to
+  // kUnionMaxBatch queries, while all query vectors fit shared memory), the tensor-core tiles above;
+  // neither produces per-candidate outputs, so asking for them takes the per-query Stage 2 instead
+  // (the probe sets alone can come from any of them).
   const bool per_cand = dbg && (dbg->cand_tok || dbg->cand_logit);
-  const bool tc = tc_eligible(idx, B, kTcMinBatchHead) && !per_cand && D.E_perm != nullptr;
-  if (tc && s1fmt(idx) == FH_STAGE1_DENSE) {
+  const int elem = D.dtype == FH_BF16 ? fh::kBF16 : fh::kF32;
+  const bool uni = B > 1 && B <= kUnionMaxBatch && !per_cand && D.E_perm != nullptr &&
+                   fh::union_supported(elem, D.d, D.v, D.b, B, idx->num_sms);
+  const bool tc = !uni && tc_eligible(idx, B, kTcMinBatchHead) && !per_cand && D.E_perm != nullptr;
+  if ((tc || uni) && tc_eligible(idx, B, kTcMinBatchHead) && s1fmt(idx) == FH_STAGE1_DENSE) {
     // Stage 1 on the tensor cores too: keys[q][k] = C[k]·h_q (+ the Gumbel term when sampling)
     fh::TcParams tp = {};
     tp.rows = D.c;
@@ -281,6 +291,38 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
         return cuda_fail(e, "debug copy");
     }
   }
+  if (uni) {
+    unsigned long long* qmask = reinterpret_cast<unsigned long long*>(base + L.qmask);
+    int32_t* list = reinterpret_cast<int32_t*>(base + L.tiles);
+    if ((e = cudaMemsetAsync(qmask, 0, (size_t)D.c * 8, st)) != cudaSuccess ||
+        (e = cudaMemsetAsync(list, 0, 4, st)) != cudaSuccess)
+      return cuda_fail(e, "memset");
+    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list + 1, list)) != cudaSuccess)
+      return cuda_fail(e, "mask launch");
+    fh::UnionParams up = {};
+    up.E_perm = D.E_perm;
+    up.C2T = D.C2T;
+    up.H = H;
+    up.v = D.v;
+    up.d = D.d;
+    up.c = D.c;
+    up.b = D.b;
+    up.B = B;
+    up.qmask = qmask;
+    up.cl_list = list + 1;
+    up.cl_count = list;
+    up.sample = sample;
+    up.tau = tau;
+    up.seed = seed;
+    up.step = step;
+    up.best = reinterpret_cast<unsigned long long*>(base + L.best);
+    up.ticket = word_at(ws, kUnionTicketOffset);
+    up.out_tok = out_tok;
+    up.status = status_of(ws);
+    if ((e = fh::launch_union_rows(up, elem, idx->num_sms, st)) != cudaSuccess)
+      return cuda_fail(e, "union stage-2 launch");
+    return FH_OK;
+  }
   if (tc) {
     // Stage 2 on the tensor cores: every tile of the cluster-major copy that some query selected,
     // masked per (cluster, query), the arg-max of each query fused in.
@@ -302,15 +344,9 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     tp.best = reinterpret_cast<unsigned long long*>(base + L.best);
     tp.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, kTcTicketOffset));
     tp.out_tok = out_tok;
-    if (B < kTcListTilesBatch && D.b % 8 == 0 && 128 % D.b == 0) {
-      // few queries: the union of the probe sets is sparse, gather its clusters into tiles
-      tp.cl_list = reinterpret_cast<int32_t*>(base + L.tiles) + 1;
-      tp.cl_count = reinterpret_cast<int32_t*>(base + L.tiles);
-    } else {
-      // many queries: the union covers most clusters, stream the contiguous tiles it touches
-      tp.tile_list = reinterpret_cast<int32_t*>(base + L.tiles) + 1;
-      tp.tile_count = reinterpret_cast<int32_t*>(base + L.tiles);
-    }
+    // the 128-row tiles that hold a cluster some query takes
+    tp.tile_list = reinterpret_cast<int32_t*>(base + L.tiles) + 1;
+    tp.tile_count = reinterpret_cast<int32_t*>(base + L.tiles);
     tp.status = status_of(ws);
     if ((e = fh::launch_tc_head(D.E_perm, H, tp, idx->num_sms, st)) != cudaSuccess)
       return cuda_fail(e, "tensor-core stage-2 launch");

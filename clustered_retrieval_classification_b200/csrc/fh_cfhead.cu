@@ -9,10 +9,11 @@
 // Kernels, one call (grid.y = query):
 //   k_cf_lut      LUT[q][t][j] = Cb[t][j]·h_q[t·w ..) (fp32, column order); zeroes the query's
 //                 histogram and list counters for this call
-//   k_cf_coarse   each block: the query's LUT into shared memory, the bound R = Σ_t max_j |LUT[t][j]|
-//                 (|ŝ| <= R) and from it the binning; then one thread per token: ŝ_u = Σ_t LUT[t][code]
-//                 in tile order, 32-bit code words read coalesced (one word row = 8 tiles of 32
-//                 consecutive tokens = 128 bytes); a 4096-bin histogram of the scores
+//   k_cf_coarse   each block: the query's LUT into shared memory (one bulk copy), the bound
+//                 R = Σ_t max_j |LUT[t][j]| (|ŝ| <= R) and from it the binning; then one thread per
+//                 token: ŝ_u = Σ_t LUT[t][code] as four partial sums (tiles t mod 4), 32-bit code words
+//                 read coalesced (one word row = 8 tiles of 32 consecutive tokens = 128 bytes) in
+//                 batches of 16 with the next batch in flight; a 4096-bin histogram of the scores
 //   k_cf_compact  each block: the boundary bin d* from the summed histogram (where the count from the
 //                 top reaches k); its tokens above d* go to the candidate list, the boundary bin's
 //                 (score, id) pairs to the boundary list (warp-aggregated appends)
@@ -113,25 +114,43 @@ __global__ void __launch_bounds__(kCfThreads) k_cf_lut(const CfParams p) {
 
 // ------------------------------------------------------------------ coarse scores
 
-constexpr int kCfWordsInFlight = 32;  // code words a thread requests before its first look-up
+constexpr int kCfWordsInFlight = 16;  // code words per batch; two batches are in flight
 
 __global__ void __launch_bounds__(kCfThreads) k_cf_coarse(const CfParams p) {
   extern __shared__ __align__(16) float lut_s[];  // T x K, then kCfBins histogram words
   __shared__ float red_s[kCfThreads / 32];
+  __shared__ __align__(8) uint64_t lut_bar;
   const int q = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int TK = p.T * p.K;
   const int G8 = p.T / 8;
   const int64_t v = p.v;
   const int64_t u = (int64_t)blockIdx.x * kCfThreads + tid;  // one token per thread
   const uint32_t* col = p.codes + (u < v ? u : 0);
-  // the first word rows of this token, in flight while the look-up table is staged
-  uint32_t wv[kCfWordsInFlight];
-#pragma unroll
-  for (int g = 0; g < kCfWordsInFlight; ++g) wv[g] = (g < G8 && u < v) ? __ldg(col + (size_t)g * v) : 0u;
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(lut_s + TK);
-  for (int i = tid; i < TK; i += kCfThreads) lut_s[i] = p.lut[(size_t)q * TK + i];
-  for (int b = tid; b < kCfBins; b += kCfThreads) hist_s[b] = 0u;
+  // the query's look-up table in one bulk copy, while each thread requests its first word rows (the
+  // barrier is initialised and made visible to the block before anyone waits on it)
+  if (tid == 0) {
+    mbar_init(&lut_bar, 1);
+    fence_mbar_init();
+  }
   __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&lut_bar, (uint32_t)TK * 4u);
+    bulk_g2s(lut_s, p.lut + (size_t)q * TK, (uint32_t)TK * 4u, &lut_bar);
+  }
+  uint32_t wa[kCfWordsInFlight], wb[kCfWordsInFlight];
+  auto load = [&](uint32_t (&w)[kCfWordsInFlight], int g0) {
+#pragma unroll
+    for (int g = 0; g < kCfWordsInFlight; ++g)
+      w[g] = (g0 + g < G8 && u < v) ? __ldg(col + (size_t)(g0 + g) * v) : 0u;
+  };
+  load(wa, 0);
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(lut_s + TK);
+  for (int b = tid; b < kCfBins; b += kCfThreads) hist_s[b] = 0u;
+  const bool lut_ok = mbar_wait(&lut_bar, 0u, p.status);
+  if (!__syncthreads_and(lut_ok)) {  // (status recorded) the copy lands before the block leaves
+    if (tid == 0) mbar_wait(&lut_bar, 0u, nullptr, 50000000ull);
+    return;
+  }
   // |ŝ_u| <= R = Σ_t max_j |LUT[t][j]| (fixed order: identical in every block)
   float part = 0.0f;
   for (int t = tid; t < p.T; t += kCfThreads) {
@@ -152,25 +171,34 @@ __global__ void __launch_bounds__(kCfThreads) k_cf_coarse(const CfParams p) {
   if (blockIdx.x == 0 && tid == 0) p.scale[q] = scale;
 
   if (u < v) {
-    float acc = 0.0f;  // Σ_t LUT[t][code], tiles in order
-#pragma unroll
-    for (int g = 0; g < kCfWordsInFlight; ++g) {
-      if (g < G8) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc += lut_s[(8 * g + j) * p.K + ((wv[g] >> (4 * j)) & 15u)];
-      }
-    }
-    for (int g0 = kCfWordsInFlight; g0 < G8; g0 += kCfWordsInFlight) {
-#pragma unroll
-      for (int g = 0; g < kCfWordsInFlight; ++g) wv[g] = (g0 + g < G8) ? __ldg(col + (size_t)(g0 + g) * v) : 0u;
+    // Σ_t LUT[t][code] as four partial sums over the tiles t ≡ 0, 1, 2, 3 (mod 4), each in tile
+    // order, then (s0 + s1) + (s2 + s3); the word batches alternate between two register sets so that
+    // one is in flight while the other is summed
+    float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+    auto sum = [&](const uint32_t (&w)[kCfWordsInFlight], int g0) {
 #pragma unroll
       for (int g = 0; g < kCfWordsInFlight; ++g) {
         if (g0 + g < G8) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) acc += lut_s[(8 * (g0 + g) + j) * p.K + ((wv[g] >> (4 * j)) & 15u)];
+          const float* lt = lut_s + (size_t)(8 * (g0 + g)) * p.K;
+          const uint32_t x = w[g];
+          a0 += lt[0 * p.K + (x & 15u)];
+          a1 += lt[1 * p.K + ((x >> 4) & 15u)];
+          a2 += lt[2 * p.K + ((x >> 8) & 15u)];
+          a3 += lt[3 * p.K + ((x >> 12) & 15u)];
+          a0 += lt[4 * p.K + ((x >> 16) & 15u)];
+          a1 += lt[5 * p.K + ((x >> 20) & 15u)];
+          a2 += lt[6 * p.K + ((x >> 24) & 15u)];
+          a3 += lt[7 * p.K + (x >> 28)];
         }
       }
+    };
+    for (int g0 = 0; g0 < G8; g0 += 2 * kCfWordsInFlight) {
+      if (g0 + kCfWordsInFlight < G8) load(wb, g0 + kCfWordsInFlight);
+      sum(wa, g0);
+      if (g0 + 2 * kCfWordsInFlight < G8) load(wa, g0 + 2 * kCfWordsInFlight);
+      if (g0 + kCfWordsInFlight < G8) sum(wb, g0 + kCfWordsInFlight);
     }
+    const float acc = (a0 + a1) + (a2 + a3);
     p.coarse[(size_t)q * v + u] = acc;
     atomicAdd(&hist_s[cf_bin(acc, scale)], 1u);
   }

@@ -64,8 +64,16 @@ constexpr int kHistBins = kHead1Bins;
 #define FH_H1_PRE_ROWS 1
 #endif
 constexpr int kHead1PreRows = FH_H1_PRE_ROWS;
+#ifndef FH_H1_S1_WARP_BYTES
+#define FH_H1_S1_WARP_BYTES 12288
+#endif
+#ifndef FH_H1_S2_WARP_BYTES
+#define FH_H1_S2_WARP_BYTES 8192
+#endif
+constexpr uint32_t kHead1Stage1WarpBytes = FH_H1_S1_WARP_BYTES;
+constexpr uint32_t kHead1Stage2WarpBytes = FH_H1_S2_WARP_BYTES;
 constexpr int kCap = kHead1BucketCap;
-static_assert(kCap % 32 == 0 && kCap <= kSelCandMax, "bucket words are ranked by warps");
+static_assert(kCap % 32 == 0 && kCap <= kSelCandMax && kCap <= 256, "bucket words are ranked by warps");
 
 // ------------------------------------------------------------------ key binning
 // x = key·scale with scale a power of two (exact for every |x| >= 2^-126), then, on each side of zero,
@@ -212,7 +220,7 @@ __device__ __forceinline__ void rank_boundary(const uint32_t* cand_key, const in
 // ------------------------------------------------------------------ shared-memory layout
 
 struct Head1Layout {
-  uint32_t bars1, bars2, hs, sc, sel, hist, histg, ownk, ownp, rkid, asc, tokr, ring, total;
+  uint32_t bars1, bars2, hs, sc, sel, hist, histg, ownk, ownp, rkid, asc, tokr, zr, ring, total;
 };
 
 __host__ __device__ inline uint32_t h1_align(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -239,7 +247,8 @@ __host__ __device__ inline Head1Layout head1_layout(uint32_t row2, int rows1_max
   L.rkid = h1_align(L.ownp + (uint32_t)rows1_max * 4u, 16);
   L.asc = h1_align(L.rkid + (uint32_t)rmax * 4u, 16);
   L.tokr = h1_align(L.asc + (uint32_t)rmax * 4u, 16);
-  L.ring = h1_align(L.tokr + (uint32_t)rmax * (uint32_t)h1_tok_words(b) * 4u, 128);
+  L.zr = h1_align(L.tokr + (uint32_t)rmax * (uint32_t)h1_tok_words(b) * 4u, 16);  // rmax * b >= its rows
+  L.ring = h1_align(L.zr + (uint32_t)rmax * (uint32_t)b * 4u, 128);
   L.total = L.ring + ring_bytes;
   return L;
 }
@@ -568,15 +577,18 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     }
     int* bsel = reinterpret_cast<int*>(sm.selbits);  // boundary ids in rank order (need <= kCap)
     if (bnd_ranks && need > 0u) {
+      // the boundary words are read by the last kCap threads, so that their loads go out together
+      // with the certain words of the first threads
       const unsigned long long* bw = prm.bucket + (size_t)dstar * kCap;
+      const int bt = tid - (NT - kCap);
       if (need == m_total) {  // the whole bin is taken: any order will do, take the positions
-        if (tid < (int)m_total) bsel[tid] = word_id(poll_tagged(bw + tid, tag, prm.status, ok));
+        if (bt >= 0 && bt < (int)m_total) bsel[bt] = word_id(poll_tagged(bw + bt, tag, prm.status, ok));
       } else {
         uint32_t* ckey = reinterpret_cast<uint32_t*>(sm.cand_key);
-        if (tid < (int)m_total) {
-          const unsigned long long w = poll_tagged(bw + tid, tag, prm.status, ok);
-          ckey[tid] = (uint32_t)(w & 0x1FFFFull) + 1u;  // 0 stays below every key
-          sm.cand_id[tid] = word_id(w);
+        if (bt >= 0 && bt < (int)m_total) {
+          const unsigned long long w = poll_tagged(bw + bt, tag, prm.status, ok);
+          ckey[bt] = (uint32_t)(w & 0x1FFFFull) + 1u;  // 0 stays below every key
+          sm.cand_id[bt] = word_id(w);
         }
         if (!__syncthreads_and(ok)) return;
         rank_boundary<kCap / 32>(ckey, sm.cand_id, m_total, need, bsel, lane, warp, W);
@@ -694,31 +706,37 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   H1_STAMP(5);
 
   // ------------------------------------------------------------------ Stage 2
-  // The C2T rows of the touched clusters first (one small copy each; b ids widened to 16-byte
-  // chunks), then this warp's first K2 candidate rows.
+  // This warp's first K2 candidate rows go out first (rows of the cluster-major copy are addressed by
+  // cluster id alone), then the C2T rows of the touched clusters (one small copy each; b ids widened
+  // to 16-byte chunks).  The logits are kept per row and turned into decision keys once the stream is
+  // over, so the token ids never stand in front of a row.
   const int nr = r1 - r0;
   const int n2 = (warp < nr) ? (nr - warp + W - 1) / W : 0;
   uint8_t* ring2 = ring + (size_t)warp * K2 * row2;
   uint64_t* b2 = bars2 + warp * K2;
-  if (tid == 0 && nrk > 0) {
-    uint32_t bytes = 0;
-    for (int i = 0; i < nrk; ++i) {
-      const int e0 = rk_id[i] * b;
-      bytes += (uint32_t)(((e0 + b + 3) & ~3) - (e0 & ~3)) * 4u;
+  float* zr = reinterpret_cast<float*>(smem + L.zr);  // logit of block row g - r0
+  auto issue_tok = [&]() {
+    if (tid == 0 && nrk > 0) {
+      uint32_t bytes = 0;
+      for (int i = 0; i < nrk; ++i) {
+        const int e0 = rk_id[i] * b;
+        bytes += (uint32_t)(((e0 + b + 3) & ~3) - (e0 & ~3)) * 4u;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive_expect_tx(tok_bar, bytes);
+      for (int i = 0; i < nrk; ++i) {
+        const int e0 = rk_id[i] * b;
+        const int s0 = e0 & ~3;
+        bulk_g2s(tokr + i * tsw, prm.C2T + s0, (uint32_t)(((e0 + b + 3) & ~3) - s0) * 4u, tok_bar);
+      }
     }
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(tok_bar, bytes);
-    for (int i = 0; i < nrk; ++i) {
-      const int e0 = rk_id[i] * b;
-      const int s0 = e0 & ~3;
-      bulk_g2s(tokr + i * tsw, prm.C2T + s0, (uint32_t)(((e0 + b + 3) & ~3) - s0) * 4u, tok_bar);
-    }
-  }
+  };
   auto token_of = [&](int q, int j) {  // rank q (global), row j of its cluster
     const int e0 = rk_id[q - rk0] * b;
     return tokr[(q - rk0) * tsw + (e0 & 3) + j];
   };
   if (!perm) {  // the rows are addressed through their token ids: wait for the C2T rows
+    issue_tok();
     const bool ok = nrk == 0 || mbar_wait(tok_bar, 0u, prm.status);
     if (!__syncthreads_and(ok)) return;
   }
@@ -735,16 +753,17 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     fence_proxy_async_smem();  // the ring was last read by Stage 1 and the selection
     issue2(lane);
   }
-  unsigned long long best = 0ull;
-  bool tok_ok = true;
-  if (perm && n2 > 0 && lane == 0)  // the C2T rows went out ahead of every E row
-    tok_ok = mbar_wait(tok_bar, 0u, prm.status);
-  tok_ok = __shfl_sync(0xFFFFFFFFu, tok_ok, 0);
+  if (perm) {
+    __syncwarp();
+    issue_tok();
+  }
   H1_STAMP(10);
-  for (int n = 0, slot = 0, phase = 0; n < n2 && tok_ok; ++n) {
+  bool ok2 = true;
+  for (int n = 0, slot = 0, phase = 0; n < n2; ++n) {
     if (!mbar_wait(&b2[slot], (uint32_t)phase, prm.status)) {
       for (int m = n + 1; m < n2 && m < n + K2; ++m)
         mbar_wait(&b2[m % K2], (uint32_t)((m / K2) & 1), nullptr, 50000000ull);
+      ok2 = false;
       break;
     }
     if (n == 0) H1_STAMP(6);
@@ -757,29 +776,42 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
         fence_proxy_async_smem();
         issue2(n + K2);
       }
-      const int q = g / b, j = g - q * b;
-      const uint32_t tok = (uint32_t)token_of(q, j);
-      float val = z;
-      if (prm.sample)
-        val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 1u, tok));
-      const unsigned long long pk = pack_best(val, tok);
-      best = pk > best ? pk : best;
-      if (want_dbg) {
-        const int ai = asc_of[q - rk0] * b + j;
-        if (prm.dbg_logit) prm.dbg_logit[ai] = z;
-        if (prm.dbg_tok) prm.dbg_tok[ai] = (int32_t)tok;
-      }
+      zr[g - r0] = z;
     }
     if (++slot == K2) {
       slot = 0;
       phase ^= 1;
     }
   }
-  if (!tok_ok) {  // (status recorded) the E rows already requested land before the block leaves
-    for (int m = 0; m < n2 && m < K2; ++m)
-      mbar_wait(&b2[m % K2], 0u, nullptr, 50000000ull);
+  // the decision keys of this warp's rows (lane l takes rows l, l + 32, ...) once the ids are in
+  bool tok_ok = ok2;
+  if (perm && n2 > 0 && ok2) {
+    if (lane == 0) tok_ok = mbar_wait(tok_bar, 0u, prm.status);
+    tok_ok = __shfl_sync(0xFFFFFFFFu, tok_ok, 0);
+  }
+  if (!tok_ok) {  // (status recorded) the C2T copies land before the block leaves
+    if (perm && tid == 0 && nrk > 0) mbar_wait(tok_bar, 0u, nullptr, 50000000ull);
     return;
   }
+  __syncwarp();
+  unsigned long long best = 0ull;
+  for (int n = lane; n < n2; n += 32) {
+    const int g = r0 + warp + W * n;
+    const int q = g / b, j = g - q * b;
+    const uint32_t tok = (uint32_t)token_of(q, j);
+    const float z = zr[g - r0];
+    float val = z;
+    if (prm.sample)
+      val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 1u, tok));
+    const unsigned long long pk = pack_best(val, tok);
+    best = pk > best ? pk : best;
+    if (want_dbg) {
+      const int ai = asc_of[q - rk0] * b + j;
+      if (prm.dbg_logit) prm.dbg_logit[ai] = z;
+      if (prm.dbg_tok) prm.dbg_tok[ai] = (int32_t)tok;
+    }
+  }
+  best = warp_max_u64(best);
 
   // ------------------------------------------------------------------ arg-max over the grid
   // Every block posts its best (value, ~token) to its slot and counts itself in with a release add;
@@ -868,17 +900,23 @@ cudaError_t launch_head1(Head1Params prm, int elem, int int4, int num_sms, cudaS
   const int kcap = (1024 / 8 - 2) / W;  // barriers per stage (the last two of bars2 are reserved)
   if (fixed + (uint32_t)W * (row2 > row1 ? row2 : row1) > budget) return cudaErrorInvalidValue;
   const uint32_t ring_bytes = (budget - fixed) / 128u * 128u;
-  auto slots = [&](uint32_t row, int64_t rows) {
+  // Rows in flight per warp: about kHead1Stage1WarpBytes / kHead1Stage2WarpBytes of copies.  Fewer
+  // bytes in flight than the ring holds make the first rows of each block land sooner and the blocks
+  // finish closer together (measured at the Llama-3.2-1B shape: 12 KiB / 8 KiB per warp gave 20.6 µs
+  // a call, 48 KiB / 24 KiB 22.2 µs, 16 KiB / 4 KiB 22.8 µs).
+  auto slots = [&](uint32_t row, int64_t rows, uint32_t warp_bytes) {
     int64_t k = ring_bytes / ((uint64_t)W * row);
     const int64_t per_warp = (rows + W - 1) / W;
+    const int64_t want = warp_bytes / row;
+    if (k > want) k = want;
     if (k > per_warp) k = per_warp;
     if (k > kcap) k = kcap;
     return (int)(k < 1 ? 1 : k);
   };
   // the crowded-bin selection copies all keys into the ring, the debug outputs list the probe set there
   if (ring_bytes < (uint32_t)((prm.c * 4 + 15) / 16 * 16)) return cudaErrorInvalidValue;
-  prm.k1 = slots(row1, rows1_max);
-  prm.k2 = slots(row2, rows2_max);
+  prm.k1 = slots(row1, rows1_max, kHead1Stage1WarpBytes);
+  prm.k2 = slots(row2, rows2_max, kHead1Stage2WarpBytes);
   prm.ring_bytes = ring_bytes;
   const size_t smem = fixed + ring_bytes;
 

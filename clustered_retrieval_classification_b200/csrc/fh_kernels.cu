@@ -11,7 +11,9 @@
 //   k_stage1_int4<M> the same from INT4 centroids with BF16 group scales, one query    (Stage 1, INT4)
 //   k_stage1_int4_mq<M,QB> INT4 for QB queries per block, each group decoded once      (Stage 1, INT4)
 //   k_select<KPT>    top-p per query                                                    (selection)
-//   k_build_qmask    per-cluster bit masks of the queries that selected it              (tensor-core Stage 2)
+//   k_build_qmask    per-cluster bit masks of the queries that selected it, and the list of
+//                    the clusters some query selected                                   (batched Stage 2)
+//   k_union_rows<E>  the union of a batch's probe sets, each row read once for the batch (batched Stage 2)
 //   k_rows<E,MODE,KPT> candidates (fused selection or given sets) or all rows (dense):
 //                    dot, arg-max / Gumbel-max, partial results, last-block reduction   (Stage 2, dense)
 // The batch-1 head is one persistent kernel (fh_head1.cu); batched BF16 heads run on the tensor
@@ -62,10 +64,13 @@ __global__ void __launch_bounds__(kThreads) k_stage1(const Stage1Params prm, int
   const uint32_t hs_addr = smem_addr(hs);
   auto src = [&](int64_t k) { return C + (size_t)k * row_bytes; };
   auto body = [&](int64_t k, uint32_t row_s) {
+    float part[QB];
+    if constexpr (QB == 1) part[0] = row_dot_partial<ELEM>(row_s, hs_addr, nch, lane);
+    else row_dot_partial_multi<ELEM, QB>(row_s, hs_addr, row_bytes, nch, nq, lane, part);
 #pragma unroll
     for (int q = 0; q < QB; ++q) {
       if (q < nq) {
-        const float s = warp_sum(row_dot_partial<ELEM>(row_s, hs_addr + q * row_bytes, nch, lane));
+        const float s = warp_sum(part[q]);
         if (lane == 0) {
           float out = s;
           if (prm.sample)
@@ -414,6 +419,141 @@ __global__ void __launch_bounds__(kThreads) k_rows(const Stage2Params prm, int K
   }
 }
 
+// ============================================================================ Stage 2 (union of the batch)
+// Batched Stage 2 over the union of the probe sets (FlashHead notes, Figure 1 Stage 2, for a batch):
+// the clusters some query selected, listed once each (in the order k_build_qmask found them), are
+// streamed once as whole rows of the cluster-major copy; every row is dotted with the queries whose probe set holds its cluster (the
+// cluster's query mask) and folded into those queries' running arg-max.  All B query vectors stay in
+// shared memory; block b takes the union's rows [R·b/G, R·(b+1)/G), R = (listed clusters)·b.
+
+struct UnionSmemLayout {
+  uint32_t bars, hs, ring, tok, msk, cls, total;
+};
+
+__host__ __device__ inline UnionSmemLayout union_layout(uint32_t row_bytes, int B, int NW, int K,
+                                                        int rows_max, int cl_max) {
+  UnionSmemLayout L;
+  L.bars = 0;  // NW * K ring barriers and the query vectors' barrier (NW * K < 128)
+  L.hs = 1024;
+  L.ring = align_up(L.hs + (uint32_t)B * row_bytes, 128);
+  L.tok = align_up(L.ring + (uint32_t)NW * K * row_bytes, 16);
+  L.msk = align_up(L.tok + (uint32_t)rows_max * 4u, 16);
+  L.cls = align_up(L.msk + (uint32_t)cl_max * 8u, 16);
+  L.total = align_up(L.cls + (uint32_t)cl_max * 4u, 128);
+  return L;
+}
+
+template <int ELEM, int NW>
+__global__ void __launch_bounds__(NW * 32) k_union_rows(const UnionParams prm, int K, int rows_max, int cl_max) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t row_bytes = (uint32_t)(prm.d * (ELEM == kBF16 ? 2 : 4));
+  const int nch = (int)(row_bytes / 16);
+  const UnionSmemLayout L = union_layout(row_bytes, prm.B, NW, K, rows_max, cl_max);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint8_t* hs = smem + L.hs;
+  uint8_t* ring = smem + L.ring;
+  int32_t* tok_s = reinterpret_cast<int32_t*>(smem + L.tok);
+  unsigned long long* msk_s = reinterpret_cast<unsigned long long*>(smem + L.msk);
+  int32_t* cl_s = reinterpret_cast<int32_t*>(smem + L.cls);  // the block's listed clusters
+  __shared__ unsigned long long blk_best[NW][64];
+  __shared__ bool is_last;
+
+  // 32-bit row arithmetic: the union has at most v < 2^31 rows
+  const uint32_t b = (uint32_t)prm.b;
+  const int n_cl = __ldg(prm.cl_count);
+  const int64_t R = (int64_t)n_cl * b;
+  const uint32_t lo = (uint32_t)(R * blockIdx.x / gridDim.x), hi = (uint32_t)(R * (blockIdx.x + 1) / gridDim.x);
+  const uint32_t c_lo = lo / b;  // first listed cluster this block touches
+  const uint32_t c_hi = hi > lo ? (hi - 1) / b + 1 : c_lo;
+  const uint8_t* Ep = static_cast<const uint8_t*>(prm.E_perm);
+  auto src = [&](uint32_t i) -> const uint8_t* {
+    const uint32_t ci = i / b;
+    return Ep + ((size_t)cl_s[ci - c_lo] * b + (i - ci * b)) * row_bytes;
+  };
+  const uint32_t first = lo + warp;
+  const int nw = (first < hi) ? (int)((hi - first + NW - 1) / NW) : 0;
+  uint8_t* ring_w = ring + (size_t)warp * K * row_bytes;
+  uint64_t* bars_w = bars + warp * K;
+
+  uint64_t* hbar = bars + NW * K;  // the query vectors
+  if (tid < NW * K + 1) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
+  for (uint32_t ci = c_lo + tid; ci < c_hi; ci += NW * 32) cl_s[ci - c_lo] = __ldg(prm.cl_list + ci);
+  __syncthreads();
+  // the query vectors (one bulk copy) and the first rows, then the token ids and the cluster masks
+  if (tid == 0) issue_row(hs, prm.H, (uint32_t)prm.B * row_bytes, hbar);
+  if (lane == 0)
+    for (int n = 0; n < K && n < nw; ++n)
+      issue_row(ring_w + (size_t)n * row_bytes, src(first + (uint32_t)(NW * n)), row_bytes, &bars_w[n]);
+  for (uint32_t i = lo + tid; i < hi; i += NW * 32) {
+    const uint32_t ci = i / b;
+    tok_s[i - lo] = __ldg(prm.C2T + (size_t)cl_s[ci - c_lo] * b + (i - ci * b));
+  }
+  for (uint32_t ci = c_lo + tid; ci < c_hi; ci += NW * 32) msk_s[ci - c_lo] = __ldg(prm.qmask + cl_s[ci - c_lo]);
+  const bool h_ok = mbar_wait(hbar, 0u, prm.status);
+  if (!__syncthreads_and(h_ok)) {  // (status recorded) the rows already requested land first
+    if (lane == 0)
+      for (int n = 0; n < K && n < nw; ++n) mbar_wait(&bars_w[n], 0u, nullptr, 50000000ull);
+    return;
+  }
+
+  const uint32_t hs_addr = smem_addr(hs);
+  unsigned long long best0 = 0ull, best1 = 0ull;  // queries lane and lane + 32
+  for (int n = 0; n < nw; ++n) {
+    const int slot = (int)(n % K);
+    if (!mbar_wait(&bars_w[slot], (uint32_t)((n / K) & 1), prm.status)) {
+      for (int m = n + 1; m < nw && m < n + K; ++m)
+        mbar_wait(&bars_w[m % K], (uint32_t)((m / K) & 1), nullptr, 50000000ull);
+      break;
+    }
+    const uint32_t i = first + (uint32_t)(NW * n);
+    const uint32_t row_s = smem_addr(ring_w + (size_t)slot * row_bytes);
+    const uint32_t tok = (uint32_t)tok_s[i - lo];
+    unsigned long long mk = msk_s[i / b - c_lo];
+    while (mk) {  // the same queries in every lane
+      const int q = __ffsll((long long)mk) - 1;
+      mk &= mk - 1;
+      const float z = warp_sum(row_dot_partial<ELEM>(row_s, hs_addr + (uint32_t)q * row_bytes, nch, lane));
+      if (lane == (q & 31)) {
+        float val = z;
+        if (prm.sample)
+          val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, 1u, tok));
+        const unsigned long long pk = pack_best(val, tok);
+        if (q < 32) best0 = pk > best0 ? pk : best0;
+        else best1 = pk > best1 ? pk : best1;
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && n + K < nw) {
+      fence_proxy_async_smem();
+      issue_row(ring_w + (size_t)slot * row_bytes, src(first + (uint32_t)(NW * (n + K))), row_bytes,
+                &bars_w[slot]);
+    }
+  }
+
+  blk_best[warp][lane] = best0;
+  blk_best[warp][lane + 32] = best1;
+  __syncthreads();
+  if (tid < prm.B) {
+    unsigned long long bb = 0ull;
+    for (int w = 0; w < NW; ++w) bb = blk_best[w][tid] > bb ? blk_best[w][tid] : bb;
+    if (bb) atomicMax(prm.best + tid, bb);
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) is_last = atomicAdd(prm.ticket, 1u) + 1u == gridDim.x;
+  __syncthreads();
+  if (is_last) {  // every other block has added its maxima: publish, and leave zeros for the next call
+    __threadfence();
+    if (tid < prm.B) {
+      const unsigned long long fin = atomicExch(prm.best + tid, 0ull);
+      prm.out_tok[tid] = fin ? (int32_t)best_id(fin) : -1;
+    }
+    if (tid == 0) atomicExch(prm.ticket, 0u);
+  }
+}
+
 // Dense head: the same kernel over all rows; logits optionally written out.
 template <int ELEM>
 __global__ void __launch_bounds__(kThreads) k_dense(const DenseParams prm, int K) {
@@ -645,9 +785,11 @@ __global__ void k_mc_reduce(const double* per_draw, int64_t N, int T, int B, dou
 
 // ============================================================================ launchers
 
+// Ring slots per warp for rows of row_bytes within `budget` bytes of ring: at least 1, at most 16 (the
+// kernels keep kWarps x 16 mbarriers in their first 1024 bytes of shared memory).
 static int ring_slots(uint32_t row_bytes, uint32_t budget) {
   int k = (int)(budget / ((uint32_t)kWarps * row_bytes));
-  return k < 1 ? 1 : (k > 8 ? 8 : k);
+  return k < 1 ? 1 : (k > 16 ? 16 : k);
 }
 
 // Raise a kernel's dynamic shared-memory limit to `bytes`, remembering the limits already set so
@@ -677,7 +819,7 @@ cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_s
   (void)pdl_primary;
   if (int4) {
     const uint32_t row_bytes = (uint32_t)(prm.d / 2);
-    const int K = ring_slots(row_bytes, 32 * 1024);
+    const int K = ring_slots(row_bytes, 96 * 1024);
     const int G = num_sms;
     const int rows_max = (int)((prm.c + G - 1) / G);
     const int nch = (int)(prm.d / 32);
@@ -714,7 +856,7 @@ cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_s
     return cudaGetLastError();
   }
   const uint32_t row_bytes = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
-  const int K = ring_slots(row_bytes, 64 * 1024);
+  const int K = ring_slots(row_bytes, 160 * 1024);
   const int QB = prm.B == 1 ? 1 : 4;
   const size_t smem = 1024 + (size_t)QB * row_bytes + (size_t)kWarps * K * row_bytes;
   dim3 grid(num_sms, (prm.B + QB - 1) / QB);
@@ -751,17 +893,23 @@ cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int
 }
 
 // qmask[cluster] |= 1 << q for every cluster in query q's probe set (qmask zeroed beforehand).
-__global__ void k_build_qmask(const int32_t* __restrict__ sel, int B, int p, unsigned long long* qmask) {
+// list (optional, with *count zeroed like qmask): the clusters with a nonzero mask, each appended once
+// by the query that sets its first bit (in no particular order).
+__global__ void k_build_qmask(const int32_t* __restrict__ sel, int B, int p, unsigned long long* qmask,
+                              int32_t* list, int32_t* count) {
   const int64_t n = (int64_t)B * p;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    atomicOr(qmask + sel[i], 1ull << (uint32_t)(i / p));
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t k = sel[i];
+    const unsigned long long old = atomicOr(qmask + k, 1ull << (uint32_t)(i / p));
+    if (list && old == 0ull) list[atomicAdd(count, 1)] = k;
+  }
 }
 
 cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
-                               cudaStream_t st) {
+                               cudaStream_t st, int32_t* list, int32_t* count) {
   const int64_t n = (int64_t)B * p;
   const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
-  k_build_qmask<<<blocks, 256, 0, st>>>(sel, B, p, qmask);
+  k_build_qmask<<<blocks, 256, 0, st>>>(sel, B, p, qmask, list, count);
   return cudaGetLastError();
 }
 
@@ -788,6 +936,55 @@ cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaSt
     if ((e = set_smem(k_rows<kF32>, smem)) != cudaSuccess) return e;
     k_rows<kF32><<<dim3(G, prm.B), kThreads, smem, st>>>(prm, K, rows_max);
   }
+  return cudaGetLastError();
+}
+
+// Warps and ring slots of the union kernel at batch B: 16 warps when two slots each fit beside the
+// query vectors (more rows in flight and more warps to hide the dot products' latency), else 8;
+// 0 slots: the query vectors leave no room for a ring of two.
+static int union_slots(uint32_t row_bytes, int B, int rows_max, int cl_max, int* nw, size_t* smem) {
+  for (int NW : {16, 8})
+    for (int K = 128 / NW - 1; K >= 2; --K) {
+      const UnionSmemLayout L = union_layout(row_bytes, B, NW, K, rows_max, cl_max);
+      if (L.total <= 200u * 1024u) {
+        *nw = NW;
+        *smem = L.total;
+        return K;
+      }
+    }
+  return 0;
+}
+
+bool union_supported(int elem, int64_t d, int64_t v, int64_t b, int B, int num_sms) {
+  if (B < 1 || B > 64) return false;
+  const uint32_t row_bytes = (uint32_t)(d * (elem == kBF16 ? 2 : 4));
+  const int rows_max = (int)((v + num_sms - 1) / num_sms);
+  size_t smem;
+  int nw;
+  return union_slots(row_bytes, B, rows_max, (int)(rows_max / b + 2), &nw, &smem) >= 2;
+}
+
+cudaError_t launch_union_rows(const UnionParams& prm, int elem, int num_sms, cudaStream_t st) {
+  const uint32_t row_bytes = (uint32_t)(prm.d * (elem == kBF16 ? 2 : 4));
+  const int G = num_sms;
+  const int rows_max = (int)((prm.v + G - 1) / G);  // the union has at most v rows
+  const int cl_max = (int)(rows_max / prm.b + 2);
+  size_t smem = 0;
+  int NW = 8;
+  const int K = union_slots(row_bytes, prm.B, rows_max, cl_max, &NW, &smem);
+  if (K < 2) return cudaErrorInvalidValue;
+  cudaError_t e;
+#define FH_UN(EL, W)                                                             \
+  do {                                                                           \
+    if ((e = set_smem(k_union_rows<EL, W>, smem)) != cudaSuccess) return e;      \
+    k_union_rows<EL, W><<<G, W * 32, smem, st>>>(prm, K, rows_max, cl_max);      \
+  } while (0)
+  if (elem == kBF16) {
+    if (NW == 16) FH_UN(kBF16, 16); else FH_UN(kBF16, 8);
+  } else {
+    if (NW == 16) FH_UN(kF32, 16); else FH_UN(kF32, 8);
+  }
+#undef FH_UN
   return cudaGetLastError();
 }
 

@@ -107,17 +107,36 @@ struct TcParams {
   int32_t* out_tok;                // B, or null
   float* out_logits;               // B x rows indexed by token, or null
   float* out_keys;                 // B x rows: write the raw products (Stage-1 keys) instead
-  int32_t* cl_list;                // rows/b scratch: gather the clusters some query takes, or null
-  int32_t* cl_count;               // 1 scratch word: their number
   int32_t* tile_list;              // rows/128 scratch: or stream the 128-row tiles some query takes
   int32_t* tile_count;             // 1 scratch word: their number (both lists null: every tile)
   uint32_t* status;
   int n_tiles, tile_rows, stages;  // set by the launcher
 };
+// Batched Stage 2 over the union of the batch's probe sets (fh_kernels.cu): the listed clusters of
+// the cluster-major copy, each row dotted with the queries whose mask bit is set.
+struct UnionParams {
+  const void* E_perm;              // v x d cluster-major copy
+  const int32_t* C2T;              // c x b
+  const void* H;                   // B x d
+  int64_t v, d, c, b;
+  int B;                           // <= 64
+  const unsigned long long* qmask; // per cluster: bit q set when query q takes it
+  const int32_t* cl_list;          // the clusters with a nonzero mask, each once, in any order
+  const int32_t* cl_count;         // their number (device)
+  int sample;
+  float tau;
+  uint64_t seed, step;
+  unsigned long long* best;        // B packed arg-maxima (zero between calls)
+  uint32_t* ticket;                // arrival count (zero between calls)
+  int32_t* out_tok;                // B
+  uint32_t* status;
+};
+bool union_supported(int elem, int64_t d, int64_t v, int64_t b, int B, int num_sms);
+cudaError_t launch_union_rows(const UnionParams& prm, int elem, int num_sms, cudaStream_t st);
 bool tc_supported(int elem, int64_t d, int B);
 cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms, cudaStream_t st);
 cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
-                               cudaStream_t st);
+                               cudaStream_t st, int32_t* list = nullptr, int32_t* count = nullptr);
 bool tc_int4_supported(int64_t d, int B, const void* scales);
 // INT4 Stage-1 keys on the tensor cores: out_keys[q][k] = Σ_j q4[k][j]·scale[k][j/32]·h_q[j] (or the
 // Gumbel key when sample != 0), dequantised to fp16 in shared memory (fh_tc.cu).

@@ -5,9 +5,10 @@
 // Used where the head is a dense contraction: the batched dense head (A = E, every row a candidate)
 // and batched FlashHead Stage 2 (A = the cluster-major copy of E; a row takes part for query q when
 // q's probe set holds the row's cluster — FlashHead notes, Module 1 and Figure 1, and Eq. 2/3 for the
-// decision).  Stage 2 lists the clusters some query selected and gathers them, 128 rows (whole
-// clusters) per tile, so every needed row is read once for all queries; the epilogue masks each
-// (row, query) pair by whether the query selected the row's cluster.
+// decision) at large batches.  Stage 2 lists the 128-row tiles that hold a cluster some query
+// selected and streams them, so every needed row is read once for all queries; the epilogue masks
+// each (row, query) pair by whether the query selected the row's cluster.  Stage-1 keys (A = C, or
+// the INT4 centroids dequantised in shared memory) use the same pipeline.
 //
 // One persistent CTA per SM, 8 warps with fixed roles:
 //   warp 0      TMA producer: per stage one K-block (64 columns) of H (Bpad rows) and of each A tile
@@ -135,10 +136,10 @@ constexpr int kTcMaxStages = 16;
 constexpr uint32_t kTcSmemMax = 226u * 1024u;
 
 // Dynamic shared memory of the kernel: `stages` stages of (H block, E blocks of the wave), the tile
-// rows (token, mask) and the wave's cluster ids, the sampling scratch, the barriers.
+// rows (token, mask), the sampling scratch, the barriers.
 struct TcLay {
   uint32_t h_bytes, e_bytes, stage_bytes;
-  uint32_t row_off, cl_off, gum_off, pair_off, bar_off, dyn;
+  uint32_t row_off, gum_off, pair_off, bar_off, dyn;
 };
 __host__ __device__ inline TcLay tc_layout(int B, int tile_rows, int wave, bool sample, int stages) {
   TcLay L;
@@ -146,8 +147,7 @@ __host__ __device__ inline TcLay tc_layout(int B, int tile_rows, int wave, bool 
   L.e_bytes = (uint32_t)tile_rows * 128u;
   L.stage_bytes = L.h_bytes + (uint32_t)wave * L.e_bytes;
   L.row_off = (uint32_t)stages * L.stage_bytes;
-  L.cl_off = L.row_off + (uint32_t)kTcRows * 12u;
-  L.gum_off = L.cl_off + (uint32_t)kTcWave * 16u * 4u;
+  L.gum_off = L.row_off + (uint32_t)kTcRows * 12u;
   L.pair_off = L.gum_off + (sample ? 4u * 32u * 32u * 4u : 0u);
   L.bar_off = L.pair_off + (sample ? 4u * 64u * 4u : 0u);
   const uint32_t end = L.bar_off + (uint32_t)(2 * kTcMaxStages + 8) * 8u;
@@ -170,7 +170,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const TcLay Lay = tc_layout(a.B, R, WT, SAMPLE, S);
   uint32_t* tok_s = reinterpret_cast<uint32_t*>(smem + Lay.row_off);                     // 128
   unsigned long long* msk_s = reinterpret_cast<unsigned long long*>(smem + Lay.row_off + 512u);  // 128
-  int32_t* wave_cl = reinterpret_cast<int32_t*>(smem + Lay.cl_off);  // kTcWave x gpt
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay.bar_off);
   uint64_t* empty = full + kTcMaxStages;
   uint64_t* tfull = empty + kTcMaxStages;  // [2] a wave's accumulators are final (MMA -> epilogue)
@@ -183,12 +182,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;
   const int KB = (int)((a.d + kTcKB - 1) / kTcKB);
-  // This CTA's tiles: bid, bid + G, ...  In gather mode tile t is the gpt clusters gpt*t .. gpt*t +
-  // gpt - 1 of the selected-cluster list (b rows each).
-  const int gpt = a.cl_list ? (int)(kTcRows / a.b) : 0;
-  const int n_cl = a.cl_list ? __ldg(a.cl_count) : 0;
-  // listed mode: the contiguous tiles some query takes, tile_list[0 .. *tile_count)
-  const int n_list = a.cl_list ? (n_cl + gpt - 1) / gpt : (a.tile_list ? __ldg(a.tile_count) : a.n_tiles);
+  // This CTA's tiles: bid, bid + G, ... of every tile, or in listed mode of the contiguous tiles some
+  // query takes, tile_list[0 .. *tile_count)
+  const int n_list = a.tile_list ? __ldg(a.tile_count) : a.n_tiles;
   const int my_tiles = n_list > (int)blockIdx.x ? (n_list - (int)blockIdx.x + G - 1) / G : 0;
   const int n_waves = (my_tiles + WT - 1) / WT;
   auto tile_at = [&](int j) {
@@ -225,21 +221,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int w = 0; w < n_waves && ok; ++w) {
       const int j0 = w * WT, nt = min(WT, my_tiles - j0);
-      if (gpt) {  // the wave's cluster ids, read once by the whole warp (no load in the issue loop)
-        for (int i = lane; i < nt * gpt; i += 32) {
-          const int slot = tile_at(j0 + i / gpt) * gpt + i % gpt;
-          wave_cl[i] = slot < n_cl ? __ldg(a.cl_list + slot) : -1;
-        }
-        __syncwarp();
-      }
       if (lane == 0) {
-        int tl[kTcWave], nc[kTcWave];
-        uint32_t bytes = Lay.h_bytes;  // H rows past B (up to Bpad) read as zeros
-        for (int j = 0; j < nt; ++j) {
-          tl[j] = tile_at(j0 + j);
-          nc[j] = gpt ? min(gpt, n_cl - tl[j] * gpt) : 0;
-          bytes += gpt ? (uint32_t)nc[j] * (uint32_t)a.b * 128u : Lay.e_bytes;
-        }
+        int tl[kTcWave];
+        for (int j = 0; j < nt; ++j) tl[j] = tile_at(j0 + j);
+        const uint32_t bytes = Lay.h_bytes + (uint32_t)nt * Lay.e_bytes;  // H rows past B read as zeros
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
           if (!tc_wait(&empty[s], (uint32_t)(((it / S) & 1) ^ 1), &abort_s, a.status)) {
@@ -249,21 +234,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           uint8_t* stg = smem + (size_t)s * Lay.stage_bytes;
           mbar_arrive_expect_tx(&full[s], bytes);
           tma_load_2d(stg, &tmH, kb * kTcKB, 0, &full[s]);
-          for (int j = 0; j < nt; ++j) {
-            uint8_t* dst = stg + Lay.h_bytes + (size_t)j * Lay.e_bytes;
-            if (gpt) {  // one box of b rows per listed cluster; the rows of absent ones stay unread
-              for (int i = 0; i < nc[j]; ++i)
-                tma_load_2d(dst + (size_t)i * a.b * 128u, &tmE, kb * kTcKB, wave_cl[j * gpt + i] * (int)a.b,
-                            &full[s]);
-            } else {
-              tma_load_2d(dst, &tmE, kb * kTcKB, tl[j] * R, &full[s]);
-            }
-          }
+          for (int j = 0; j < nt; ++j)
+            tma_load_2d(stg + Lay.h_bytes + (size_t)j * Lay.e_bytes, &tmE, kb * kTcKB, tl[j] * R, &full[s]);
         }
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      // the next wave rewrites the cluster ids only after lane 0 issued every load of this one
-      __syncwarp();
     }
     if (lane == 0) {
       // leave no copy in flight: the last loads have landed (at once when all went well)
@@ -323,21 +298,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = 0; j < nt; ++j) {
         const int t = tile_at(j0 + j);
         if constexpr (!KEYS) {  // the tile's rows: token and query mask (0: no query takes the row, or no row)
-          const int r = et;
-          int64_t row, cl;
-          bool valid;
-          if (a.cl_list) {
-            const int slot = t * gpt + r / (int)a.b;
-            valid = slot < n_cl;
-            cl = valid ? __ldg(a.cl_list + slot) : 0;
-            row = cl * a.b + r % (int)a.b;
-          } else {
-            row = (int64_t)t * kTcRows + r;
-            valid = row < a.rows;
-            cl = a.qmask ? row / a.b : 0;
-          }
-          tok_s[r] = valid ? (a.row_tok ? (uint32_t)__ldg(a.row_tok + row) : (uint32_t)row) : 0u;
-          msk_s[r] = valid ? (a.qmask ? __ldg(a.qmask + cl) : ~0ull) : 0ull;
+          const int64_t row = (int64_t)t * kTcRows + et;
+          const bool valid = row < a.rows;
+          const int64_t cl = a.qmask ? row / a.b : 0;
+          tok_s[et] = valid ? (a.row_tok ? (uint32_t)__ldg(a.row_tok + row) : (uint32_t)row) : 0u;
+          msk_s[et] = valid ? (a.qmask ? __ldg(a.qmask + cl) : ~0ull) : 0ull;
           group_sync();
         }
         const uint32_t tbase = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(acc * 256 + j * R);
@@ -483,32 +448,6 @@ __global__ void __launch_bounds__(1024) k_selected_tiles(const unsigned long lon
   if (threadIdx.x == 0) *count = base_s;
 }
 
-// The clusters some query takes (nonzero mask), in ascending order; one block.
-__global__ void __launch_bounds__(1024) k_selected_clusters(const unsigned long long* __restrict__ qmask,
-                                                            int64_t c, int32_t* list, int32_t* count) {
-  __shared__ int base_s;
-  __shared__ int wsum[32];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  if (threadIdx.x == 0) base_s = 0;
-  __syncthreads();
-  for (int64_t k0 = 0; k0 < c; k0 += blockDim.x) {
-    const int64_t k = k0 + threadIdx.x;
-    const bool act = k < c && qmask[k] != 0ull;
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, act);
-    if (lane == 0) wsum[wid] = __popc(bal);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
-      before += i < wid ? wsum[i] : 0;
-      total += wsum[i];
-    }
-    if (act) list[base_s + before + __popc(bal & ((1u << lane) - 1u))] = (int32_t)k;
-    __syncthreads();
-    if (threadIdx.x == 0) base_s += total;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) *count = base_s;
-}
 
 // ------------------------------------------------------------------ host side
 
@@ -554,7 +493,7 @@ cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, TcParams
   cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(kern), dyn);
   if (e != cudaSuccess) return e;
   // every SM when the tiles are listed on the device; otherwise no more CTAs than tiles
-  const int grid = (p.cl_list || p.tile_list || p.n_tiles >= num_sms) ? num_sms : p.n_tiles;
+  const int grid = (p.tile_list || p.n_tiles >= num_sms) ? num_sms : p.n_tiles;
   kern<<<grid, kTcThreads, dyn, st>>>(mE, mH, p);
   return cudaGetLastError();
 }
@@ -855,23 +794,16 @@ bool tc_supported(int elem, int64_t d, int B) {
 
 cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms, cudaStream_t st) {
   if (p.B < 1 || p.B > 64 || p.rows < 1 || (p.qmask && p.b < 1)) return cudaErrorInvalidValue;
-  if (p.out_keys && (p.qmask || p.cl_list)) return cudaErrorInvalidValue;
+  if (p.out_keys && p.qmask) return cudaErrorInvalidValue;
   // Stage-1 keys of few rows take 64-row tiles when that gives every SM at most one
   p.tile_rows = (p.out_keys && (p.rows + 63) / 64 <= num_sms) ? 64 : kTcRows;
   p.n_tiles = (int)((p.rows + p.tile_rows - 1) / p.tile_rows);
   uint32_t box = (uint32_t)p.tile_rows;
   if (p.tile_list) {  // the selected tiles, listed on the device (the kernel reads their count)
-    if (!p.qmask || p.cl_list) return cudaErrorInvalidValue;
+    if (!p.qmask) return cudaErrorInvalidValue;
     k_selected_tiles<<<1, 1024, 0, st>>>(p.qmask, p.rows, p.b, p.n_tiles, p.tile_list, p.tile_count);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-  }
-  if (p.cl_list) {  // the selected clusters, listed on the device (the kernel reads their count)
-    if (p.b < 8 || kTcRows % p.b != 0) return cudaErrorInvalidValue;  // whole 8-row swizzle atoms per box
-    k_selected_clusters<<<1, 1024, 0, st>>>(p.qmask, p.rows / p.b, p.cl_list, p.cl_count);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    box = (uint32_t)p.b;
   }
   CUtensorMap mE, mH;
   if (!make_map(&mE, A, p.d, p.rows, box) || !make_map(&mH, H, p.d, p.B, (uint32_t)((p.B + 15) / 16 * 16)))

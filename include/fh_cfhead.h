@@ -11,7 +11,8 @@
  *   - the columns of E are cut into T = d / w tiles of w consecutive columns; tile t has a codebook
  *     Cb[t] of K <= 16 entries of w fp32 values, and every token u one 4-bit code I[u][t] < K per tile;
  *   - per query h: LUT[t][j] = Cb[t][j]·h[t·w .. t·w + w) (fp32, in column order);
- *   - coarse score ŝ_u = Σ_t LUT[t][I[u][t]] (fp32, summed in tile order);
+ *   - coarse score ŝ_u = Σ_t LUT[t][I[u][t]] (fp32: four partial sums over the tiles t ≡ 0, 1, 2, 3
+ *     (mod 4), each in tile order, then (s0 + s1) + (s2 + s3));
  *   - candidates = the k tokens with the largest coarse scores, ordered (score desc, token id asc);
  *   - exact logits z_u = E[u]·h (fp32 accumulation of BF16 products) for the candidates, and the
  *     token = arg-max of z (greedy) or of z/τ + G(seed, step, q, FH_RNG_STAGE2, u) (sampling: a

@@ -1,12 +1,12 @@
 """Parity with the oracle at the full sizes the benchmark runs, in the kernels those sizes select.
 
 * Gemma-3-1B-shaped INT4 Stage 1 (v=262144, d=1152, c=16384, p=1024): batch 1 runs the persistent
-  kernel with 512 threads (more than 8192 clusters), batch 8 the INT4 tensor-core Stage 1 and the
-  per-query Stage 2, batch 32 the INT4 tensor-core Stage 1 and the tensor-core Stage 2.
+  kernel with 512 threads (more than 8192 clusters), batches 8 and 32 the INT4 tensor-core Stage 1
+  with the union Stage 2 (8) or the tensor-core Stage 2 (32).
 * The crowded boundary bin at c > 8192 (the 512-thread full-selection branch).
-* Llama-3.2-1B-shaped batches of 16 and 64 queries (d=2048: 32 K-blocks per tile) on the
-  tensor-core Stage 1 and Stage 2, greedy and sampling; the tensor-core Stage-1 keys element by
-  element.
+* Llama-3.2-1B-shaped batches of 16, 32 and 64 queries (d=2048: 32 K-blocks per tile) on the
+  tensor-core Stage 1 with the union Stage 2 (16) or the tensor-core Stage 2 (32, 64), greedy and
+  sampling; the tensor-core Stage-1 keys element by element.
 * The Qwen-3-0.6B-shaped Monte Carlo marginal (c=9496, p=512), which selects with 20 keys per
   thread, on likely targets (each query's dense top 8) with relative tolerances.
 
@@ -89,8 +89,8 @@ def test_llama_stage1_keys_tensor_core(fh, orc, llama_host, llama_index, B):
     assert np.abs(g - o).max() <= LOGIT_TOL
 
 
-@pytest.mark.parametrize("B", [16, 64])
-def test_llama_batched_greedy_tensor_core(fh, orc, llama_host, llama_index, B):
+@pytest.mark.parametrize("B", [16, 32, 64])
+def test_llama_batched_greedy(fh, orc, llama_host, llama_index, B):
     idx, H = llama_host
     n_set, n_tok = check_head(fh, orc, idx, H, idx.cfg.p, batch=B, debug="sel", I=llama_index)
     # most queries must be decided (same set as the oracle, top-1 margin > 4e-3)
@@ -102,16 +102,17 @@ def test_llama_batched_greedy_tensor_core(fh, orc, llama_host, llama_index, B):
     assert np.array_equal(tok[d], o["tok"][d])
 
 
-@pytest.mark.parametrize("B", [16, 64])
-def test_llama_batched_sampling_tensor_core(fh, orc, llama_host, llama_index, B):
+@pytest.mark.parametrize("B", [16, 32, 64])
+def test_llama_batched_sampling(fh, orc, llama_host, llama_index, B):
     idx, H = llama_host
     check_head(fh, orc, idx, H, idx.cfg.p, batch=B, sample=True, tau=0.8, seed=synth.SAMPLE_SEED,
                step=B, debug="sel", I=llama_index)
 
 
 def test_llama_batch_tokens_match_batch1(fh, llama_host, llama_index):
-    """The tensor-core batch and the persistent batch-1 kernel sum the same logits in different
-    orders; their tokens agree wherever fp32 rounding cannot decide between two candidates."""
+    """The union Stage 2 of a 16-query batch and the persistent batch-1 kernel sum the same logits
+    in different orders; their tokens agree wherever fp32 rounding cannot decide between two
+    candidates."""
     idx, H = llama_host
     Hd = dev(H[:16], "bf16")
     tb = fh.head_greedy(llama_index, Hd, idx.cfg.p).cpu().numpy()

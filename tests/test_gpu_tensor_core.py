@@ -1,7 +1,8 @@
 """Parity of the tensor-core (tcgen05) path with the fp64 oracle.
 
 Batches of 2..64 queries on a BF16 index take the tensor-core kernel for the dense head; FlashHead
-takes it from 12 queries on when no debug outputs are requested.  Sizes span several 128-row tiles with a
+takes it for its Stage-1 keys from 12 queries on and for its Stage 2 above 16 queries (below, the
+union of the probe sets is streamed on the CUDA cores) when no per-candidate outputs are requested.  Sizes span several 128-row tiles with a
 ragged tail (v = 32064), batches that are not a multiple of the 16-query MMA width, and a d that is
 not a multiple of the 64-element K-block.  Logits are compared element by element (|Δ| <= 2e-3);
 token ids must be identical wherever the oracle's margins decide them (parity.MARGIN)."""
@@ -77,9 +78,9 @@ def small(fh):
 @pytest.mark.parametrize("sample", [False, True])
 def test_flashhead_batched_without_debug(fh, orc, small, B, sample):
     """Tokens equal the oracle's wherever its set and token margins decide them; every other token
-    comes from a cluster the oracle selected or one within the margin of its threshold.  B = 4 and 8
-    run the per-query CUDA-core Stage 2, B = 12 gathers the selected clusters into tensor-core tiles,
-    B >= 16 streams the tiles that hold a selected cluster."""
+    comes from a cluster the oracle selected or one within the margin of its threshold.  B = 4 … 16
+    stream the union of the probe sets on the CUDA cores (tensor-core Stage-1 keys from 12 on),
+    B = 33 and 64 stream the tensor-core tiles that hold a selected cluster."""
     idx, H, I = small
     cfg = idx.cfg
     Hd = dev(H[:B], "bf16")
@@ -101,12 +102,12 @@ def test_flashhead_batched_without_debug(fh, orc, small, B, sample):
 
 
 def test_flashhead_batched_matches_cuda_core_path(fh, mid, mid_index):
-    """The tensor-core Stage 2 (no debug outputs) and the per-query CUDA-core Stage 2 (taken when
-    debug outputs are requested) select the same sets and agree on every token whose logit margin
-    exceeds the fp32 accumulation-order difference."""
+    """The tensor-core Stage 2 (no debug outputs, 40 queries) and the per-query CUDA-core Stage 2
+    (taken when debug outputs are requested) select the same sets and agree on every token whose
+    logit margin exceeds the fp32 accumulation-order difference."""
     idx, H = mid
     cfg = idx.cfg
-    B = 24
+    B = 40
     Hd = dev(H[:B], "bf16")
     tc = fh.head_greedy(mid_index, Hd, cfg.p).cpu().numpy()
     P = cfg.p * cfg.b

@@ -606,18 +606,26 @@ def run_reference(args):
 
 
 def ncu_case(args):
-    """A few batch-1 greedy calls of the Llama-shaped head on a single index copy, nothing timed."""
+    """A few calls of one head on a single index copy, nothing timed: the Llama-shaped greedy, sampling
+    or dense head, the Gemma-shaped INT4 greedy head (`int4`) or the Llama-shaped coarse-fine head
+    (`cf`), at --batch queries."""
     from clustered_retrieval_classification_b200 import flashhead as F
     F.load()
-    cfg = synth.CONFIGS["llama"]
+    cfg = synth.CONFIGS["gemma" if args.ncu_what == "int4" else "llama"]
     idx = synth.make_index(cfg)
-    R = Replicated(F, idx, replicas=1)
     Hd = F.device_array(synth.make_queries(cfg, 128), "bf16")
     B = args.batch
-    if args.ncu_what == "dense":
-        step = dense_step(F, R, Hd, B)
+    if args.ncu_what == "cf":
+        cb, words = synth.cf_index(idx.E, "bf16")
+        CI = F.cf_index_from_host(idx.E, cb, words)
+
+        def step(k):
+            F.cf_head(CI, Hd[:B], synth.CF_TOPK)
+    elif args.ncu_what == "dense":
+        step = dense_step(F, Replicated(F, idx, replicas=1), Hd, B)
     else:
-        step = head_step(F, R, Hd, B, cfg.p, mode=args.ncu_what)
+        R = Replicated(F, idx, int4=args.ncu_what == "int4", replicas=1)
+        step = head_step(F, R, Hd, B, cfg.p, mode="sample" if args.ncu_what == "sample" else "greedy")
     for k in range(min(args.steps, 64)):
         step(k)
     torch.cuda.synchronize()
@@ -716,7 +724,7 @@ def main():
     ap.add_argument("--ncu-case", action="store_true",
                     help="run --steps untimed calls on one index copy (about 1.1 GB on the device) and "
                          "exit: the case the committed ncu captures use")
-    ap.add_argument("--ncu-what", default="greedy", choices=["greedy", "dense", "sample"],
+    ap.add_argument("--ncu-what", default="greedy", choices=["greedy", "dense", "sample", "int4", "cf"],
                     help="with --ncu-case: which head (at --batch queries) to call")
     ap.add_argument("--pc-sweep", action="store_true",
                     help="time the batch-1 greedy head of the Llama-shaped vocabulary at "

@@ -122,16 +122,16 @@ uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<
 uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
 
 // The tensor-core path: BF16 E (and, for FlashHead, its cluster-major copy), batches up to 64.  The
-// dense head takes it from 2 queries on; FlashHead's Stage 1 from kTcMinBatchHead (below it the
-// CUDA-core kernels read the centroids as fast), its Stage 2 above kUnionMaxBatch (measured at the
-// Llama-3.2-1B shape: the union kernel 70 / 103 / 124 µs a call at 4 / 12 / 16 queries against
+// dense head and FlashHead's Stage-1 keys take it from 2 queries on (measured at the Llama-3.2-1B
+// shape: Stage-1 keys 16 µs at 16 queries, the CUDA-core kernel 24.5 µs at 4); FlashHead's Stage 2
+// above kUnionMaxBatch (the union kernel 70 / 103 / 124 µs a call at 4 / 12 / 16 queries against
 // 73 / 145 / 148 µs before it; at 24 and 32 queries its 8-warp form, all that fits beside the query
 // vectors, took 237 and 290 µs against the tensor cores' 155 and 158 µs).
 constexpr int kTcMinBatchDense = 2;
-#ifndef FH_TC_MIN_BATCH_HEAD
-#define FH_TC_MIN_BATCH_HEAD 12
+#ifndef FH_TC_MIN_BATCH_STAGE1
+#define FH_TC_MIN_BATCH_STAGE1 2
 #endif
-constexpr int kTcMinBatchHead = FH_TC_MIN_BATCH_HEAD;
+constexpr int kTcMinBatchStage1 = FH_TC_MIN_BATCH_STAGE1;
 #ifndef FH_UNION_MAX_BATCH
 #define FH_UNION_MAX_BATCH 16
 #endif
@@ -249,8 +249,8 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   const int elem = D.dtype == FH_BF16 ? fh::kBF16 : fh::kF32;
   const bool uni = B > 1 && B <= kUnionMaxBatch && !per_cand && D.E_perm != nullptr &&
                    fh::union_supported(elem, D.d, D.v, D.b, B, idx->num_sms);
-  const bool tc = !uni && tc_eligible(idx, B, kTcMinBatchHead) && !per_cand && D.E_perm != nullptr;
-  if ((tc || uni) && tc_eligible(idx, B, kTcMinBatchHead) && s1fmt(idx) == FH_STAGE1_DENSE) {
+  const bool tc = !uni && tc_eligible(idx, B, kTcMinBatchDense) && !per_cand && D.E_perm != nullptr;
+  if ((tc || uni) && tc_eligible(idx, B, kTcMinBatchStage1) && s1fmt(idx) == FH_STAGE1_DENSE) {
     // Stage 1 on the tensor cores too: keys[q][k] = C[k]·h_q (+ the Gumbel term when sampling)
     fh::TcParams tp = {};
     tp.rows = D.c;
@@ -676,7 +676,7 @@ fh_status fh_stage1_scores(const fh_index* idx, const void* H, int B, float* out
   if (!out_s) return fail(FH_ERR_ARG, "out_s is NULL");
   if ((r = check_ws(ws, ws_bytes, kHeaderBytes)) != FH_OK) return r;
   cudaError_t e;
-  if (tc_eligible(idx, B, kTcMinBatchHead) && s1fmt(idx) == FH_STAGE1_DENSE) {
+  if (tc_eligible(idx, B, kTcMinBatchStage1) && s1fmt(idx) == FH_STAGE1_DENSE) {
     // the kernel the fused head runs at these batches: keys mode of the tensor-core head
     fh::TcParams tp = {};
     tp.rows = idx->desc.c;

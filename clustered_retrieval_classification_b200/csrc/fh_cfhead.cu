@@ -92,6 +92,10 @@ struct CfParams {
 };
 
 // ------------------------------------------------------------------ look-up tables
+// LUT[q][t][j] at (q·T + t)·16 + j: every tile takes 16 entries whatever K is (entries past K are
+// zero), so the score loop addresses a tile's entries with compile-time offsets.
+constexpr int kCfLutStride = FH_CF_MAX_K;
+static_assert(kCfLutStride == 16, "4-bit codes index 16 entries");
 
 __global__ void __launch_bounds__(kCfThreads) k_cf_lut(const CfParams p) {
   const int q = blockIdx.y;
@@ -103,13 +107,15 @@ __global__ void __launch_bounds__(kCfThreads) k_cf_lut(const CfParams p) {
       p.bnd_cnt[q] = 0u;
     }
   }
-  if (i >= p.T * p.K) return;
-  const int t = i / p.K;
-  const float* c = p.cb + (size_t)i * p.w;
-  const uint16_t* h = p.H + (size_t)q * p.d + (size_t)t * p.w;
+  if (i >= p.T * kCfLutStride) return;
+  const int t = i / kCfLutStride, j = i % kCfLutStride;  // tile t, entry j (zero past K)
   float acc = 0.0f;
-  for (int e = 0; e < p.w; ++e) acc = fmaf(c[e], __uint_as_float((uint32_t)h[e] << 16), acc);
-  p.lut[(size_t)q * p.T * p.K + i] = acc;
+  if (j < p.K) {
+    const float* c = p.cb + ((size_t)t * p.K + j) * p.w;
+    const uint16_t* h = p.H + (size_t)q * p.d + (size_t)t * p.w;
+    for (int e = 0; e < p.w; ++e) acc = fmaf(c[e], __uint_as_float((uint32_t)h[e] << 16), acc);
+  }
+  p.lut[(size_t)q * p.T * kCfLutStride + i] = acc;
 }
 
 // ------------------------------------------------------------------ coarse scores
@@ -117,11 +123,11 @@ __global__ void __launch_bounds__(kCfThreads) k_cf_lut(const CfParams p) {
 constexpr int kCfWordsInFlight = 16;  // code words per batch; two batches are in flight
 
 __global__ void __launch_bounds__(kCfThreads) k_cf_coarse(const CfParams p) {
-  extern __shared__ __align__(16) float lut_s[];  // T x K, then kCfBins histogram words
+  extern __shared__ __align__(16) float lut_s[];  // T x 16, then kCfBins histogram words
   __shared__ float red_s[kCfThreads / 32];
   __shared__ __align__(8) uint64_t lut_bar;
   const int q = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int TK = p.T * p.K;
+  const int TK = p.T * kCfLutStride;
   const int G8 = p.T / 8;
   const int64_t v = p.v;
   const int64_t u = (int64_t)blockIdx.x * kCfThreads + tid;  // one token per thread
@@ -155,7 +161,9 @@ __global__ void __launch_bounds__(kCfThreads) k_cf_coarse(const CfParams p) {
   float part = 0.0f;
   for (int t = tid; t < p.T; t += kCfThreads) {
     float m = 0.0f;
-    for (int j = 0; j < p.K; ++j) m = fmaxf(m, fabsf(lut_s[t * p.K + j]));
+    // entries in rotated order: the lanes of a warp read different banks
+    for (int j = 0, jr = t % p.K; j < p.K; ++j, jr = (jr + 1 == p.K) ? 0 : jr + 1)
+      m = fmaxf(m, fabsf(lut_s[t * kCfLutStride + jr]));
     part += m;
   }
   part = warp_sum(part);
@@ -179,16 +187,16 @@ __global__ void __launch_bounds__(kCfThreads) k_cf_coarse(const CfParams p) {
 #pragma unroll
       for (int g = 0; g < kCfWordsInFlight; ++g) {
         if (g0 + g < G8) {
-          const float* lt = lut_s + (size_t)(8 * (g0 + g)) * p.K;
+          const float* lt = lut_s + (size_t)(8 * (g0 + g)) * kCfLutStride;
           const uint32_t x = w[g];
-          a0 += lt[0 * p.K + (x & 15u)];
-          a1 += lt[1 * p.K + ((x >> 4) & 15u)];
-          a2 += lt[2 * p.K + ((x >> 8) & 15u)];
-          a3 += lt[3 * p.K + ((x >> 12) & 15u)];
-          a0 += lt[4 * p.K + ((x >> 16) & 15u)];
-          a1 += lt[5 * p.K + ((x >> 20) & 15u)];
-          a2 += lt[6 * p.K + ((x >> 24) & 15u)];
-          a3 += lt[7 * p.K + (x >> 28)];
+          a0 += lt[0 * kCfLutStride + (x & 15u)];
+          a1 += lt[1 * kCfLutStride + ((x >> 4) & 15u)];
+          a2 += lt[2 * kCfLutStride + ((x >> 8) & 15u)];
+          a3 += lt[3 * kCfLutStride + ((x >> 12) & 15u)];
+          a0 += lt[4 * kCfLutStride + ((x >> 16) & 15u)];
+          a1 += lt[5 * kCfLutStride + ((x >> 20) & 15u)];
+          a2 += lt[6 * kCfLutStride + ((x >> 24) & 15u)];
+          a3 += lt[7 * kCfLutStride + (x >> 28)];
         }
       }
     };
@@ -315,23 +323,47 @@ constexpr int kCfResolveThreads = 1024;
 
 // In the block's shared histogram, the digit d where the count from the top (desc) or from the bottom
 // (asc) first reaches `target`; returns d and the count strictly before it in that direction.
+// The first digit, in the given order, at which the running count reaches `target`, and the count
+// before it.  Warp 0: lane l sums the 8 digits at ordered positions 8l .. 8l+7, a warp scan finds the
+// lane where the running count crosses `target`, and that lane walks its 8 digits.
 __device__ __forceinline__ void cf_pick_digit(const uint32_t* h256, uint32_t target, bool desc,
                                               uint32_t* digit, uint32_t* before) {
-  if (threadIdx.x == 0) {
-    uint32_t cum = 0;
-    for (int i = 0; i < 256; ++i) {
-      const int d = desc ? 255 - i : i;
-      if (cum + h256[d] >= target) {
-        *digit = (uint32_t)d;
-        *before = cum;
-        break;
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    uint32_t c[8], sum = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int pos = 8 * lane + i;
+      c[i] = h256[desc ? 255 - pos : pos];
+      sum += c[i];
+    }
+    uint32_t incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t excl = incl - sum;
+    if (excl < target && target <= incl) {
+      uint32_t cum = excl;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (cum + c[i] >= target) {
+          const int pos = 8 * lane + i;
+          *digit = (uint32_t)(desc ? 255 - pos : pos);
+          *before = cum;
+          break;
+        }
+        cum += c[i];
       }
-      cum += h256[d];
     }
   }
 }
 
+constexpr uint32_t kCfResolveStage = 12288;  // boundary entries staged in shared memory (96 KiB)
+
 __global__ void __launch_bounds__(kCfResolveThreads) k_cf_resolve(const CfParams p) {
+  extern __shared__ __align__(16) unsigned long long bl_s[];  // kCfResolveStage entries
   __shared__ uint32_t h256[256];
   __shared__ uint32_t digit_s, before_s;
   const int q = blockIdx.y, tid = threadIdx.x;
@@ -341,7 +373,13 @@ __global__ void __launch_bounds__(kCfResolveThreads) k_cf_resolve(const CfParams
   const uint32_t m = p.bnd_cnt[q];
   if (have >= k || m == 0u) return;
   uint32_t need = k - have;
+  // the boundary list, read once into shared memory when it fits (the passes below re-read it)
   const unsigned long long* bl = p.blist + (size_t)q * p.v;
+  if (m <= kCfResolveStage) {
+    for (uint32_t i = tid; i < m; i += kCfResolveThreads) bl_s[i] = bl[i];
+    bl = bl_s;
+    __syncthreads();
+  }
   // 1. the exact threshold image T: 8-bit radix passes from the top of the score images
   uint32_t prefix = 0u, mask = 0u;
   for (int shift = 24; shift >= 0; shift -= 8) {
@@ -449,7 +487,7 @@ CfLayout cf_layout(const fh_cf_index* idx, int B, int k) {
     off = up(off + bytes);
     return at;
   };
-  L.lut = take((size_t)B * T * D.K * 4);
+  L.lut = take((size_t)B * T * kCfLutStride * 4);
   L.scale = take((size_t)B * 4);
   L.hist = take((size_t)B * kCfBins * 4);
   L.coarse = take((size_t)B * D.v * 4);
@@ -516,7 +554,7 @@ int cf_blocks(const fh_cf_index* idx, int B, int64_t work_items) {
 
 // The look-up tables and the coarse scores (with their histogram) of every query.
 cudaError_t cf_launch_coarse(const fh_cf_index* idx, const CfParams& p, cudaStream_t st) {
-  const int TK = p.T * p.K;
+  const int TK = p.T * kCfLutStride;
   k_cf_lut<<<dim3((TK + kCfThreads - 1) / kCfThreads, p.B), kCfThreads, 0, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -596,7 +634,9 @@ fh_status fh_cf_head(const fh_cf_index* idx, const void* H, int B, int k, int sa
   if (e != cudaSuccess) return cuda_err(e, "coarse-score launch");
   k_cf_compact<<<dim3(cf_blocks(idx, B, p.v), B), kCfThreads, 0, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_err(e, "compaction launch");
-  k_cf_resolve<<<dim3(1, B), kCfResolveThreads, 0, st>>>(p);
+  if ((e = set_smem_attr(reinterpret_cast<const void*>(k_cf_resolve), kCfResolveStage * 8u)) != cudaSuccess)
+    return cuda_err(e, "resolve attribute");
+  k_cf_resolve<<<dim3(1, B), kCfResolveThreads, kCfResolveStage * 8u, st>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_err(e, "boundary launch");
   if (dbg_coarse &&
       (e = cudaMemcpyAsync(dbg_coarse, p.coarse, (size_t)B * p.v * 4, cudaMemcpyDeviceToDevice, st)) != cudaSuccess)

@@ -209,8 +209,9 @@ fh_status fh_dense_head(const fh_index* idx, const void* H, int B, int sample, f
    run the same device code. */
 
 /* Stage-1 scores s = C·h_q (FlashHead notes, Figure 1 Stage 1), fp32.  out_s: device, B x c.
-   Runs the kernel the fused heads run at batch B: BF16 batches of 12 or more on the tensor cores,
-   the CUDA-core Stage-1 kernel otherwise. */
+   Runs the kernel the fused heads run at batch B: batches of 2 or more on the tensor cores (BF16
+   centroids directly, INT4 centroids dequantised to fp16 in shared memory), the CUDA-core Stage-1
+   kernel at B = 1 and for fp32 indexes. */
 fh_status fh_stage1_scores(const fh_index* idx, const void* H, int B, float* out_s,
                            void* ws, size_t ws_bytes, fh_stream stream);
 

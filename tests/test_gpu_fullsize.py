@@ -81,7 +81,7 @@ def test_crowded_boundary_bin_512_threads(fh, orc, perturb):
 # ----------------------------------------------------------------------------- Llama batches
 
 
-@pytest.mark.parametrize("B", [16, 64])
+@pytest.mark.parametrize("B", [2, 16, 64])
 def test_llama_stage1_keys_tensor_core(fh, orc, llama_host, llama_index, B):
     idx, H = llama_host
     g = fh.stage1_scores(llama_index, dev(H[:B], "bf16")).cpu().numpy()

@@ -98,13 +98,16 @@ def test_select_bit_exact(fh, orc, name, keys, p):
 
 
 def test_stage1_scores(fh, orc, tiny, mid):
+    """fp32 (tiny): the CUDA-core kernel at every batch; BF16 (mid): the CUDA-core kernel at B = 1,
+    the tensor cores from B = 2 (partial 16-query blocks at 2 and 5)."""
     for idx, H in (tiny, mid):
         cfg = idx.cfg
         I = load(fh, idx)
-        Hq = H[:5]
-        g = fh.stage1_scores(I, dev(Hq, cfg.dtype)).cpu().numpy()
-        o = orc.stage1_scores(idx.C, cfg.dtype, Hq, cfg.c, cfg.d)
-        assert np.abs(g - o).max() <= LOGIT_TOL
+        for B in (1, 2, 5):
+            Hq = H[:B]
+            g = fh.stage1_scores(I, dev(Hq, cfg.dtype)).cpu().numpy()
+            o = orc.stage1_scores(idx.C, cfg.dtype, Hq, cfg.c, cfg.d)
+            assert np.abs(g - o).max() <= LOGIT_TOL
 
 
 @pytest.mark.parametrize("B", [1, 3, 8])

@@ -389,7 +389,19 @@ def sweep(F, T, R, cfg, idx, Hd, Hh, args, peak):
     g = F.head_greedy(R[0], Hd[:64], cfg.p).cpu().numpy()
     d = F.dense_head(R[0], Hd[:64]).cpu().numpy()
     out["agreement_flashhead_vs_dense_top1"] = float(np.mean(g == d))
+    # the p part of the p/c trade-off (FlashHead summary, Table 7) on this index, batch 1; the
+    # c part needs other indexes: --pc-sweep
+    pc = {}
+    for p in (128, 256, 512):
+        t, n, _ = T.b2b(head_step(F, R, Hd, 1, p), K, W, repeats=3)
+        us = 1e3 * statistics.median(t) / n
+        by = costmodel.head_bytes(cfg.v, cfg.d, cfg.c, p, 1, p, 2)
+        pc[f"c{cfg.c}_p{p}"] = {"us_per_call": us, "bytes": by, "frac": by / (us * 1e-6) / 1e9 / peak}
+    out["pc_tradeoff_batch1"] = pc
     del R
+    torch.cuda.empty_cache()
+    # the index builder on this embedding matrix: one iteration from seeded initial tokens
+    out["kmeans_llama"] = kmeans_row(F, cfg, idx)
     torch.cuda.empty_cache()
     # Gemma-shaped INT4 Stage 1
     gcfg = synth.CONFIGS["gemma"]
@@ -607,15 +619,22 @@ def run_reference(args):
 
 def ncu_case(args):
     """A few calls of one head on a single index copy, nothing timed: the Llama-shaped greedy, sampling
-    or dense head, the Gemma-shaped INT4 greedy head (`int4`) or the Llama-shaped coarse-fine head
-    (`cf`), at --batch queries."""
+    or dense head, the Gemma-shaped INT4 greedy head (`int4`), the Llama-shaped coarse-fine head
+    (`cf`) or the Qwen-shaped Monte Carlo marginal (`mc`), at --batch queries."""
     from clustered_retrieval_classification_b200 import flashhead as F
     F.load()
-    cfg = synth.CONFIGS["gemma" if args.ncu_what == "int4" else "llama"]
+    cfg = synth.CONFIGS[{"int4": "gemma", "mc": "qwen"}.get(args.ncu_what, "llama")]
     idx = synth.make_index(cfg)
     Hd = F.device_array(synth.make_queries(cfg, 128), "bf16")
     B = args.batch
-    if args.ncu_what == "cf":
+    if args.ncu_what == "mc":  # the Monte Carlo marginal of 8 targets per query, 1000 draws
+        QI = F.index_from_host(idx.E, idx.C, idx.C2T, "bf16", cluster_major=False)
+        tg = F.device_array(synth.make_targets(cfg.v, B, 8), "i32")
+        ws = QI.workspace(F.FH_OP_MC, B, cfg.p, 8, 1000)
+
+        def step(k):
+            F.mc_token_prob(QI, Hd[:B], tg, cfg.p, 1.0, 1000, synth.MC_SEED, ws=ws)
+    elif args.ncu_what == "cf":
         cb, words = synth.cf_index(idx.E, "bf16")
         CI = F.cf_index_from_host(idx.E, cb, words)
 
@@ -675,6 +694,28 @@ def pc_sweep(args):
     return 0
 
 
+def kmeans_row(F, cfg, idx, iters=1):
+    """One timed run of the index builder (equal-size spherical k-means) on the embeddings of `idx`
+    into cfg.c clusters, with the two validity checks of its result."""
+    v, c, b = cfg.v, cfg.c, cfg.b
+    E = F.device_array(idx.E, cfg.dtype)
+    init = F.device_array(synth.init_tokens(v, c), "i32")
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    r = F.kmeans_build(E, c, init, iters=iters, eps=1e-4)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    labels = r["labels"].cpu().numpy()
+    C2T = r["C2T"].cpu().numpy()
+    return {"iters": r["iters"], "rounds": r["rounds"], "ms_total": ms,
+            "ms_per_iter": ms / max(r["iters"], 1),
+            "similarity_tflop_per_iter": 2.0 * v * c * cfg.d / 1e12,
+            "objective": r["objective"].cpu().numpy().tolist(),
+            "equal_size": bool(np.all(np.bincount(labels, minlength=c) == b)),
+            "c2t_is_permutation": bool(np.array_equal(np.sort(C2T.ravel()), np.arange(v)))}
+
+
 def kmeans_bench(args):
     """The index builder (equal-size spherical k-means, FlashHead notes Module 1) on the
     Llama-shaped embedding matrix (v = 128256, d = 2048, BF16) into c = 8016 clusters of 16:
@@ -686,27 +727,9 @@ def kmeans_bench(args):
     from clustered_retrieval_classification_b200 import flashhead as F
     F.load()
     cfg = synth.CONFIGS["llama"]
-    idx = synth.make_index(cfg)
-    v, d, c, b = cfg.v, cfg.d, cfg.c, cfg.b
-    E = F.device_array(idx.E, "bf16")
-    init = F.device_array(synth.init_tokens(v, c), "i32")
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record()
-    r = F.kmeans_build(E, c, init, iters=args.kmeans_iters, eps=1e-4)
-    t1.record()
-    torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1)
-    labels = r["labels"].cpu().numpy()
-    C2T = r["C2T"].cpu().numpy()
-    it = max(r["iters"], 1)
-    print(json.dumps({"kmeans": {
-        "workload": "llama-3.2-1b-shaped embeddings v=128256 d=2048 bf16, c=8016 (b=16)",
-        "iters": r["iters"], "rounds": r["rounds"], "ms_total": ms, "ms_per_iter": ms / it,
-        "similarity_tflop_per_iter": 2.0 * v * c * d / 1e12,
-        "objective": r["objective"].cpu().numpy().tolist(),
-        "equal_size": bool(np.all(np.bincount(labels, minlength=c) == b)),
-        "c2t_is_permutation": bool(np.array_equal(np.sort(C2T.ravel()), np.arange(v)))}}),
-        flush=True)
+    row = kmeans_row(F, cfg, synth.make_index(cfg), iters=args.kmeans_iters)
+    row = {"workload": "llama-3.2-1b-shaped embeddings v=128256 d=2048 bf16, c=8016 (b=16)", **row}
+    print(json.dumps({"kmeans": row}), flush=True)
     return 0
 
 
@@ -724,7 +747,7 @@ def main():
     ap.add_argument("--ncu-case", action="store_true",
                     help="run --steps untimed calls on one index copy (about 1.1 GB on the device) and "
                          "exit: the case the committed ncu captures use")
-    ap.add_argument("--ncu-what", default="greedy", choices=["greedy", "dense", "sample", "int4", "cf"],
+    ap.add_argument("--ncu-what", default="greedy", choices=["greedy", "dense", "sample", "int4", "cf", "mc"],
                     help="with --ncu-case: which head (at --batch queries) to call")
     ap.add_argument("--pc-sweep", action="store_true",
                     help="time the batch-1 greedy head of the Llama-shaped vocabulary at "

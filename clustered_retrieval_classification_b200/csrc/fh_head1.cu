@@ -382,13 +382,24 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   if (lane == 0) red_s[warp] = hsq;
   float hreg[INT4_MCH ? INT4_MCH : 1][INT4_MCH ? 32 : 1];
   if constexpr (INT4_MCH > 0) {
-    const uint16_t* Hs = reinterpret_cast<const uint16_t*>(hs);
+    // lane l keeps the 32 columns of its groups l, l + 32, ...: four 16-byte loads per group (lanes
+    // 64 bytes apart: 4-way bank conflicts, where 2-byte loads at that stride were 16-way)
+    const uint32_t hs_a = smem_addr(hs);
 #pragma unroll
     for (int m = 0; m < INT4_MCH; ++m) {
       const int ch = lane + 32 * m;
 #pragma unroll
-      for (int e = 0; e < 32; ++e)
-        hreg[m][e] = (ch < nch4) ? __uint_as_float((uint32_t)Hs[32 * ch + e] << 16) : 0.0f;
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = ch < nch4 ? lds_v4(hs_a + 64u * (uint32_t)ch + 16u * (uint32_t)i) : make_uint4(0u, 0u, 0u, 0u);
+        hreg[m][8 * i + 0] = bf16_lo(v.x);
+        hreg[m][8 * i + 1] = bf16_hi(v.x);
+        hreg[m][8 * i + 2] = bf16_lo(v.y);
+        hreg[m][8 * i + 3] = bf16_hi(v.y);
+        hreg[m][8 * i + 4] = bf16_lo(v.z);
+        hreg[m][8 * i + 5] = bf16_hi(v.z);
+        hreg[m][8 * i + 6] = bf16_lo(v.w);
+        hreg[m][8 * i + 7] = bf16_hi(v.w);
+      }
     }
   }
   __syncthreads();

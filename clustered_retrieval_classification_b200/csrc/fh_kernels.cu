@@ -114,13 +114,22 @@ __global__ void __launch_bounds__(kThreads) k_stage1_int4(const Stage1Params prm
   for (int64_t i = tid; i < (hi - lo) * nch; i += kThreads) sc_s[i] = prm.scales[lo * nch + i];
   // this lane's slice of h
   float hreg[MCH][32];
-  const uint16_t* H = static_cast<const uint16_t*>(prm.H) + (size_t)q * d;
+  const uint4* H = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(prm.H) + (size_t)q * d);
 #pragma unroll
   for (int m = 0; m < MCH; ++m) {
     const int ch = lane + 32 * m;
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      hreg[m][e] = (ch < nch) ? __uint_as_float((uint32_t)H[32 * ch + e] << 16) : 0.0f;
+    for (int i = 0; i < 4; ++i) {  // the group's 32 columns: four 16-byte loads
+      const uint4 v = (ch < nch) ? __ldg(H + 4 * ch + i) : make_uint4(0u, 0u, 0u, 0u);
+      hreg[m][8 * i + 0] = bf16_lo(v.x);
+      hreg[m][8 * i + 1] = bf16_hi(v.x);
+      hreg[m][8 * i + 2] = bf16_lo(v.y);
+      hreg[m][8 * i + 3] = bf16_hi(v.y);
+      hreg[m][8 * i + 4] = bf16_lo(v.z);
+      hreg[m][8 * i + 5] = bf16_hi(v.z);
+      hreg[m][8 * i + 6] = bf16_lo(v.w);
+      hreg[m][8 * i + 7] = bf16_hi(v.w);
+    }
   }
   __syncthreads();
 

@@ -133,7 +133,7 @@ __device__ __forceinline__ bool warp_stream_rows(int64_t first, int64_t hi, int 
 // A nibble n decodes to q = (n ^ 8) - 8 through the float pattern 0x4B000000 | (n ^ 8) = 2^23 + (n ^ 8).
 __device__ __forceinline__ float int4_group_dot(const uint4 w, const float* hg) {
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};
-  float acc = 0.0f;
+  float acc_e = 0.0f, acc_o = 0.0f;  // even and odd columns: two FMA chains, added at the end
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const uint32_t even = (words[i] & 0x0F0F0F0Fu) ^ 0x08080808u;         // columns 8i + 0,2,4,6
@@ -142,11 +142,11 @@ __device__ __forceinline__ float int4_group_dot(const uint4 w, const float* hg) 
     for (int j = 0; j < 4; ++j) {
       const float qe = __uint_as_float(__byte_perm(even, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
       const float qo = __uint_as_float(__byte_perm(odd, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
-      acc = fmaf(qe, hg[8 * i + 2 * j], acc);
-      acc = fmaf(qo, hg[8 * i + 2 * j + 1], acc);
+      acc_e = fmaf(qe, hg[8 * i + 2 * j], acc_e);
+      acc_o = fmaf(qo, hg[8 * i + 2 * j + 1], acc_o);
     }
   }
-  return acc;
+  return acc_e + acc_o;
 }
 
 // The 32 values of one INT4 group (columns 0..31, low nibble = even column), decoded exactly.

@@ -39,8 +39,9 @@ constexpr size_t kHeaderBytes = 1024 + 4096;  // control words, then the score h
 constexpr size_t kGenOffset = 536;             // batch-1 head: tag of the last completed call
 constexpr size_t kTcTicketOffset = 544;        // tensor-core head: arrival ticket (zero between calls)
 constexpr size_t kKeysReadyOffset = 552;       // batch-1 head: arrivals before its full selection
-constexpr size_t kArriveOffset = 556;          // batch-1 head: arrivals at its final reduction
+constexpr size_t kArriveOffset = 556;          // batch-1 head: blocks done (zero between calls)
 constexpr size_t kUnionTicketOffset = 560;     // batched union Stage 2: arrival ticket (zero between calls)
+constexpr size_t kBestOffset = 568;            // batch-1 head: the call's packed maximum (zero between calls)
 constexpr size_t kAlign = 256;
 
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -49,7 +50,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 // Workspace regions of one call; offsets from the workspace base.
 struct Layout {
-  size_t keys = 0, sel = 0, part = 0, bucket = 0, slots = 0, qmask = 0, best = 0, tiles = 0, z = 0, s = 0,
+  size_t keys = 0, sel = 0, part = 0, bucket = 0, qmask = 0, best = 0, tiles = 0, z = 0, s = 0,
          zmax = 0, Z = 0,
          cluster_of = 0, per_draw = 0;
   size_t total = 0;
@@ -77,7 +78,6 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
     }
     if (B == 1 && fh::head1_threads(D.c) != 0) {  // the persistent batch-1 kernel's word table
       L.bucket = take((size_t)fh::kHead1Bins * fh::kHead1BucketCap * 8);
-      L.slots = take((size_t)idx->num_sms * 8);    // and its per-block maxima
     }
   } else if (op == FH_OP_DENSE) {
     const int G = fh::stage2_blocks(D.v, B, idx->num_sms);
@@ -109,14 +109,14 @@ fh_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 // Workspace header (first kHeaderBytes): status word at 0, per-query tickets at 16 (64 x 4 bytes),
 // the persistent head's call generation at 536 (the tag of the last completed call), the tensor-core
-// head's ticket at 544, the persistent head's key-arrival count at 552 and its final-reduction arrival
-// count at 556, the union Stage 2's ticket at 560; bytes
+// head's ticket at 544, the persistent head's key-arrival count at 552 and its count of finished
+// blocks at 556, the union Stage 2's ticket at 560, the persistent head's packed arg-max at 568; bytes
 // [1024, 5120) hold its 1024-bin score histogram in every layout, so no other call ever writes there.
-// The tickets, the arrival counts and the generation only grow; the histogram returns to zero at the
-// end of every call, the word table is tagged with the call generation, and the per-block maxima
-// (the `slots` region) are rewritten by every call.
+// The per-query tickets, the key-arrival count and the generation only grow; the other tickets, the
+// finished-block count, the arg-max and the histogram return to zero at the end of every call, and
+// the word table is tagged with the call generation.
 // A new workspace must start zeroed (fh_ws_status re-zeroes the header after a device-side error,
-// keeping the generation moving).
+// keeping the generation moving; a workspace whose call failed must pass through it before reuse).
 uint32_t* status_of(void* ws) { return reinterpret_cast<uint32_t*>(ws); }
 uint32_t* tickets_of(void* ws) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + 16); }
 uint32_t* word_at(void* ws, size_t off) { return reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + off); }
@@ -226,7 +226,7 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     h.seed = seed;
     h.step = step;
     h.arrive = word_at(ws, kArriveOffset);
-    h.slots = reinterpret_cast<unsigned long long*>(base + L.slots);
+    h.best = reinterpret_cast<unsigned long long*>(base + kBestOffset);
     h.hist = word_at(ws, 1024);
     h.gen = word_at(ws, kGenOffset);
     h.keys_ready = word_at(ws, kKeysReadyOffset);

@@ -352,8 +352,6 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   }
   uint32_t tag = __ldcg(prm.gen) + 1u;  // this call's tag on its words (never 0)
   if (tag == 0u) tag = 1u;
-  uint32_t arrive_base = 0u;  // arrivals of earlier calls (the reducer block waits for G more)
-  if (bid == 0 && tid == 0) arrive_base = __ldcg(prm.arrive);
   if (lane >= pre && lane < K1 && lane < n1)
     issue_row(ring1 + (size_t)lane * row1, src1 + (size_t)(first1 + (int64_t)W * lane) * row1, row1,
               &b1[lane]);
@@ -380,26 +378,26 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   }
   hsq = warp_sum(hsq);
   if (lane == 0) red_s[warp] = hsq;
-  float hreg[INT4_MCH ? INT4_MCH : 1][INT4_MCH ? 32 : 1];
+  // INT4 rows are read as 32-bit words of 8 columns (four words share one group scale): lane l takes
+  // the words l, l + 32, ..., so a row of any width keeps every lane busy but the last pass's, and
+  // keeps the 8 columns of h of each of its words in registers (one conflict-free 16-byte load each).
+  constexpr int kWpl = INT4_MCH ? 4 * INT4_MCH : 1;  // words per lane, at most
+  const int nw4 = nch4 * 4;                            // words per INT4 row
+  float hreg[kWpl][INT4_MCH ? 8 : 1];
   if constexpr (INT4_MCH > 0) {
-    // lane l keeps the 32 columns of its groups l, l + 32, ...: four 16-byte loads per group (lanes
-    // 64 bytes apart: 4-way bank conflicts, where 2-byte loads at that stride were 16-way)
     const uint32_t hs_a = smem_addr(hs);
 #pragma unroll
-    for (int m = 0; m < INT4_MCH; ++m) {
-      const int ch = lane + 32 * m;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = ch < nch4 ? lds_v4(hs_a + 64u * (uint32_t)ch + 16u * (uint32_t)i) : make_uint4(0u, 0u, 0u, 0u);
-        hreg[m][8 * i + 0] = bf16_lo(v.x);
-        hreg[m][8 * i + 1] = bf16_hi(v.x);
-        hreg[m][8 * i + 2] = bf16_lo(v.y);
-        hreg[m][8 * i + 3] = bf16_hi(v.y);
-        hreg[m][8 * i + 4] = bf16_lo(v.z);
-        hreg[m][8 * i + 5] = bf16_hi(v.z);
-        hreg[m][8 * i + 6] = bf16_lo(v.w);
-        hreg[m][8 * i + 7] = bf16_hi(v.w);
-      }
+    for (int i = 0; i < kWpl; ++i) {
+      const int wd = lane + 32 * i;
+      const uint4 v = wd < nw4 ? lds_v4(hs_a + 16u * (uint32_t)wd) : make_uint4(0u, 0u, 0u, 0u);
+      hreg[i][0] = bf16_lo(v.x);
+      hreg[i][1] = bf16_hi(v.x);
+      hreg[i][2] = bf16_lo(v.y);
+      hreg[i][3] = bf16_hi(v.y);
+      hreg[i][4] = bf16_lo(v.z);
+      hreg[i][5] = bf16_hi(v.z);
+      hreg[i][6] = bf16_lo(v.w);
+      hreg[i][7] = bf16_hi(v.w);
     }
   }
   __syncthreads();
@@ -422,13 +420,15 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
     float s;
     if constexpr (INT4_MCH > 0) {
       float part = 0.0f;
+      const uint16_t* scr = sc_s + (k - (int)lo1) * nch4;
+      const uint32_t* roww = reinterpret_cast<const uint32_t*>(ring1 + (size_t)slot * row1);
 #pragma unroll
-      for (int m = 0; m < INT4_MCH; ++m) {
-        const int ch = lane + 32 * m;
-        if (ch < nch4) {
-          const uint4 w = lds_v4(row_s + ch * 16);
-          const float scale = __uint_as_float((uint32_t)sc_s[(k - (int)lo1) * nch4 + ch] << 16);
-          part = fmaf(scale, int4_group_dot(w, hreg[m]), part);
+      for (int i = 0; i < kWpl; ++i) {
+        const int wd = lane + 32 * i;
+        if (wd < nw4) {
+          const uint32_t w = roww[wd];
+          const float scale = __uint_as_float((uint32_t)scr[wd >> 2] << 16);
+          part = fmaf(scale, int4_word_dot(w, hreg[i]), part);
         }
       }
       s = warp_sum(part);
@@ -825,52 +825,34 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   best = warp_max_u64(best);
 
   // ------------------------------------------------------------------ arg-max over the grid
-  // Every block posts its best (value, ~token) to its slot and counts itself in with a release add;
-  // block 0 waits for all G arrivals of this call, reduces the slots, writes the token and returns
-  // the histogram to zero for the next call.  No other block waits for anything here.
+  // Every block folds its best (value, ~token) into the call's maximum with one relaxed 64-bit max and
+  // counts itself in with an acquire-release add; the block that arrives last reads the maximum,
+  // writes the token and returns the maximum, the count and the histogram to zero for the next call.
+  // No block waits for another here.
   if (lane == 0) warp_best[warp] = best;
   __syncthreads();
   H1_STAMP(7);
   if (tid == 0) {
     unsigned long long bb = 0ull;
     for (int w = 0; w < W; ++w) bb = warp_best[w] > bb ? warp_best[w] : bb;
-    st_relaxed_u64(prm.slots + bid, bb);
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(prm.arrive) : "memory");
-  }
-  if (bid != 0) return;
-  if (tid == 0) {
-    const uint32_t target = arrive_base + uG;
-    const uint64_t t0 = global_timer_ns();
-    abort_s = false;
-    for (uint32_t it = 1;; ++it) {
-      uint32_t a;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(a) : "l"(prm.arrive) : "memory");
-      if ((int32_t)(a - target) >= 0) break;
-      if ((it & 63u) == 0 && global_timer_ns() - t0 > 500000000ull) {
-        set_status(prm.status, kStatusTimeout);
-        abort_s = true;
-        break;
-      }
-    }
+    asm volatile("red.relaxed.gpu.global.max.u64 [%0], %1;" ::"l"(prm.best), "l"(bb) : "memory");
+    uint32_t old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(prm.arrive) : "memory");
+    abort_s = old != uG - 1u;  // (not the last block)
   }
   __syncthreads();
-  H1_STAMP(8);
   if (abort_s) return;
-  unsigned long long mine = 0ull;
-  for (int i = tid; i < G; i += NT) {
-    const unsigned long long v = __ldcg(prm.slots + i);
-    mine = v > mine ? v : mine;
-  }
-  mine = warp_max_u64(mine);
-  if (lane == 0) warp_best[warp] = mine;
+  H1_STAMP(8);
   for (int i = tid; i < kHistBins; i += NT) prm.hist[i] = 0u;
   if (tag == 0xFFFFFFFFu) {  // the tags wrap after this call: no older word may alias a new tag
+#pragma unroll 1
     for (int i = tid; i < kHistBins * kCap; i += NT) prm.bucket[i] = 0ull;
   }
-  __syncthreads();
   if (tid == 0) {
-    unsigned long long fin = 0ull;
-    for (int w = 0; w < W; ++w) fin = warp_best[w] > fin ? warp_best[w] : fin;
+    unsigned long long fin;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(fin) : "l"(prm.best) : "memory");
+    st_relaxed_u64(prm.best, 0ull);
+    *prm.arrive = 0u;
     *prm.gen = tag;
     prm.out_tok[0] = (int32_t)best_id(fin);
   }

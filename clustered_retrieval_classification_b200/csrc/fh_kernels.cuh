@@ -164,8 +164,8 @@ struct Head1Params {
   int sample;
   float tau;
   uint64_t seed, step;
-  uint32_t* arrive;               // final-reduction arrivals (grows by gridDim.x per call)
-  unsigned long long* slots;      // gridDim.x packed (key, ~token) maxima, one per block
+  uint32_t* arrive;               // blocks done with the call (zero between calls)
+  unsigned long long* best;       // the call's packed (key, ~token) maximum (zero between calls)
   uint32_t* hist;                 // kHead1Bins-bin key histogram (zero between calls)
   uint32_t* gen;                  // tag of the last completed call (a call tags its words gen+1)
   uint32_t* keys_ready;           // arrivals once the keys are written (grows by gridDim.x per use)

@@ -149,6 +149,21 @@ __device__ __forceinline__ float int4_group_dot(const uint4 w, const float* hg) 
   return acc_e + acc_o;
 }
 
+// One 32-bit word of an INT4 row: columns 0..7 of h (hw), low nibble = even column.
+__device__ __forceinline__ float int4_word_dot(const uint32_t w, const float* hw) {
+  const uint32_t even = (w & 0x0F0F0F0Fu) ^ 0x08080808u;
+  const uint32_t odd = ((w >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;
+  float acc_e = 0.0f, acc_o = 0.0f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float qe = __uint_as_float(__byte_perm(even, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
+    const float qo = __uint_as_float(__byte_perm(odd, 0x4B000000u, 0x7440u + j)) - 8388616.0f;
+    acc_e = fmaf(qe, hw[2 * j], acc_e);
+    acc_o = fmaf(qo, hw[2 * j + 1], acc_o);
+  }
+  return acc_e + acc_o;
+}
+
 // The 32 values of one INT4 group (columns 0..31, low nibble = even column), decoded exactly.
 __device__ __forceinline__ void int4_decode32(const uint4 w, float (&dq)[32]) {
   const uint32_t words[4] = {w.x, w.y, w.z, w.w};

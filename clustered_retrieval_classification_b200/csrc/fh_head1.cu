@@ -408,7 +408,11 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   const bool all = prm.p >= c;
 
   // ------------------------------------------------------------------ Stage 1
+  // The score of the warp's row n stays in lane n (n1 <= 32: a block has at most NT rows) until the
+  // stream is over; the keys are then formed and counted by all lanes at once.
   const uint32_t hs_addr = smem_addr(hs);
+  float my_s = 0.0f;
+  int n_done = 0;
   for (int n = 0, slot = 0, phase = 0; n < n1; ++n) {
     if (!mbar_wait(&b1[slot], (uint32_t)phase, prm.status)) {
       for (int m = n + 1; m < n1 && m < n + K1; ++m)
@@ -436,23 +440,28 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
       s = warp_sum(row_dot_partial<ELEM>(row_s, hs_addr, nch2, lane));
     }
     __syncwarp();
-    if (lane == 0) {
-      if (n + K1 < n1) {
-        fence_proxy_async_smem();
-        issue_row(ring1 + (size_t)slot * row1, src1 + (size_t)(first1 + (int64_t)W * (n + K1)) * row1,
-                  row1, &b1[slot]);
-      }
-      float key = s;
-      if (prm.sample)
-        key = s / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 0u, (uint32_t)k));
-      prm.keys[k] = key;
-      own_keys[k - (int)lo1] = key;
-      if (!all) own_pos[k - (int)lo1] = atomicAdd(&hist_s[bin(key)], 1u);
+    if (lane == 0 && n + K1 < n1) {
+      fence_proxy_async_smem();
+      issue_row(ring1 + (size_t)slot * row1, src1 + (size_t)(first1 + (int64_t)W * (n + K1)) * row1,
+                row1, &b1[slot]);
     }
+    my_s = lane == n ? s : my_s;
+    n_done = n + 1;
+    if (n == 0) H1_STAMP(13);
     if (++slot == K1) {
       slot = 0;
       phase ^= 1;
     }
+  }
+  H1_STAMP(14);
+  if (lane < n_done) {
+    const int k = (int)first1 + W * lane;
+    float key = my_s;
+    if (prm.sample)
+      key = my_s / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, 0u, 0u, (uint32_t)k));
+    prm.keys[k] = key;
+    own_keys[k - (int)lo1] = key;
+    if (!all) own_pos[k - (int)lo1] = atomicAdd(&hist_s[bin(key)], 1u);
   }
   __syncthreads();
   H1_STAMP(2);

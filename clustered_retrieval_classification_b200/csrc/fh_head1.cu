@@ -735,18 +735,22 @@ __global__ void __launch_bounds__(NT, 1) k_head1(const Head1Params prm) {
   uint8_t* ring2 = ring + (size_t)warp * K2 * row2;
   uint64_t* b2 = bars2 + warp * K2;
   float* zr = reinterpret_cast<float*>(smem + L.zr);  // logit of block row g - r0
+  // The C2T copies go out from the last warp, one lane a cluster (warp 0 carries the block's other
+  // serial work).
   auto issue_tok = [&]() {
-    if (tid == 0 && nrk > 0) {
+    if (warp == W - 1 && nrk > 0) {
       uint32_t bytes = 0;
-      for (int i = 0; i < nrk; ++i) {
+      for (int i = lane; i < nrk; i += 32) {
         const int e0 = rk_id[i] * b;
         bytes += (uint32_t)(((e0 + b + 3) & ~3) - (e0 & ~3)) * 4u;
       }
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(tok_bar, bytes);
-      for (int i = 0; i < nrk; ++i) {
+      bytes = __reduce_add_sync(0xFFFFFFFFu, bytes);
+      if (lane == 0) mbar_arrive_expect_tx(tok_bar, bytes);
+      __syncwarp();
+      for (int i = lane; i < nrk; i += 32) {
         const int e0 = rk_id[i] * b;
         const int s0 = e0 & ~3;
+        fence_proxy_async_smem();
         bulk_g2s(tokr + i * tsw, prm.C2T + s0, (uint32_t)(((e0 + b + 3) & ~3) - s0) * 4u, tok_bar);
       }
     }

@@ -141,9 +141,20 @@ struct TcLay {
   uint32_t h_bytes, e_bytes, stage_bytes;
   uint32_t row_off, gum_off, pair_off, bar_off, dyn;
 };
-__host__ __device__ inline TcLay tc_layout(int B, int tile_rows, int wave, bool sample, int stages) {
+// Where the epilogue bounds the kernel, the queries fill the MMA's 128 rows: qrows = 32 or 64 rows
+// (the batch, zero-padded) repeated copies = 128 / qrows times, so that every epilogue warp's
+// tensor-memory lanes hold live queries (lane l: query l % qrows) and the warps holding copies of the
+// same queries split a tile's rows between them.  Otherwise one copy of the batch padded to 16 rows
+// (the MMA's rows past it read whatever follows in shared memory; their lanes are never read).
+__host__ __device__ inline void tc_query_layout(int B, bool copies, int& qrows, int& ncopies) {
+  qrows = copies ? (B <= 32 ? 32 : 64) : (B + 15) / 16 * 16;
+  ncopies = copies ? 128 / qrows : 1;
+}
+
+__host__ __device__ inline TcLay tc_layout(int qrows, int copies, int tile_rows, int wave, bool sample,
+                                           int stages) {
   TcLay L;
-  L.h_bytes = (uint32_t)((B + 15) / 16 * 16) * 128u;  // multiple of 2048: keeps E blocks 1024-aligned
+  L.h_bytes = (uint32_t)(qrows * copies) * 128u;  // multiple of 2048: E blocks stay 1024-aligned
   L.e_bytes = (uint32_t)tile_rows * 128u;
   L.stage_bytes = L.h_bytes + (uint32_t)wave * L.e_bytes;
   L.row_off = (uint32_t)stages * L.stage_bytes;
@@ -167,7 +178,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023u) & ~uintptr_t(1023));
   constexpr int WT = KEYS ? 1 : kTcWave;
   const int R = a.tile_rows, S = a.stages;
-  const TcLay Lay = tc_layout(a.B, R, WT, SAMPLE, S);
+  const int Bq = a.qrows, D = a.copies;  // query rows of one copy, copies
+  const TcLay Lay = tc_layout(Bq, D, R, WT, SAMPLE, S);
   uint32_t* tok_s = reinterpret_cast<uint32_t*>(smem + Lay.row_off);                     // 128
   unsigned long long* msk_s = reinterpret_cast<unsigned long long*>(smem + Lay.row_off + 512u);  // 128
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay.bar_off);
@@ -222,8 +234,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int w = 0; w < n_waves && ok; ++w) {
       const int j0 = w * WT, nt = min(WT, my_tiles - j0);
       if (lane == 0) {
-        int tl[kTcWave];
-        for (int j = 0; j < nt; ++j) tl[j] = tile_at(j0 + j);
+        // the wave's E tiles go out before the query rows (the bytes that come from HBM first)
+        static_assert(kTcWave == 2, "two tiles a wave");
+        const int y0 = tile_at(j0) * R, y1 = nt > 1 ? tile_at(j0 + 1) * R : y0;
         const uint32_t bytes = Lay.h_bytes + (uint32_t)nt * Lay.e_bytes;  // H rows past B read as zeros
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = it % S;
@@ -233,9 +246,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           uint8_t* stg = smem + (size_t)s * Lay.stage_bytes;
           mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d(stg, &tmH, kb * kTcKB, 0, &full[s]);
-          for (int j = 0; j < nt; ++j)
-            tma_load_2d(stg + Lay.h_bytes + (size_t)j * Lay.e_bytes, &tmE, kb * kTcKB, tl[j] * R, &full[s]);
+          tma_load_2d(stg + Lay.h_bytes, &tmE, kb * kTcKB, y0, &full[s]);
+          if (nt > 1) tma_load_2d(stg + Lay.h_bytes + Lay.e_bytes, &tmE, kb * kTcKB, y1, &full[s]);
+          for (int r = 0; r < D; ++r) tma_load_2d(stg + (size_t)r * Bq * 128u, &tmH, kb * kTcKB, 0, &full[s]);
         }
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -286,8 +299,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (warp >= 4) {
     // ---------------------------------------------------------------- epilogue: one query per thread
-    const int et = tid - 128;             // 0..127: this thread's query and its tile-row duty
-    const int q = et;                     // lane q of tensor memory (warp quarter = warp % 4)
+    const int et = tid - 128;             // 0..127: this thread's lane of tensor memory and tile-row duty
+    const int qmod = 128 / D;             // lanes per copy of the queries
+    const int q = et & (qmod - 1);        // its query (warp quarter = warp % 4)
+    const int rep = et / qmod;            // its copy of the queries: it takes chunks rep, rep + D, ...
     const bool q_live = q < a.B;          // lanes past the batch take no row but join every warp step
     uint32_t bk = 0u, bt = 0xFFFFFFFFu;   // best key image and its token
     auto group_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
@@ -307,7 +322,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         const uint32_t tbase = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(acc * 256 + j * R);
         const int64_t row0 = (int64_t)t * R;  // contiguous mode: first row of the tile
-        for (int c0 = 0; c0 < R; c0 += 32) {
+        for (int c0 = 32 * rep; c0 < R; c0 += 32 * D) {
           uint32_t v[32];
           tmem_ld16(tbase + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(v));
           tmem_ld16(tbase + (uint32_t)c0 + 16u, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
@@ -360,7 +375,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               for (int step = 16; step > 0; step >>= 1)
                 if (i + step < 32 && bal_s[32 + i + step] <= k) i += step;
               const uint32_t ql = __fns(bal_s[i], 0u, (int)(k - bal_s[32 + i]) + 1);
-              const uint32_t qq = (uint32_t)(32 * (warp & 3)) + ql;
+              const uint32_t qq = (uint32_t)((32 * (warp & 3)) & (qmod - 1)) + ql;
               gum[i * 32 + (int)ql] = gumbel_from_u32(philox_word(a.seed, a.step, qq, 1u, tok_s[c0 + i]));
             }
             __syncwarp();
@@ -484,12 +499,12 @@ cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, TcParams
   const int wave = keys ? 1 : kTcWave;
   int S = kTcMaxStages;
   for (; S >= 2; --S)
-    if (tc_layout(p.B, p.tile_rows, wave, sample, S).dyn <= kTcSmemMax) break;
+    if (tc_layout(p.qrows, p.copies, p.tile_rows, wave, sample, S).dyn <= kTcSmemMax) break;
   if (S < 2) return cudaErrorInvalidValue;
   p.stages = S;
   auto kern = keys ? (sample ? k_tc_head<true, true> : k_tc_head<true, false>)
                    : (sample ? k_tc_head<false, true> : k_tc_head<false, false>);
-  const uint32_t dyn = tc_layout(p.B, p.tile_rows, wave, sample, S).dyn;
+  const uint32_t dyn = tc_layout(p.qrows, p.copies, p.tile_rows, wave, sample, S).dyn;
   cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(kern), dyn);
   if (e != cudaSuccess) return e;
   // every SM when the tiles are listed on the device; otherwise no more CTAs than tiles
@@ -806,7 +821,11 @@ cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms
     if (e != cudaSuccess) return e;
   }
   CUtensorMap mE, mH;
-  if (!make_map(&mE, A, p.d, p.rows, box) || !make_map(&mH, H, p.d, p.B, (uint32_t)((p.B + 15) / 16 * 16)))
+  // copies of the queries where the epilogue bounds the kernel: the head modes, sampled keys, and
+  // keys of more than 32 queries (measured at the Llama-3.2-1B shape; below that the plain keys'
+  // epilogue is light, and copies multiply the query bytes each stage brings in)
+  tc_query_layout(p.B, !p.out_keys || p.sample || p.B > 32, p.qrows, p.copies);
+  if (!make_map(&mE, A, p.d, p.rows, box) || !make_map(&mH, H, p.d, p.B, (uint32_t)p.qrows))
     return cudaErrorInvalidValue;
   return launch_kernel(mE, mH, p, num_sms, st);
 }

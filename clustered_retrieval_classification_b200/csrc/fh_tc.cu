@@ -36,6 +36,11 @@ namespace {
 
 constexpr int kTcKB = 64;          // K elements per stage: one 128-byte swizzle atom per row
 constexpr int kTcThreads = 256;
+// The tensor-core head: warps 0-3 (TMA producer, MMA issuer, tensor-memory owner, spare) and eight
+// epilogue warps, two on each quarter of the tensor-memory lanes, reading 16-row chunks.
+constexpr int kTcEpiWarps = 8;
+constexpr int kTcHeadThreads = 128 + 32 * kTcEpiWarps;
+constexpr int kTcChunk = 16;
 
 // ------------------------------------------------------------------ tcgen05 / TMA primitives
 
@@ -139,7 +144,7 @@ constexpr uint32_t kTcSmemMax = 226u * 1024u;
 // rows (token, mask), the sampling scratch, the barriers.
 struct TcLay {
   uint32_t h_bytes, e_bytes, stage_bytes;
-  uint32_t row_off, gum_off, pair_off, bar_off, dyn;
+  uint32_t row_off, gum_off, bar_off, dyn;
 };
 // Where the epilogue bounds the kernel, the queries fill the MMA's 128 rows: qrows = 32 or 64 rows
 // (the batch, zero-padded) repeated copies = 128 / qrows times, so that every epilogue warp's
@@ -159,8 +164,7 @@ __host__ __device__ inline TcLay tc_layout(int qrows, int copies, int tile_rows,
   L.stage_bytes = L.h_bytes + (uint32_t)wave * L.e_bytes;
   L.row_off = (uint32_t)stages * L.stage_bytes;
   L.gum_off = L.row_off + (uint32_t)kTcRows * 12u;
-  L.pair_off = L.gum_off + (sample ? 4u * 32u * 32u * 4u : 0u);
-  L.bar_off = L.pair_off + (sample ? 4u * 64u * 4u : 0u);
+  L.bar_off = L.gum_off + (sample ? (uint32_t)kTcEpiWarps * kTcChunk * 32u * 4u : 0u);  // G[row][lane] a warp
   const uint32_t end = L.bar_off + (uint32_t)(2 * kTcMaxStages + 8) * 8u;
   // the last stage's H operand is read as 128 rows of 128 B
   const uint32_t h_end = (uint32_t)(stages > 0 ? stages - 1 : 0) * L.stage_bytes + 128u * 128u;
@@ -171,7 +175,7 @@ __host__ __device__ inline TcLay tc_layout(int qrows, int copies, int tile_rows,
 // KEYS: write the products (Stage-1 keys) instead of reducing an arg-max; SAMPLE: add the Gumbel
 // term.  Separate instantiations keep each epilogue's code out of the other modes' instruction stream.
 template <bool KEYS, bool SAMPLE>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcHeadThreads, 1)
     k_tc_head(const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmH,
               const TcParams a) {
   extern __shared__ uint8_t smem_raw[];
@@ -211,7 +215,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 4);
+      mbar_init(&tempty[i], kTcEpiWarps);
     }
     mbar_init(drain, 1);
     abort_s = 0;
@@ -298,39 +302,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    // ---------------------------------------------------------------- epilogue: one query per thread
-    const int et = tid - 128;             // 0..127: this thread's lane of tensor memory and tile-row duty
-    const int qmod = 128 / D;             // lanes per copy of the queries
-    const int q = et & (qmod - 1);        // its query (warp quarter = warp % 4)
-    const int rep = et / qmod;            // its copy of the queries: it takes chunks rep, rep + D, ...
-    const bool q_live = q < a.B;          // lanes past the batch take no row but join every warp step
-    uint32_t bk = 0u, bt = 0xFFFFFFFFu;   // best key image and its token
-    auto group_sync = [] { asm volatile("bar.sync 1, 128;" ::: "memory"); };
+    // ---------------------------------------------------------------- epilogue
+    // Thread et reads lane el = et % 128 of tensor memory (its warp's quarter), which holds query
+    // q = el % (128 / D) of copy el / (128 / D); with its half h = et / 128 that names one of 2·D slots,
+    // and the 16-row chunks of a tile go round robin over the slots.
+    const int et = tid - 128;                    // 0 .. 32·kTcEpiWarps - 1
+    const int el = et & 127;                     // its lane of tensor memory
+    const int qmod = 128 / D;                    // lanes per copy of the queries
+    const int q = el & (qmod - 1);               // its query
+    const int slot = el / qmod + D * (et >> 7);  // its chunks: slot, slot + 2·D, ...
+    const bool q_live = q < a.B;                 // lanes past the batch take no row but join every warp step
+    uint32_t bk = 0u, bt = 0xFFFFFFFFu;          // best key image and its token
+    auto group_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(32 * kTcEpiWarps) : "memory"); };
+    // A tile's rows: token and query mask (0: no query takes the row, or no row), staged by the first
+    // 128 threads.  The next tile's are loaded into registers while the current tile is reduced.
+    uint32_t tok_n = 0u;
+    unsigned long long msk_n = 0ull;
+    auto load_rows = [&](int jj) {
+      const int64_t row = (int64_t)tile_at(jj) * kTcRows + et;
+      const bool valid = row < a.rows;
+      const int64_t cl = a.qmask ? row / a.b : 0;
+      tok_n = valid ? (a.row_tok ? (uint32_t)__ldg(a.row_tok + row) : (uint32_t)row) : 0u;
+      msk_n = valid ? (a.qmask ? __ldg(a.qmask + cl) : ~0ull) : 0ull;
+    };
+    if (!KEYS && my_tiles > 0 && et < 128) load_rows(0);
     for (int w = 0; w < n_waves; ++w) {
       const int j0 = w * WT, nt = min(WT, my_tiles - j0), acc = w & 1;
       if (!tc_wait(&tfull[acc], (uint32_t)((w >> 1) & 1), &abort_s, a.status)) break;
       tc_fence_after();
       for (int j = 0; j < nt; ++j) {
         const int t = tile_at(j0 + j);
-        if constexpr (!KEYS) {  // the tile's rows: token and query mask (0: no query takes the row, or no row)
-          const int64_t row = (int64_t)t * kTcRows + et;
-          const bool valid = row < a.rows;
-          const int64_t cl = a.qmask ? row / a.b : 0;
-          tok_s[et] = valid ? (a.row_tok ? (uint32_t)__ldg(a.row_tok + row) : (uint32_t)row) : 0u;
-          msk_s[et] = valid ? (a.qmask ? __ldg(a.qmask + cl) : ~0ull) : 0ull;
+        if constexpr (!KEYS) {
+          if (et < 128) {
+            tok_s[et] = tok_n;
+            msk_s[et] = msk_n;
+          }
           group_sync();
+          if (et < 128 && j0 + j + 1 < my_tiles) load_rows(j0 + j + 1);
         }
         const uint32_t tbase = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(acc * 256 + j * R);
         const int64_t row0 = (int64_t)t * R;  // contiguous mode: first row of the tile
-        for (int c0 = 32 * rep; c0 < R; c0 += 32 * D) {
-          uint32_t v[32];
-          tmem_ld16(tbase + (uint32_t)c0, *reinterpret_cast<uint32_t(*)[16]>(v));
-          tmem_ld16(tbase + (uint32_t)c0 + 16u, *reinterpret_cast<uint32_t(*)[16]>(v + 16));
+        for (int c0 = kTcChunk * slot; c0 < R; c0 += kTcChunk * 2 * D) {
+          uint32_t v[kTcChunk];
+          tmem_ld16(tbase + (uint32_t)c0, v);
           tmem_ld_wait();
           if constexpr (KEYS) {  // Stage-1 keys (contiguous rows): s[q][row] or s/τ + G(q, stream 0, row)
             if (q < a.B) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
+              for (int i = 0; i < kTcChunk; ++i) {
                 const int64_t row = row0 + c0 + i;
                 if (row < a.rows) {
                   const float z = __uint_as_float(v[i]);
@@ -341,61 +360,42 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
             continue;
           }
-          if constexpr (!SAMPLE) {
-            if (!q_live) continue;  // (uniform per warp when B is a multiple of 32)
-          }
+          // the chunk's rows this thread's query takes (bit i: row c0 + i), from the rows' query masks
+          uint32_t tm = 0u;
+#pragma unroll
+          for (int i = 0; i < kTcChunk; ++i) tm |= (uint32_t)((msk_s[c0 + i] >> q) & 1ull) << i;
+          if (!q_live) tm = 0u;
+          if (__ballot_sync(0xFFFFFFFFu, tm != 0u) == 0u) continue;  // no lane takes a row of the chunk
           float* gum = nullptr;
           if constexpr (SAMPLE) {
-            // The Gumbel terms G(q, 1, token) of the (row, query) pairs this warp takes in the chunk,
-            // spread evenly over the lanes: a row is taken by few of the warp's 32 queries, so one
-            // evaluation per row and lane would leave most lanes idle.  Lane i lists row i's takers
-            // (a ballot), a scan gives each row its first pair, and pair k goes to lane k % 32.
-            uint32_t* bal_s = reinterpret_cast<uint32_t*>(smem + Lay.pair_off) + (warp & 3) * 64;
-            gum = reinterpret_cast<float*>(smem + Lay.gum_off) + (warp & 3) * 1024;
-            uint32_t my_bal = 0u;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const uint32_t bi = __ballot_sync(0xFFFFFFFFu, q_live && ((msk_s[c0 + i] >> q) & 1ull));
-              if (lane == i) my_bal = bi;
+            // the Gumbel terms G(q, 1, token) of the rows this thread takes, two at a time (two
+            // independent Philox chains), in the warp's buffer at [row][lane]
+            gum = reinterpret_cast<float*>(smem + Lay.gum_off) + (warp - 4) * (kTcChunk * 32);
+            for (uint32_t rest = tm; rest != 0u;) {
+              const int ia = __ffs(rest) - 1;
+              rest &= rest - 1u;
+              const int ib = rest ? __ffs(rest) - 1 : ia;
+              if (rest) rest &= rest - 1u;
+              const uint32_t wa = philox_word(a.seed, a.step, (uint32_t)q, 1u, tok_s[c0 + ia]);
+              const uint32_t wb = philox_word(a.seed, a.step, (uint32_t)q, 1u, tok_s[c0 + ib]);
+              gum[ia * 32 + lane] = gumbel_from_u32(wa);
+              gum[ib * 32 + lane] = gumbel_from_u32(wb);
             }
-            const uint32_t my_cnt = __popc(my_bal);
-            uint32_t incl = my_cnt;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-              if (lane >= o) incl += y;
-            }
-            bal_s[lane] = my_bal;
-            bal_s[32 + lane] = incl - my_cnt;  // the row's first pair
-            const uint32_t pairs = __shfl_sync(0xFFFFFFFFu, incl, 31);
-            __syncwarp();
-            for (uint32_t k = (uint32_t)lane; k < pairs; k += 32u) {
-              int i = 0;  // the last row whose first pair is <= k
-#pragma unroll
-              for (int step = 16; step > 0; step >>= 1)
-                if (i + step < 32 && bal_s[32 + i + step] <= k) i += step;
-              const uint32_t ql = __fns(bal_s[i], 0u, (int)(k - bal_s[32 + i]) + 1);
-              const uint32_t qq = (uint32_t)((32 * (warp & 3)) & (qmod - 1)) + ql;
-              gum[i * 32 + (int)ql] = gumbel_from_u32(philox_word(a.seed, a.step, qq, 1u, tok_s[c0 + i]));
-            }
-            __syncwarp();
           }
+          // the decision over the chunk, branch-free: every row's loads are independent of the others'
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const unsigned long long mk = msk_s[c0 + i];
-            if (!q_live || !((mk >> q) & 1ull)) continue;
+          for (int i = 0; i < kTcChunk; ++i) {
+            const bool take = (tm >> i) & 1u;
             const uint32_t tk = tok_s[c0 + i];
             const float z = __uint_as_float(v[i]);
-            if (a.out_logits) a.out_logits[(int64_t)q * a.rows + tk] = z;
+            if (a.out_logits && take) a.out_logits[(int64_t)q * a.rows + tk] = z;
             float val = z;
-            if constexpr (SAMPLE) val = z / a.tau + gum[i * 32 + lane];
+            if constexpr (SAMPLE) val = z / a.tau + (take ? gum[i * 32 + lane] : 0.0f);
             const uint32_t key = float_key(val);
-            if (key > bk || (key == bk && tk < bt)) {
-              bk = key;
-              bt = tk;
-            }
+            const bool better = take && (key > bk || (key == bk && tk < bt));
+            bk = better ? key : bk;
+            bt = better ? tk : bt;
           }
-          if constexpr (SAMPLE) __syncwarp();  // the warp's G buffer is rewritten for the next chunk
         }
         if constexpr (!KEYS) group_sync();  // the tile rows are rewritten for the next tile
       }
@@ -509,7 +509,7 @@ cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, TcParams
   if (e != cudaSuccess) return e;
   // every SM when the tiles are listed on the device; otherwise no more CTAs than tiles
   const int grid = (p.tile_list || p.n_tiles >= num_sms) ? num_sms : p.n_tiles;
-  kern<<<grid, kTcThreads, dyn, st>>>(mE, mH, p);
+  kern<<<grid, kTcHeadThreads, dyn, st>>>(mE, mH, p);
   return cudaGetLastError();
 }
 

@@ -112,6 +112,7 @@ struct TcParams {
   uint32_t* status;
   int n_tiles, tile_rows, stages;  // set by the launcher
   int qrows, copies;               // query rows of one copy in the MMA's 128 rows, copies (launcher)
+  int kbs;                         // K-blocks per pipeline stage (launcher)
 };
 // Batched Stage 2 over the union of the batch's probe sets (fh_kernels.cu): the listed clusters of
 // the cluster-major copy, each row dotted with the queries whose mask bit is set.

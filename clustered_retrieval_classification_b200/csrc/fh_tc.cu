@@ -41,6 +41,16 @@ constexpr int kTcThreads = 256;
 constexpr int kTcEpiWarps = 8;
 constexpr int kTcHeadThreads = 128 + 32 * kTcEpiWarps;
 constexpr int kTcChunk = 16;
+// K-blocks per pipeline stage: a stage then fetches a row's consecutive K-blocks together (the keys'
+// 64-row tiles fetched 128 bytes of each row per stage: 20.5 µs for the Llama-shaped keys at one
+// K-block per stage, 15.3 at two, 12.0 at four, no better at eight; the head modes' 128-row tiles
+// gain ~3 % at two); fewer when two stages would not fit.
+#ifndef FH_TC_KEYS_KBS
+#define FH_TC_KEYS_KBS 4
+#endif
+#ifndef FH_TC_HEAD_KBS
+#define FH_TC_HEAD_KBS 2
+#endif
 
 // ------------------------------------------------------------------ tcgen05 / TMA primitives
 
@@ -143,7 +153,7 @@ constexpr uint32_t kTcSmemMax = 226u * 1024u;
 // Dynamic shared memory of the kernel: `stages` stages of (H block, E blocks of the wave), the tile
 // rows (token, mask), the sampling scratch, the barriers.
 struct TcLay {
-  uint32_t h_bytes, e_bytes, stage_bytes;
+  uint32_t h_bytes, e_bytes, sub_bytes, stage_bytes;  // one K-block: H, one E tile, H + the wave; a stage
   uint32_t row_off, gum_off, bar_off, dyn;
 };
 // Where the epilogue bounds the kernel, the queries fill the MMA's 128 rows: qrows = 32 or 64 rows
@@ -156,18 +166,21 @@ __host__ __device__ inline void tc_query_layout(int B, bool copies, int& qrows, 
   ncopies = copies ? 128 / qrows : 1;
 }
 
+// A stage holds kbs consecutive K-blocks, each laid out as [H][E tile 0][E tile 1 ...].
 __host__ __device__ inline TcLay tc_layout(int qrows, int copies, int tile_rows, int wave, bool sample,
-                                           int stages) {
+                                           int stages, int kbs) {
   TcLay L;
   L.h_bytes = (uint32_t)(qrows * copies) * 128u;  // multiple of 2048: E blocks stay 1024-aligned
   L.e_bytes = (uint32_t)tile_rows * 128u;
-  L.stage_bytes = L.h_bytes + (uint32_t)wave * L.e_bytes;
+  L.sub_bytes = L.h_bytes + (uint32_t)wave * L.e_bytes;
+  L.stage_bytes = (uint32_t)kbs * L.sub_bytes;
   L.row_off = (uint32_t)stages * L.stage_bytes;
   L.gum_off = L.row_off + (uint32_t)kTcRows * 12u;
   L.bar_off = L.gum_off + (sample ? (uint32_t)kTcEpiWarps * kTcChunk * 32u * 4u : 0u);  // G[row][lane] a warp
   const uint32_t end = L.bar_off + (uint32_t)(2 * kTcMaxStages + 8) * 8u;
-  // the last stage's H operand is read as 128 rows of 128 B
-  const uint32_t h_end = (uint32_t)(stages > 0 ? stages - 1 : 0) * L.stage_bytes + 128u * 128u;
+  // the last K-block's H operand is read as 128 rows of 128 B
+  const uint32_t h_end = (uint32_t)(stages > 0 ? stages - 1 : 0) * L.stage_bytes +
+                         (uint32_t)(kbs - 1) * L.sub_bytes + 128u * 128u;
   L.dyn = (end > h_end ? end : h_end) + 1024u;  // + alignment slack
   return L;
 }
@@ -183,7 +196,8 @@ __global__ void __launch_bounds__(kTcHeadThreads, 1)
   constexpr int WT = KEYS ? 1 : kTcWave;
   const int R = a.tile_rows, S = a.stages;
   const int Bq = a.qrows, D = a.copies;  // query rows of one copy, copies
-  const TcLay Lay = tc_layout(Bq, D, R, WT, SAMPLE, S);
+  const int KBS = a.kbs;                  // K-blocks per stage
+  const TcLay Lay = tc_layout(Bq, D, R, WT, SAMPLE, S, KBS);
   uint32_t* tok_s = reinterpret_cast<uint32_t*>(smem + Lay.row_off);                     // 128
   unsigned long long* msk_s = reinterpret_cast<unsigned long long*>(smem + Lay.row_off + 512u);  // 128
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Lay.bar_off);
@@ -198,6 +212,7 @@ __global__ void __launch_bounds__(kTcHeadThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;
   const int KB = (int)((a.d + kTcKB - 1) / kTcKB);
+  const int NG = (KB + KBS - 1) / KBS;  // stages a wave takes
   // This CTA's tiles: bid, bid + G, ... of every tile, or in listed mode of the contiguous tiles some
   // query takes, tile_list[0 .. *tile_count)
   const int n_list = a.tile_list ? __ldg(a.tile_count) : a.n_tiles;
@@ -241,18 +256,25 @@ __global__ void __launch_bounds__(kTcHeadThreads, 1)
         // the wave's E tiles go out before the query rows (the bytes that come from HBM first)
         static_assert(kTcWave == 2, "two tiles a wave");
         const int y0 = tile_at(j0) * R, y1 = nt > 1 ? tile_at(j0 + 1) * R : y0;
-        const uint32_t bytes = Lay.h_bytes + (uint32_t)nt * Lay.e_bytes;  // H rows past B read as zeros
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t kb_bytes = Lay.h_bytes + (uint32_t)nt * Lay.e_bytes;  // H rows past B read as zeros
+        for (int g = 0; g < NG; ++g, ++it) {
           const int s = it % S;
           if (!tc_wait(&empty[s], (uint32_t)(((it / S) & 1) ^ 1), &abort_s, a.status)) {
             ok = false;
             break;
           }
+          const int kb0 = g * KBS, kbn = min(KBS, KB - kb0);
           uint8_t* stg = smem + (size_t)s * Lay.stage_bytes;
-          mbar_arrive_expect_tx(&full[s], bytes);
-          tma_load_2d(stg + Lay.h_bytes, &tmE, kb * kTcKB, y0, &full[s]);
-          if (nt > 1) tma_load_2d(stg + Lay.h_bytes + Lay.e_bytes, &tmE, kb * kTcKB, y1, &full[s]);
-          for (int r = 0; r < D; ++r) tma_load_2d(stg + (size_t)r * Bq * 128u, &tmH, kb * kTcKB, 0, &full[s]);
+          mbar_arrive_expect_tx(&full[s], (uint32_t)kbn * kb_bytes);
+          for (int kk = 0; kk < kbn; ++kk) {  // a row's consecutive K-blocks go out together
+            uint8_t* sub = stg + (size_t)kk * Lay.sub_bytes;
+            tma_load_2d(sub + Lay.h_bytes, &tmE, (kb0 + kk) * kTcKB, y0, &full[s]);
+            if (nt > 1) tma_load_2d(sub + Lay.h_bytes + Lay.e_bytes, &tmE, (kb0 + kk) * kTcKB, y1, &full[s]);
+          }
+          for (int kk = 0; kk < kbn; ++kk)
+            for (int r = 0; r < D; ++r)
+              tma_load_2d(stg + (size_t)kk * Lay.sub_bytes + (size_t)r * Bq * 128u, &tmH, (kb0 + kk) * kTcKB,
+                          0, &full[s]);
         }
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
@@ -274,7 +296,7 @@ __global__ void __launch_bounds__(kTcHeadThreads, 1)
         const int nt = min(WT, my_tiles - w * WT), acc = w & 1;
         if (!tc_wait(&tempty[acc], (uint32_t)(((w >> 1) & 1) ^ 1), &abort_s, a.status)) break;
         tc_fence_after();
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        for (int g = 0; g < NG; ++g, ++it) {
           const int s = it % S;
           if (!tc_wait(&full[s], (uint32_t)((it / S) & 1), &abort_s, a.status)) {
             ok = false;
@@ -282,14 +304,18 @@ __global__ void __launch_bounds__(kTcHeadThreads, 1)
           }
           tc_fence_after();
           // (TMA writes and MMA reads are both async-proxy operations ordered by the barrier)
-          const uint32_t ha = sbase + (uint32_t)s * Lay.stage_bytes;
-          for (int j = 0; j < nt; ++j) {
-            const uint32_t ea = ha + Lay.h_bytes + (uint32_t)j * Lay.e_bytes;
-            const uint32_t d_tmem = tmem + (uint32_t)(acc * 256 + j * R);
+          const int kb0 = g * KBS, kbn = min(KBS, KB - kb0);
+          for (int kk = 0; kk < kbn; ++kk) {
+            const int kb = kb0 + kk;
+            const uint32_t ha = sbase + (uint32_t)s * Lay.stage_bytes + (uint32_t)kk * Lay.sub_bytes;
+            for (int j = 0; j < nt; ++j) {
+              const uint32_t ea = ha + Lay.h_bytes + (uint32_t)j * Lay.e_bytes;
+              const uint32_t d_tmem = tmem + (uint32_t)(acc * 256 + j * R);
 #pragma unroll
-            for (int k = 0; k < kTcKB / 16; ++k)  // 16 BF16 = 32 bytes along K per instruction
-              mma_bf16(d_tmem, sw128_desc(ha + 32u * k), sw128_desc(ea + 32u * k), idesc,
-                       (uint32_t)((kb | k) != 0));
+              for (int k = 0; k < kTcKB / 16; ++k)  // 16 BF16 = 32 bytes along K per instruction
+                mma_bf16(d_tmem, sw128_desc(ha + 32u * k), sw128_desc(ea + 32u * k), idesc,
+                         (uint32_t)((kb | k) != 0));
+            }
           }
           mma_commit(&empty[s]);  // the stage is free once these MMAs have read it
           issued = true;
@@ -497,14 +523,18 @@ cudaError_t launch_kernel(const CUtensorMap& mE, const CUtensorMap& mH, TcParams
                           cudaStream_t st) {
   const bool keys = p.out_keys != nullptr, sample = p.sample != 0;
   const int wave = keys ? 1 : kTcWave;
-  int S = kTcMaxStages;
-  for (; S >= 2; --S)
-    if (tc_layout(p.qrows, p.copies, p.tile_rows, wave, sample, S).dyn <= kTcSmemMax) break;
+  int S = 0;
+  for (;;) {  // the most stages that fit at this many K-blocks a stage; fewer K-blocks if not two
+    for (S = kTcMaxStages; S >= 2; --S)
+      if (tc_layout(p.qrows, p.copies, p.tile_rows, wave, sample, S, p.kbs).dyn <= kTcSmemMax) break;
+    if (S >= 2 || p.kbs <= 1) break;
+    p.kbs /= 2;
+  }
   if (S < 2) return cudaErrorInvalidValue;
   p.stages = S;
   auto kern = keys ? (sample ? k_tc_head<true, true> : k_tc_head<true, false>)
                    : (sample ? k_tc_head<false, true> : k_tc_head<false, false>);
-  const uint32_t dyn = tc_layout(p.qrows, p.copies, p.tile_rows, wave, sample, S).dyn;
+  const uint32_t dyn = tc_layout(p.qrows, p.copies, p.tile_rows, wave, sample, S, p.kbs).dyn;
   cudaError_t e = set_smem_attr(reinterpret_cast<const void*>(kern), dyn);
   if (e != cudaSuccess) return e;
   // every SM when the tiles are listed on the device; otherwise no more CTAs than tiles
@@ -825,6 +855,8 @@ cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms
   // keys of more than 32 queries (measured at the Llama-3.2-1B shape; below that the plain keys'
   // epilogue is light, and copies multiply the query bytes each stage brings in)
   tc_query_layout(p.B, !p.out_keys || p.sample || p.B > 32, p.qrows, p.copies);
+  // K-blocks per stage: the keys' small tiles fetch a row's consecutive K-blocks together
+  p.kbs = p.out_keys ? FH_TC_KEYS_KBS : FH_TC_HEAD_KBS;
   if (!make_map(&mE, A, p.d, p.rows, box) || !make_map(&mH, H, p.d, p.B, (uint32_t)p.qrows))
     return cudaErrorInvalidValue;
   return launch_kernel(mE, mH, p, num_sms, st);

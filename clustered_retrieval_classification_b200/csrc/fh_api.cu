@@ -56,6 +56,11 @@ struct Layout {
   size_t total = 0;
 };
 
+// The query masks (c words), the flags of the 128-row tiles of the cluster-major copy and the count of
+// the list that follows them: one region, zeroed before each batched Stage 2.
+int64_t tile_count_of(const fh_index_desc& D) { return (D.v + 127) / 128; }
+size_t qmask_region_bytes(const fh_index_desc& D) { return (size_t)D.c * 8 + (size_t)(tile_count_of(D) + 1) * 4; }
+
 Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
   const fh_index_desc& D = idx->desc;
   Layout L;
@@ -71,10 +76,11 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
     L.keys = take((size_t)B * D.c * 4);
     L.sel = take((size_t)B * p * 4);
     L.part = take((size_t)G * B * 8);
-    if (B > 1) {  // tensor-core Stage 2: per-cluster query masks, the selected clusters, arg-maxima
-      L.qmask = take((size_t)D.c * 8);
+    if (B > 1) {  // batched Stage 2: per-cluster query masks, then per-tile flags and the list's count
+      // (zeroed together before each call), the arg-maxima, the listed clusters or tiles
+      L.qmask = take(qmask_region_bytes(D));
       L.best = take((size_t)B * 8);
-      L.tiles = take((size_t)(std::max<int64_t>(D.c, (D.v + 127) / 128) + 1) * 4);
+      L.tiles = take((size_t)std::max<int64_t>(D.c, (D.v + 127) / 128) * 4);
     }
     if (B == 1 && fh::head1_threads(D.c) != 0) {  // the persistent batch-1 kernel's word table
       L.bucket = take((size_t)fh::kHead1Bins * fh::kHead1BucketCap * 8);
@@ -293,11 +299,11 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   }
   if (uni) {
     unsigned long long* qmask = reinterpret_cast<unsigned long long*>(base + L.qmask);
+    int32_t* count = reinterpret_cast<int32_t*>(qmask + D.c) + tile_count_of(D);
     int32_t* list = reinterpret_cast<int32_t*>(base + L.tiles);
-    if ((e = cudaMemsetAsync(qmask, 0, (size_t)D.c * 8, st)) != cudaSuccess ||
-        (e = cudaMemsetAsync(list, 0, 4, st)) != cudaSuccess)
+    if ((e = cudaMemsetAsync(qmask, 0, qmask_region_bytes(D), st)) != cudaSuccess)
       return cuda_fail(e, "memset");
-    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list + 1, list)) != cudaSuccess)
+    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count)) != cudaSuccess)
       return cuda_fail(e, "mask launch");
     fh::UnionParams up = {};
     up.E_perm = D.E_perm;
@@ -309,8 +315,8 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     up.b = D.b;
     up.B = B;
     up.qmask = qmask;
-    up.cl_list = list + 1;
-    up.cl_count = list;
+    up.cl_list = list;
+    up.cl_count = count;
     up.sample = sample;
     up.tau = tau;
     up.seed = seed;
@@ -327,8 +333,13 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     // Stage 2 on the tensor cores: every tile of the cluster-major copy that some query selected,
     // masked per (cluster, query), the arg-max of each query fused in.
     unsigned long long* qmask = reinterpret_cast<unsigned long long*>(base + L.qmask);
-    if ((e = cudaMemsetAsync(qmask, 0, (size_t)D.c * 8, st)) != cudaSuccess) return cuda_fail(e, "memset");
-    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st)) != cudaSuccess)
+    uint32_t* flags = reinterpret_cast<uint32_t*>(qmask + D.c);
+    int32_t* count = reinterpret_cast<int32_t*>(flags + tile_count_of(D));
+    int32_t* list = reinterpret_cast<int32_t*>(base + L.tiles);
+    if ((e = cudaMemsetAsync(qmask, 0, qmask_region_bytes(D), st)) != cudaSuccess)
+      return cuda_fail(e, "memset");
+    // the query masks and, as their clusters are first selected, the 128-row tiles that hold them
+    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count, flags, D.b, D.v, 128)) != cudaSuccess)
       return cuda_fail(e, "mask launch");
     fh::TcParams tp = {};
     tp.rows = D.v;
@@ -345,8 +356,8 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     tp.ticket = reinterpret_cast<unsigned long long*>(word_at(ws, kTcTicketOffset));
     tp.out_tok = out_tok;
     // the 128-row tiles that hold a cluster some query takes
-    tp.tile_list = reinterpret_cast<int32_t*>(base + L.tiles) + 1;
-    tp.tile_count = reinterpret_cast<int32_t*>(base + L.tiles);
+    tp.tile_list = list;
+    tp.tile_count = count;
     tp.status = status_of(ws);
     if ((e = fh::launch_tc_head(D.E_perm, H, tp, idx->num_sms, st)) != cudaSuccess)
       return cuda_fail(e, "tensor-core stage-2 launch");

@@ -12,7 +12,7 @@
 //   k_stage1_int4_mq<M,QB> INT4 for QB queries per block, each group decoded once      (Stage 1, INT4)
 //   k_select<KPT>    top-p per query                                                    (selection)
 //   k_build_qmask    per-cluster bit masks of the queries that selected it, and the list of
-//                    the clusters some query selected                                   (batched Stage 2)
+//                    the clusters (or 128-row tiles) some query selected                (batched Stage 2)
 //   k_union_rows<E>  the union of a batch's probe sets, each row read once for the batch (batched Stage 2)
 //   k_rows<E,MODE,KPT> candidates (fused selection or given sets) or all rows (dense):
 //                    dot, arg-max / Gumbel-max, partial results, last-block reduction   (Stage 2, dense)
@@ -904,21 +904,33 @@ cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int
 // qmask[cluster] |= 1 << q for every cluster in query q's probe set (qmask zeroed beforehand).
 // list (optional, with *count zeroed like qmask): the clusters with a nonzero mask, each appended once
 // by the query that sets its first bit (in no particular order).
+// Bit q of qmask[k]: query q selected cluster k.  The first selection of a cluster lists it (the
+// union Stage 2) or, with tile_flags, lists every tile_rows-row tile of the cluster-major copy it
+// overlaps that no earlier cluster listed (the tensor-core Stage 2; any order will do).
 __global__ void k_build_qmask(const int32_t* __restrict__ sel, int B, int p, unsigned long long* qmask,
-                              int32_t* list, int32_t* count) {
+                              int32_t* list, int32_t* count, uint32_t* tile_flags, int64_t b,
+                              int64_t rows, int tile_rows) {
   const int64_t n = (int64_t)B * p;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int32_t k = sel[i];
     const unsigned long long old = atomicOr(qmask + k, 1ull << (uint32_t)(i / p));
-    if (list && old == 0ull) list[atomicAdd(count, 1)] = k;
+    if (!list || old != 0ull) continue;
+    if (!tile_flags) {
+      list[atomicAdd(count, 1)] = k;
+    } else {
+      const int64_t r0 = (int64_t)k * b, r1 = (r0 + b < rows ? r0 + b : rows) - 1;
+      for (int64_t t = r0 / tile_rows; t <= r1 / tile_rows; ++t)
+        if (atomicExch(tile_flags + t, 1u) == 0u) list[atomicAdd(count, 1)] = (int32_t)t;
+    }
   }
 }
 
 cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
-                               cudaStream_t st, int32_t* list, int32_t* count) {
+                               cudaStream_t st, int32_t* list, int32_t* count, uint32_t* tile_flags,
+                               int64_t b, int64_t rows, int tile_rows) {
   const int64_t n = (int64_t)B * p;
   const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
-  k_build_qmask<<<blocks, 256, 0, st>>>(sel, B, p, qmask, list, count);
+  k_build_qmask<<<blocks, 256, 0, st>>>(sel, B, p, qmask, list, count, tile_flags, b, rows, tile_rows);
   return cudaGetLastError();
 }
 

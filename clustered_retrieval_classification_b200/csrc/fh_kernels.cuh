@@ -107,8 +107,8 @@ struct TcParams {
   int32_t* out_tok;                // B, or null
   float* out_logits;               // B x rows indexed by token, or null
   float* out_keys;                 // B x rows: write the raw products (Stage-1 keys) instead
-  int32_t* tile_list;              // rows/128 scratch: or stream the 128-row tiles some query takes
-  int32_t* tile_count;             // 1 scratch word: their number (both lists null: every tile)
+  int32_t* tile_list;              // the 128-row tiles some query takes, any order (null: every tile)
+  int32_t* tile_count;             // their number (device word, written before the launch)
   uint32_t* status;
   int n_tiles, tile_rows, stages;  // set by the launcher
   int qrows, copies;               // query rows of one copy in the MMA's 128 rows, copies (launcher)
@@ -137,8 +137,13 @@ bool union_supported(int elem, int64_t d, int64_t v, int64_t b, int B, int num_s
 cudaError_t launch_union_rows(const UnionParams& prm, int elem, int num_sms, cudaStream_t st);
 bool tc_supported(int elem, int64_t d, int B);
 cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms, cudaStream_t st);
+// qmask: c words, zero before the call; list/count (count zero before the call): the clusters some
+// query selected, or with tile_flags (zero before the call) the tile_rows-row tiles of the
+// cluster-major copy (rows rows, b per cluster) that hold one.
 cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
-                               cudaStream_t st, int32_t* list = nullptr, int32_t* count = nullptr);
+                               cudaStream_t st, int32_t* list = nullptr, int32_t* count = nullptr,
+                               uint32_t* tile_flags = nullptr, int64_t b = 0, int64_t rows = 0,
+                               int tile_rows = 128);
 bool tc_int4_supported(int64_t d, int B, const void* scales);
 // INT4 Stage-1 keys on the tensor cores: out_keys[q][k] = Σ_j q4[k][j]·scale[k][j/32]·h_q[j] (or the
 // Gumbel key when sample != 0), dequantised to fp16 in shared memory (fh_tc.cu).

@@ -457,39 +457,6 @@ __global__ void __launch_bounds__(kTcHeadThreads, 1)
   }
 }
 
-// The 128-row tiles of which some query takes a cluster, in ascending order; one block.
-__global__ void __launch_bounds__(1024) k_selected_tiles(const unsigned long long* __restrict__ qmask,
-                                                         int64_t rows, int64_t b, int n_tiles,
-                                                         int32_t* list, int32_t* count) {
-  __shared__ int base_s;
-  __shared__ int wsum[32];
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  if (threadIdx.x == 0) base_s = 0;
-  __syncthreads();
-  for (int t0 = 0; t0 < n_tiles; t0 += blockDim.x) {
-    const int t = t0 + (int)threadIdx.x;
-    bool act = false;
-    if (t < n_tiles) {
-      const int64_t r0 = (int64_t)t * kTcRows, r1 = min(r0 + kTcRows, rows) - 1;
-      for (int64_t cl = r0 / b; cl <= r1 / b && !act; ++cl) act = qmask[cl] != 0ull;
-    }
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, act);
-    if (lane == 0) wsum[wid] = __popc(bal);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
-      before += i < wid ? wsum[i] : 0;
-      total += wsum[i];
-    }
-    if (act) list[base_s + before + __popc(bal & ((1u << lane) - 1u))] = t;
-    __syncthreads();
-    if (threadIdx.x == 0) base_s += total;
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) *count = base_s;
-}
-
-
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -844,12 +811,8 @@ cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms
   p.tile_rows = (p.out_keys && (p.rows + 63) / 64 <= num_sms) ? 64 : kTcRows;
   p.n_tiles = (int)((p.rows + p.tile_rows - 1) / p.tile_rows);
   uint32_t box = (uint32_t)p.tile_rows;
-  if (p.tile_list) {  // the selected tiles, listed on the device (the kernel reads their count)
-    if (!p.qmask) return cudaErrorInvalidValue;
-    k_selected_tiles<<<1, 1024, 0, st>>>(p.qmask, p.rows, p.b, p.n_tiles, p.tile_list, p.tile_count);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  // listed tiles (the kernel reads their count on the device): filled by the query-mask builder
+  if (p.tile_list && (!p.qmask || !p.tile_count)) return cudaErrorInvalidValue;
   CUtensorMap mE, mH;
   // copies of the queries where the epilogue bounds the kernel: the head modes, sampled keys, and
   // keys of more than 32 queries (measured at the Llama-3.2-1B shape; below that the plain keys'

@@ -133,3 +133,51 @@ def test_workspace_reuse_across_batch_sizes(fh, orc, mid, mid_index):
         decided = o["tok_margin"] > MARGIN
         assert np.array_equal(tok[decided], o["tok"][decided])
     fh.ws_status(ws)
+
+
+STRADDLE = synth.scaled(synth.CONFIGS["llama"], v=12000, c=500, d=256, p=40, name="llama-b24")
+
+
+@pytest.mark.parametrize("B", [20, 33])
+@pytest.mark.parametrize("sample", [False, True])
+def test_flashhead_batched_clusters_straddle_tiles(fh, orc, B, sample):
+    """b = 24 rows a cluster: clusters straddle the 128-row tiles of the cluster-major copy, so the
+    tile list must hold every tile a selected cluster overlaps (the last tile is partial, v = 12000);
+    the tensor-core Stage 2 against the oracle."""
+    idx = synth.make_index(STRADDLE)
+    H = synth.make_queries(STRADDLE, B)
+    I = fh.index_from_host(idx.E, idx.C, idx.C2T, "bf16")
+    cfg = idx.cfg
+    Hd = dev(H, "bf16")
+    if sample:
+        tok = fh.head_sample(I, Hd, cfg.p, 0.8, synth.SAMPLE_SEED, 7).cpu().numpy()
+    else:
+        tok = fh.head_greedy(I, Hd, cfg.p).cpu().numpy()
+    o = orc.head(idx, H, cfg.p, sample=sample, tau=0.8, seed=synth.SAMPLE_SEED, step=7)
+    decided = (o["set_margin"] > MARGIN) & (o["tok_margin"] > MARGIN)
+    assert np.array_equal(tok[decided], o["tok"][decided]), np.nonzero(tok != o["tok"])
+    assert decided.sum() >= max(1, B // 4)
+    # every token is a candidate of its query: from a cluster the oracle selected, or one within the
+    # margin of the threshold
+    s = orc.stage1_scores(idx.C, cfg.dtype, H, cfg.c, cfg.d)
+    keys = orc.gumbel_keys(s, 0.8, synth.SAMPLE_SEED, 7, 0) if sample else s
+    for q in range(B):
+        k = np.sort(keys[q])[::-1]
+        thr = 0.5 * (k[cfg.p - 1] + k[cfg.p])
+        allowed = set(np.asarray(o["sel"][q]).tolist()) | set(np.nonzero(np.abs(keys[q] - thr) <= MARGIN)[0].tolist())
+        assert any(int(tok[q]) in idx.C2T[cl] for cl in allowed), q
+
+
+@pytest.mark.parametrize("d", [200, 320])
+@pytest.mark.parametrize("B", [2, 40])
+def test_stage1_keys_partial_stage(fh, orc, d, B):
+    """Tensor-core Stage-1 keys stream several consecutive K-blocks per pipeline stage; d = 320 (five
+    64-column K-blocks: a stage of four, then one of one) and d = 200 (a partial last K-block) check
+    the partial stages element by element."""
+    idx = synth.random_index(v=4000, d=d, c=500, seed=41, dtype="bf16")
+    rng = np.random.default_rng(43)
+    H = synth.store((rng.standard_normal((B, d)) * 0.5).astype(np.float32), "bf16")
+    I = fh.index_from_host(idx.E, idx.C, idx.C2T, "bf16")
+    g = fh.stage1_scores(I, dev(H, "bf16")).cpu().numpy()
+    o = orc.stage1_scores(idx.C, "bf16", H, idx.c, d)
+    assert np.abs(g - o).max() <= LOGIT_TOL

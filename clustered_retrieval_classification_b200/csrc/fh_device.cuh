@@ -25,15 +25,24 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // acc += Σ_i a_i·b_i over the 8 BF16 values of two 16-byte chunks, in element order.
+// c + a_lo·b_lo, then + a_hi·b_hi, for two pairs of BF16 patterns: the mixed-precision FMA multiplies
+// the BF16 inputs and adds in FP32 with one rounding, the value of fmaf on the widened inputs (the
+// product of two BF16 values is exact in FP32) without the two widening operations per element.
+__device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t b, float c) {
+  float r;
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t.reg .f32 t;\n\t"
+      "mov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 t, al, bl, %3;\n\tfma.rn.f32.bf16 %0, ah, bh, t;\n\t}"
+      : "=f"(r)
+      : "r"(a), "r"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ float dot8_bf16(const uint4& a, const uint4& b, float acc) {
-  acc = fmaf(bf16_lo(a.x), bf16_lo(b.x), acc);
-  acc = fmaf(bf16_hi(a.x), bf16_hi(b.x), acc);
-  acc = fmaf(bf16_lo(a.y), bf16_lo(b.y), acc);
-  acc = fmaf(bf16_hi(a.y), bf16_hi(b.y), acc);
-  acc = fmaf(bf16_lo(a.z), bf16_lo(b.z), acc);
-  acc = fmaf(bf16_hi(a.z), bf16_hi(b.z), acc);
-  acc = fmaf(bf16_lo(a.w), bf16_lo(b.w), acc);
-  acc = fmaf(bf16_hi(a.w), bf16_hi(b.w), acc);
+  acc = fma2_bf16(a.x, b.x, acc);
+  acc = fma2_bf16(a.y, b.y, acc);
+  acc = fma2_bf16(a.z, b.z, acc);
+  acc = fma2_bf16(a.w, b.w, acc);
   return acc;
 }
 

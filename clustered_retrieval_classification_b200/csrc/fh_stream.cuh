@@ -23,10 +23,10 @@ __device__ __forceinline__ float row_dot_partial(uint32_t row_s, uint32_t h_s, i
     const uint4 a = lds_v4(row_s + ch * 16);
     const uint4 h = lds_v4(h_s + ch * 16);
     if (ELEM == 1) {
-      a0 = fmaf(bf16_hi(a.x), bf16_hi(h.x), fmaf(bf16_lo(a.x), bf16_lo(h.x), a0));
-      a1 = fmaf(bf16_hi(a.y), bf16_hi(h.y), fmaf(bf16_lo(a.y), bf16_lo(h.y), a1));
-      a2 = fmaf(bf16_hi(a.z), bf16_hi(h.z), fmaf(bf16_lo(a.z), bf16_lo(h.z), a2));
-      a3 = fmaf(bf16_hi(a.w), bf16_hi(h.w), fmaf(bf16_lo(a.w), bf16_lo(h.w), a3));
+      a0 = fma2_bf16(a.x, h.x, a0);
+      a1 = fma2_bf16(a.y, h.y, a1);
+      a2 = fma2_bf16(a.z, h.z, a2);
+      a3 = fma2_bf16(a.w, h.w, a3);
     } else {
       a0 = fmaf(__uint_as_float(a.x), __uint_as_float(h.x), a0);
       a1 = fmaf(__uint_as_float(a.y), __uint_as_float(h.y), a1);
@@ -38,8 +38,8 @@ __device__ __forceinline__ float row_dot_partial(uint32_t row_s, uint32_t h_s, i
 }
 
 // Lane-partial dot products of one staged row with QB staged query vectors (QB rows of row bytes
-// from h_s; the first nq are live): the row's chunk is read and widened once for all queries, and
-// the QB sums are independent FMA chains.
+// from h_s; the first nq are live): the row's chunk is read once for all queries, and the QB sums
+// are independent FMA chains.
 template <int ELEM, int QB>
 __device__ __forceinline__ void row_dot_partial_multi(uint32_t row_s, uint32_t h_s, uint32_t row_bytes,
                                                       int nch, int nq, int lane, float (&acc)[QB]) {
@@ -49,10 +49,7 @@ __device__ __forceinline__ void row_dot_partial_multi(uint32_t row_s, uint32_t h
   for (int ch = lane; ch < nch; ch += 32) {
     const uint4 a = lds_v4(row_s + ch * 16);
     float af[8];
-    if (ELEM == 1) {
-      af[0] = bf16_lo(a.x); af[1] = bf16_hi(a.x); af[2] = bf16_lo(a.y); af[3] = bf16_hi(a.y);
-      af[4] = bf16_lo(a.z); af[5] = bf16_hi(a.z); af[6] = bf16_lo(a.w); af[7] = bf16_hi(a.w);
-    } else {
+    if (ELEM != 1) {
       af[0] = __uint_as_float(a.x); af[1] = __uint_as_float(a.y);
       af[2] = __uint_as_float(a.z); af[3] = __uint_as_float(a.w);
     }
@@ -62,10 +59,10 @@ __device__ __forceinline__ void row_dot_partial_multi(uint32_t row_s, uint32_t h
         const uint4 h = lds_v4(h_s + (uint32_t)q * row_bytes + ch * 16);
         if (ELEM == 1) {
           float t = acc[q];
-          t = fmaf(af[0], bf16_lo(h.x), t); t = fmaf(af[1], bf16_hi(h.x), t);
-          t = fmaf(af[2], bf16_lo(h.y), t); t = fmaf(af[3], bf16_hi(h.y), t);
-          t = fmaf(af[4], bf16_lo(h.z), t); t = fmaf(af[5], bf16_hi(h.z), t);
-          t = fmaf(af[6], bf16_lo(h.w), t); t = fmaf(af[7], bf16_hi(h.w), t);
+          t = fma2_bf16(a.x, h.x, t);
+          t = fma2_bf16(a.y, h.y, t);
+          t = fma2_bf16(a.z, h.z, t);
+          t = fma2_bf16(a.w, h.w, t);
           acc[q] = t;
         } else {
           float t = acc[q];

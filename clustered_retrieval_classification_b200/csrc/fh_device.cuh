@@ -26,8 +26,8 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 
 // acc += Σ_i a_i·b_i over the 8 BF16 values of two 16-byte chunks, in element order.
 // c + a_lo·b_lo, then + a_hi·b_hi, for two pairs of BF16 patterns: the mixed-precision FMA multiplies
-// the BF16 inputs and adds in FP32 with one rounding, the value of fmaf on the widened inputs (the
-// product of two BF16 values is exact in FP32) without the two widening operations per element.
+// the BF16 inputs and adds in FP32 with one rounding, as fmaf does on the inputs widened to FP32 (an
+// exact widening), so the value is the same, without the two widening operations per element.
 __device__ __forceinline__ float fma2_bf16(uint32_t a, uint32_t b, float c) {
   float r;
   asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t.reg .f32 t;\n\t"

@@ -452,8 +452,80 @@ __host__ __device__ inline UnionSmemLayout union_layout(uint32_t row_bytes, int 
   return L;
 }
 
-template <int ELEM, int NW>
-__global__ void __launch_bounds__(NW * 32) k_union_rows(const UnionParams prm, int K, int rows_max, int cl_max) {
+// Lane-partial dot products of a row held in registers (chunk lane + 32·j in ra[j], the first RCH
+// chunks of the lane) with one or two staged query vectors: the same four chains, in the same order,
+// as row_dot_partial, so the sums are bit-identical to it.
+template <int ELEM, int RCH>
+__device__ __forceinline__ float cached_dot_partial(const uint4 (&ra)[RCH], uint32_t h_s, int nch, int lane) {
+  float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
+#pragma unroll
+  for (int j = 0; j < RCH; ++j) {
+    const int ch = lane + 32 * j;
+    if (ch < nch) {
+      const uint4 h = lds_v4(h_s + ch * 16);
+      if (ELEM == kBF16) {
+        a0 = fma2_bf16(ra[j].x, h.x, a0);
+        a1 = fma2_bf16(ra[j].y, h.y, a1);
+        a2 = fma2_bf16(ra[j].z, h.z, a2);
+        a3 = fma2_bf16(ra[j].w, h.w, a3);
+      } else {
+        a0 = fmaf(__uint_as_float(ra[j].x), __uint_as_float(h.x), a0);
+        a1 = fmaf(__uint_as_float(ra[j].y), __uint_as_float(h.y), a1);
+        a2 = fmaf(__uint_as_float(ra[j].z), __uint_as_float(h.z), a2);
+        a3 = fmaf(__uint_as_float(ra[j].w), __uint_as_float(h.w), a3);
+      }
+    }
+  }
+  return (a0 + a1) + (a2 + a3);
+}
+
+template <int ELEM, int RCH>
+__device__ __forceinline__ void cached_dot2_partial(const uint4 (&ra)[RCH], uint32_t h0, uint32_t h1, int nch,
+                                                    int lane, float& z0, float& z1) {
+  float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f, b0 = 0.0f, b1 = 0.0f, b2 = 0.0f, b3 = 0.0f;
+#pragma unroll
+  for (int j = 0; j < RCH; ++j) {
+    const int ch = lane + 32 * j;
+    if (ch < nch) {
+      const uint4 x = lds_v4(h0 + ch * 16), y = lds_v4(h1 + ch * 16);
+      if (ELEM == kBF16) {
+        a0 = fma2_bf16(ra[j].x, x.x, a0);
+        a1 = fma2_bf16(ra[j].y, x.y, a1);
+        a2 = fma2_bf16(ra[j].z, x.z, a2);
+        a3 = fma2_bf16(ra[j].w, x.w, a3);
+        b0 = fma2_bf16(ra[j].x, y.x, b0);
+        b1 = fma2_bf16(ra[j].y, y.y, b1);
+        b2 = fma2_bf16(ra[j].z, y.z, b2);
+        b3 = fma2_bf16(ra[j].w, y.w, b3);
+      } else {
+        a0 = fmaf(__uint_as_float(ra[j].x), __uint_as_float(x.x), a0);
+        a1 = fmaf(__uint_as_float(ra[j].y), __uint_as_float(x.y), a1);
+        a2 = fmaf(__uint_as_float(ra[j].z), __uint_as_float(x.z), a2);
+        a3 = fmaf(__uint_as_float(ra[j].w), __uint_as_float(x.w), a3);
+        b0 = fmaf(__uint_as_float(ra[j].x), __uint_as_float(y.x), b0);
+        b1 = fmaf(__uint_as_float(ra[j].y), __uint_as_float(y.y), b1);
+        b2 = fmaf(__uint_as_float(ra[j].z), __uint_as_float(y.z), b2);
+        b3 = fmaf(__uint_as_float(ra[j].w), __uint_as_float(y.w), b3);
+      }
+    }
+  }
+  z0 = (a0 + a1) + (a2 + a3);
+  z1 = (b0 + b1) + (b2 + b3);
+}
+
+// Two warp sums with their shuffles interleaved (each the same butterfly as warp_sum).
+__device__ __forceinline__ void warp_sum2(float& x, float& y) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float tx = __shfl_xor_sync(0xFFFFFFFFu, x, off);
+    const float ty = __shfl_xor_sync(0xFFFFFFFFu, y, off);
+    x += tx;
+    y += ty;
+  }
+}
+
+template <int ELEM, int NW, int RCH>
+__global__ void __launch_bounds__(NW * 32, 1) k_union_rows(const UnionParams prm, int K, int rows_max, int cl_max) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t row_bytes = (uint32_t)(prm.d * (ELEM == kBF16 ? 2 : 4));
@@ -509,6 +581,24 @@ __global__ void __launch_bounds__(NW * 32) k_union_rows(const UnionParams prm, i
 
   const uint32_t hs_addr = smem_addr(hs);
   unsigned long long best0 = 0ull, best1 = 0ull;  // queries lane and lane + 32
+  auto fold = [&](int q, float z, uint32_t tok) {
+    if (lane == (q & 31)) {
+      float val = z;
+      if (prm.sample)
+        val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, 1u, tok));
+      const unsigned long long pk = pack_best(val, tok);
+      if (q < 32) best0 = pk > best0 ? pk : best0;
+      else best1 = pk > best1 ? pk : best1;
+    }
+  };
+  auto refill = [&](int n, int slot) {  // the slot's next row, once every lane is done reading it
+    __syncwarp();
+    if (lane == 0 && n + K < nw) {
+      fence_proxy_async_smem();
+      issue_row(ring_w + (size_t)slot * row_bytes, src(first + (uint32_t)(NW * (n + K))), row_bytes,
+                &bars_w[slot]);
+    }
+  };
   for (int n = 0; n < nw; ++n) {
     const int slot = (int)(n % K);
     if (!mbar_wait(&bars_w[slot], (uint32_t)((n / K) & 1), prm.status)) {
@@ -520,24 +610,41 @@ __global__ void __launch_bounds__(NW * 32) k_union_rows(const UnionParams prm, i
     const uint32_t row_s = smem_addr(ring_w + (size_t)slot * row_bytes);
     const uint32_t tok = (uint32_t)tok_s[i - lo];
     unsigned long long mk = msk_s[i / b - c_lo];
-    while (mk) {  // the same queries in every lane
-      const int q = __ffsll((long long)mk) - 1;
-      mk &= mk - 1;
-      const float z = warp_sum(row_dot_partial<ELEM>(row_s, hs_addr + (uint32_t)q * row_bytes, nch, lane));
-      if (lane == (q & 31)) {
-        float val = z;
-        if (prm.sample)
-          val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, 1u, tok));
-        const unsigned long long pk = pack_best(val, tok);
-        if (q < 32) best0 = pk > best0 ? pk : best0;
-        else best1 = pk > best1 ? pk : best1;
+    if constexpr (RCH > 0) {
+      // the row into registers, its slot refilled at once, then the cluster's queries two at a time
+      uint4 ra[RCH];
+#pragma unroll
+      for (int j = 0; j < RCH; ++j) {
+        const int ch = lane + 32 * j;
+        ra[j] = ch < nch ? lds_v4(row_s + ch * 16) : make_uint4(0u, 0u, 0u, 0u);
       }
-    }
-    __syncwarp();
-    if (lane == 0 && n + K < nw) {
-      fence_proxy_async_smem();
-      issue_row(ring_w + (size_t)slot * row_bytes, src(first + (uint32_t)(NW * (n + K))), row_bytes,
-                &bars_w[slot]);
+#pragma unroll
+      for (int j = 0; j < RCH; ++j)  // the loads have returned before the slot is handed back
+        asm volatile("" : "+r"(ra[j].x), "+r"(ra[j].y), "+r"(ra[j].z), "+r"(ra[j].w));
+      refill(n, slot);
+      while (mk) {  // the same queries in every lane
+        const int q0 = __ffsll((long long)mk) - 1;
+        mk &= mk - 1;
+        if (mk) {
+          const int q1 = __ffsll((long long)mk) - 1;
+          mk &= mk - 1;
+          float z0, z1;
+          cached_dot2_partial<ELEM, RCH>(ra, hs_addr + (uint32_t)q0 * row_bytes, hs_addr + (uint32_t)q1 * row_bytes,
+                                         nch, lane, z0, z1);
+          warp_sum2(z0, z1);
+          fold(q0, z0, tok);
+          fold(q1, z1, tok);
+        } else {
+          fold(q0, warp_sum(cached_dot_partial<ELEM, RCH>(ra, hs_addr + (uint32_t)q0 * row_bytes, nch, lane)), tok);
+        }
+      }
+    } else {
+      while (mk) {  // the same queries in every lane
+        const int q = __ffsll((long long)mk) - 1;
+        mk &= mk - 1;
+        fold(q, warp_sum(row_dot_partial<ELEM>(row_s, hs_addr + (uint32_t)q * row_bytes, nch, lane)), tok);
+      }
+      refill(n, slot);
     }
   }
 
@@ -960,19 +1067,31 @@ cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaSt
   return cudaGetLastError();
 }
 
-// Warps and ring slots of the union kernel at batch B: 16 warps when two slots each fit beside the
-// query vectors (more rows in flight and more warps to hide the dot products' latency), else 8;
-// 0 slots: the query vectors leave no room for a ring of two.
+// Warps and ring slots of the union kernel at batch B: the most warps (16, 12, 8) for which a ring
+// of two slots each fits beside the query vectors, with as many slots as fit, within the opt-in
+// shared memory of a block less the kernel's static arrays; 0 slots: the query vectors leave no room
+// for a ring of two.  More warps beat more rows in flight (Llama shape, greedy, µs a call at 8 / 12 /
+// 16 queries: 16 warps × 2 slots 69.2 / 84.2 / 99.5; the split with the most rows in flight, 8 × 5,
+// 8 × 5 and 12 × 3, 90.5 / 113.3 / 109.6).
+#ifndef FH_UNION_SMEM_CAP
+#define FH_UNION_SMEM_CAP (227u * 1024u)
+#endif
+#ifndef FH_UNION_WARPS
+#define FH_UNION_WARPS 0  // 16, 12 or 8 to fix the warp count
+#endif
 static int union_slots(uint32_t row_bytes, int B, int rows_max, int cl_max, int* nw, size_t* smem) {
-  for (int NW : {16, 8})
+  for (int NW : {16, 12, 8}) {
+    if (FH_UNION_WARPS != 0 && NW != FH_UNION_WARPS) continue;
+    const uint32_t cap = FH_UNION_SMEM_CAP - (uint32_t)NW * 64u * 8u - 128u;  // blk_best, is_last
     for (int K = 128 / NW - 1; K >= 2; --K) {
       const UnionSmemLayout L = union_layout(row_bytes, B, NW, K, rows_max, cl_max);
-      if (L.total <= 200u * 1024u) {
+      if (L.total <= cap) {
         *nw = NW;
         *smem = L.total;
         return K;
       }
     }
+  }
   return 0;
 }
 
@@ -980,8 +1099,8 @@ bool union_supported(int elem, int64_t d, int64_t v, int64_t b, int B, int num_s
   if (B < 1 || B > 64) return false;
   const uint32_t row_bytes = (uint32_t)(d * (elem == kBF16 ? 2 : 4));
   const int rows_max = (int)((v + num_sms - 1) / num_sms);
-  size_t smem;
-  int nw;
+  size_t smem = 0;
+  int nw = 0;
   return union_slots(row_bytes, B, rows_max, (int)(rows_max / b + 2), &nw, &smem) >= 2;
 }
 
@@ -991,20 +1110,29 @@ cudaError_t launch_union_rows(const UnionParams& prm, int elem, int num_sms, cud
   const int rows_max = (int)((prm.v + G - 1) / G);  // the union has at most v rows
   const int cl_max = (int)(rows_max / prm.b + 2);
   size_t smem = 0;
-  int NW = 8;
+  int NW = 0;
   const int K = union_slots(row_bytes, prm.B, rows_max, cl_max, &NW, &smem);
   if (K < 2) return cudaErrorInvalidValue;
+  // rows of up to 256 16-byte chunks (4 KB) are held in registers, 8 chunks a lane
+  const bool cached = row_bytes <= 256u * 16u;
   cudaError_t e;
-#define FH_UN(EL, W)                                                             \
-  do {                                                                           \
-    if ((e = set_smem(k_union_rows<EL, W>, smem)) != cudaSuccess) return e;      \
-    k_union_rows<EL, W><<<G, W * 32, smem, st>>>(prm, K, rows_max, cl_max);      \
+#define FH_UN(EL, W, R)                                                             \
+  do {                                                                              \
+    if ((e = set_smem(k_union_rows<EL, W, R>, smem)) != cudaSuccess) return e;      \
+    k_union_rows<EL, W, R><<<G, W * 32, smem, st>>>(prm, K, rows_max, cl_max);      \
+  } while (0)
+#define FH_UN_W(EL, R)                 \
+  do {                                 \
+    if (NW == 16) FH_UN(EL, 16, R);    \
+    else if (NW == 12) FH_UN(EL, 12, R); \
+    else FH_UN(EL, 8, R);              \
   } while (0)
   if (elem == kBF16) {
-    if (NW == 16) FH_UN(kBF16, 16); else FH_UN(kBF16, 8);
+    if (cached) FH_UN_W(kBF16, 8); else FH_UN_W(kBF16, 0);
   } else {
-    if (NW == 16) FH_UN(kF32, 16); else FH_UN(kF32, 8);
+    if (cached) FH_UN_W(kF32, 8); else FH_UN_W(kF32, 0);
   }
+#undef FH_UN_W
 #undef FH_UN
   return cudaGetLastError();
 }

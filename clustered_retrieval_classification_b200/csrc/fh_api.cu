@@ -77,7 +77,7 @@ Layout layout_for(const fh_index* idx, int op, int B, int p, int T, int64_t N) {
     L.sel = take((size_t)B * p * 4);
     L.part = take((size_t)G * B * 8);
     if (B > 1) {  // batched Stage 2: per-cluster query masks, then per-tile flags and the list's count
-      // (zeroed together before each call), the arg-maxima, the listed clusters or tiles
+      // (cleared together by each call's selection kernel), the arg-maxima, the listed clusters or tiles
       L.qmask = take(qmask_region_bytes(D));
       L.best = take((size_t)B * 8);
       L.tiles = take((size_t)std::max<int64_t>(D.c, (D.v + 127) / 128) * 4);
@@ -256,6 +256,10 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   const bool uni = B > 1 && B <= kUnionMaxBatch && !per_cand && D.E_perm != nullptr &&
                    fh::union_supported(elem, D.d, D.v, D.b, B, idx->num_sms);
   const bool tc = !uni && tc_eligible(idx, B, kTcMinBatchDense) && !per_cand && D.E_perm != nullptr;
+  // the query masks, the list's count and the tile flags of a batched Stage 2 are cleared by the
+  // selection kernel that precedes their builder
+  void* mask_region = (uni || tc) ? static_cast<void*>(base + L.qmask) : nullptr;
+  const size_t mask_bytes = (uni || tc) ? qmask_region_bytes(D) : 0;
   if ((tc || uni) && tc_eligible(idx, B, kTcMinBatchStage1) && s1fmt(idx) == FH_STAGE1_DENSE) {
     // Stage 1 on the tensor cores too: keys[q][k] = C[k]·h_q (+ the Gumbel term when sampling)
     fh::TcParams tp = {};
@@ -271,7 +275,7 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     tp.status = status_of(ws);
     if ((e = fh::launch_tc_head(D.C, H, tp, idx->num_sms, st)) != cudaSuccess)
       return cuda_fail(e, "tensor-core stage-1 launch");
-    if ((e = fh::launch_select(keys, sel, B, D.c, p, st)) != cudaSuccess)
+    if ((e = fh::launch_select(keys, sel, B, D.c, p, st, mask_region, mask_bytes)) != cudaSuccess)
       return cuda_fail(e, "select launch");
     if (dbg && dbg->sel &&
         (e = cudaMemcpyAsync(dbg->sel, sel, (size_t)B * p * 4, cudaMemcpyDeviceToDevice, st)) !=
@@ -289,7 +293,7 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     e = launch_stage1_for(idx, s1, st);
     if (e != cudaSuccess) return cuda_fail(e, "stage-1 launch");
     if (!fused) {
-      if ((e = fh::launch_select(keys, sel, B, D.c, p, st)) != cudaSuccess)
+      if ((e = fh::launch_select(keys, sel, B, D.c, p, st, mask_region, mask_bytes)) != cudaSuccess)
         return cuda_fail(e, "select launch");
       if (dbg && dbg->sel &&
           (e = cudaMemcpyAsync(dbg->sel, sel, (size_t)B * p * 4, cudaMemcpyDeviceToDevice, st)) !=
@@ -301,8 +305,6 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     unsigned long long* qmask = reinterpret_cast<unsigned long long*>(base + L.qmask);
     int32_t* count = reinterpret_cast<int32_t*>(qmask + D.c) + tile_count_of(D);
     int32_t* list = reinterpret_cast<int32_t*>(base + L.tiles);
-    if ((e = cudaMemsetAsync(qmask, 0, qmask_region_bytes(D), st)) != cudaSuccess)
-      return cuda_fail(e, "memset");
     if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count)) != cudaSuccess)
       return cuda_fail(e, "mask launch");
     fh::UnionParams up = {};
@@ -336,8 +338,6 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     uint32_t* flags = reinterpret_cast<uint32_t*>(qmask + D.c);
     int32_t* count = reinterpret_cast<int32_t*>(flags + tile_count_of(D));
     int32_t* list = reinterpret_cast<int32_t*>(base + L.tiles);
-    if ((e = cudaMemsetAsync(qmask, 0, qmask_region_bytes(D), st)) != cudaSuccess)
-      return cuda_fail(e, "memset");
     // the query masks and, as their clusters are first selected, the 128-row tiles that hold them
     if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count, flags, D.b, D.v, 128)) != cudaSuccess)
       return cuda_fail(e, "mask launch");

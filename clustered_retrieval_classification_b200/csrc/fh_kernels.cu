@@ -294,10 +294,14 @@ __global__ void k_cand_logits(const void* E, int64_t d, const void* H, int B, co
 
 // ============================================================================ selection kernel
 
+// zero / zero_words (optional): a region the blocks clear for the kernel that follows (the query
+// masks of a batched Stage 2), which saves it a separate memset.
 template <int NT, int KPT>
-__global__ void __launch_bounds__(NT) k_select(const float* keys, int32_t* sel, int64_t c, int p) {
+__global__ void __launch_bounds__(NT) k_select(const float* keys, int32_t* sel, int64_t c, int p,
+                                               uint32_t* zero, int zero_words) {
   __shared__ SelectSmem<NT> sm;
   const int q = blockIdx.x;
+  for (int i = q * NT + (int)threadIdx.x; i < zero_words; i += (int)gridDim.x * NT) zero[i] = 0u;
   uint32_t key[KPT];
   load_key_images<KPT>(keys + (size_t)q * c, (int)c, key);
   block_select_topp<NT, KPT>(key, (int)c, p, sm, sel + (size_t)q * p);
@@ -999,13 +1003,30 @@ cudaError_t launch_gumbel_keys(const float* s, float* keys, int B, int64_t c, fl
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p, cudaStream_t st) {
-  if (c <= 512 * 4) k_select<512, 4><<<B, 512, 0, st>>>(keys, sel, c, p);
-  else if (c <= 512 * 8) k_select<512, 8><<<B, 512, 0, st>>>(keys, sel, c, p);
-  else if (c <= 512 * 16) k_select<512, 16><<<B, 512, 0, st>>>(keys, sel, c, p);
-  else if (c <= 512 * 32) k_select<512, 32><<<B, 512, 0, st>>>(keys, sel, c, p);
-  else k_select<1024, 32><<<B, 1024, 0, st>>>(keys, sel, c, p);
+cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p, cudaStream_t st,
+                          void* zero, size_t zero_bytes) {
+  uint32_t* z = static_cast<uint32_t*>(zero);
+  const int zw = zero ? (int)(zero_bytes / 4) : 0;  // a few hundred KB at most
+  if (c <= 512 * 4) k_select<512, 4><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
+  else if (c <= 512 * 8) k_select<512, 8><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
+  else if (c <= 512 * 16) k_select<512, 16><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
+  else if (c <= 512 * 32) k_select<512, 32><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
+  else k_select<1024, 32><<<B, 1024, 0, st>>>(keys, sel, c, p, z, zw);
   return cudaGetLastError();
+}
+
+// List slots for the lanes that claim one: one returning add per converged group of lanes (rather
+// than one per lane, which serialises on the counter's address), each claimant's slot ranked by lane.
+// Returns -1 to the others.
+__device__ __forceinline__ int32_t claim_slot(int32_t* count, bool need) {
+  const unsigned act = __activemask();
+  const unsigned m = __ballot_sync(act, need);
+  if (m == 0u) return -1;
+  const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+  int32_t base = 0;
+  if (lane == leader) base = atomicAdd(count, __popc(m));
+  base = __shfl_sync(act, base, leader);
+  return need ? base + __popc(m & ((1u << lane) - 1u)) : -1;
 }
 
 // qmask[cluster] |= 1 << q for every cluster in query q's probe set (qmask zeroed beforehand).
@@ -1018,16 +1039,24 @@ __global__ void k_build_qmask(const int32_t* __restrict__ sel, int B, int p, uns
                               int32_t* list, int32_t* count, uint32_t* tile_flags, int64_t b,
                               int64_t rows, int tile_rows) {
   const int64_t n = (int64_t)B * p;
+  // a cluster of b rows overlaps at most this many tiles
+  const int64_t span = tile_flags ? (b - 1 + tile_rows - 1) / tile_rows + 1 : 1;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int32_t k = sel[i];
     const unsigned long long old = atomicOr(qmask + k, 1ull << (uint32_t)(i / p));
-    if (!list || old != 0ull) continue;
+    if (!list) continue;
+    const bool first = old == 0ull;
     if (!tile_flags) {
-      list[atomicAdd(count, 1)] = k;
+      const int32_t s = claim_slot(count, first);
+      if (first) list[s] = k;
     } else {
       const int64_t r0 = (int64_t)k * b, r1 = (r0 + b < rows ? r0 + b : rows) - 1;
-      for (int64_t t = r0 / tile_rows; t <= r1 / tile_rows; ++t)
-        if (atomicExch(tile_flags + t, 1u) == 0u) list[atomicAdd(count, 1)] = (int32_t)t;
+      for (int64_t j = 0; j < span; ++j) {
+        const int64_t t = r0 / tile_rows + j;
+        const bool mine = first && t <= r1 / tile_rows && atomicExch(tile_flags + t, 1u) == 0u;
+        const int32_t s = claim_slot(count, mine);
+        if (mine) list[s] = (int32_t)t;
+      }
     }
   }
 }

@@ -196,8 +196,9 @@ cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_s
 cudaError_t launch_gumbel_keys(const float* s, float* keys, int B, int64_t c, float tau,
                                uint64_t seed, uint64_t step, uint32_t rng_stream,
                                cudaStream_t st);
+// zero / zero_bytes (optional, a multiple of 4): a region cleared on the way, for the next kernel.
 cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p,
-                          cudaStream_t st);
+                          cudaStream_t st, void* zero = nullptr, size_t zero_bytes = 0);
 cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st);
 cudaError_t launch_dense(const DenseParams& prm, int elem, int num_sms, cudaStream_t st);
 cudaError_t launch_gather(const int32_t* C2T, int64_t b, const int32_t* sel, int B, int p,

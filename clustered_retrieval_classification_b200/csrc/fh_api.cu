@@ -260,6 +260,9 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
   // selection kernel that precedes their builder
   void* mask_region = (uni || tc) ? static_cast<void*>(base + L.qmask) : nullptr;
   const size_t mask_bytes = (uni || tc) ? qmask_region_bytes(D) : 0;
+  // the mask builder may overlap the selection kernel's tail unless a copy of the probe sets sits
+  // between them on the stream
+  const bool overlap = !(dbg && dbg->sel);
   if ((tc || uni) && tc_eligible(idx, B, kTcMinBatchStage1) && s1fmt(idx) == FH_STAGE1_DENSE) {
     // Stage 1 on the tensor cores too: keys[q][k] = C[k]·h_q (+ the Gumbel term when sampling)
     fh::TcParams tp = {};
@@ -305,7 +308,8 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     unsigned long long* qmask = reinterpret_cast<unsigned long long*>(base + L.qmask);
     int32_t* count = reinterpret_cast<int32_t*>(qmask + D.c) + tile_count_of(D);
     int32_t* list = reinterpret_cast<int32_t*>(base + L.tiles);
-    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count)) != cudaSuccess)
+    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count, nullptr, 0, 0, 128, overlap)) !=
+        cudaSuccess)
       return cuda_fail(e, "mask launch");
     fh::UnionParams up = {};
     up.E_perm = D.E_perm;
@@ -339,7 +343,8 @@ fh_status run_head(const fh_index* idx, const void* H, int B, int p, int sample,
     int32_t* count = reinterpret_cast<int32_t*>(flags + tile_count_of(D));
     int32_t* list = reinterpret_cast<int32_t*>(base + L.tiles);
     // the query masks and, as their clusters are first selected, the 128-row tiles that hold them
-    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count, flags, D.b, D.v, 128)) != cudaSuccess)
+    if ((e = fh::launch_build_qmask(sel, B, p, qmask, st, list, count, flags, D.b, D.v, 128, overlap)) !=
+        cudaSuccess)
       return cuda_fail(e, "mask launch");
     fh::TcParams tp = {};
     tp.rows = D.v;

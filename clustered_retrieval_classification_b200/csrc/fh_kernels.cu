@@ -22,6 +22,7 @@
 //   k_validate_c2t, k_build_perm                                                        (index load)
 //   k_mc_*                                                                              (Monte Carlo)
 #include <mutex>
+#include <utility>
 #include <unordered_map>
 
 #include "fh_kernels.cuh"
@@ -301,7 +302,10 @@ __global__ void __launch_bounds__(NT) k_select(const float* keys, int32_t* sel, 
                                                uint32_t* zero, int zero_words) {
   __shared__ SelectSmem<NT> sm;
   const int q = blockIdx.x;
+  pdl_launch_dependents();
+  // the cleared region was last read by an earlier call, which had finished before this call began
   for (int i = q * NT + (int)threadIdx.x; i < zero_words; i += (int)gridDim.x * NT) zero[i] = 0u;
+  pdl_wait_prior();  // the keys
   uint32_t key[KPT];
   load_key_images<KPT>(keys + (size_t)q * c, (int)c, key);
   block_select_topp<NT, KPT>(key, (int)c, p, sm, sel + (size_t)q * p);
@@ -544,9 +548,18 @@ __global__ void __launch_bounds__(NW * 32, 1) k_union_rows(const UnionParams prm
   __shared__ unsigned long long blk_best[NW][64];
   __shared__ bool is_last;
 
+  uint64_t* hbar = bars + NW * K;  // the query vectors
+  if (tid < NW * K + 1) mbar_init(&bars[tid], 1);
+  fence_mbar_init();
+  __syncthreads();
+  // The query vectors are inputs of the whole call, complete before its first kernel began, so they
+  // are requested before the wait for the mask builder, which may still be running.
+  if (tid == 0) issue_row(hs, prm.H, (uint32_t)prm.B * row_bytes, hbar);
+  pdl_wait_prior();
+
   // 32-bit row arithmetic: the union has at most v < 2^31 rows
   const uint32_t b = (uint32_t)prm.b;
-  const int n_cl = __ldg(prm.cl_count);
+  const int n_cl = __ldcg(prm.cl_count);
   const int64_t R = (int64_t)n_cl * b;
   const uint32_t lo = (uint32_t)(R * blockIdx.x / gridDim.x), hi = (uint32_t)(R * (blockIdx.x + 1) / gridDim.x);
   const uint32_t c_lo = lo / b;  // first listed cluster this block touches
@@ -561,13 +574,9 @@ __global__ void __launch_bounds__(NW * 32, 1) k_union_rows(const UnionParams prm
   uint8_t* ring_w = ring + (size_t)warp * K * row_bytes;
   uint64_t* bars_w = bars + warp * K;
 
-  uint64_t* hbar = bars + NW * K;  // the query vectors
-  if (tid < NW * K + 1) mbar_init(&bars[tid], 1);
-  fence_mbar_init();
-  for (uint32_t ci = c_lo + tid; ci < c_hi; ci += NW * 32) cl_s[ci - c_lo] = __ldg(prm.cl_list + ci);
+  for (uint32_t ci = c_lo + tid; ci < c_hi; ci += NW * 32) cl_s[ci - c_lo] = __ldcg(prm.cl_list + ci);
   __syncthreads();
-  // the query vectors (one bulk copy) and the first rows, then the token ids and the cluster masks
-  if (tid == 0) issue_row(hs, prm.H, (uint32_t)prm.B * row_bytes, hbar);
+  // the first rows, then the token ids and the cluster masks
   if (lane == 0)
     for (int n = 0; n < K && n < nw; ++n)
       issue_row(ring_w + (size_t)n * row_bytes, src(first + (uint32_t)(NW * n)), row_bytes, &bars_w[n]);
@@ -575,7 +584,7 @@ __global__ void __launch_bounds__(NW * 32, 1) k_union_rows(const UnionParams prm
     const uint32_t ci = i / b;
     tok_s[i - lo] = __ldg(prm.C2T + (size_t)cl_s[ci - c_lo] * b + (i - ci * b));
   }
-  for (uint32_t ci = c_lo + tid; ci < c_hi; ci += NW * 32) msk_s[ci - c_lo] = __ldg(prm.qmask + cl_s[ci - c_lo]);
+  for (uint32_t ci = c_lo + tid; ci < c_hi; ci += NW * 32) msk_s[ci - c_lo] = __ldcg(prm.qmask + cl_s[ci - c_lo]);
   const bool h_ok = mbar_wait(hbar, 0u, prm.status);
   if (!__syncthreads_and(h_ok)) {  // (status recorded) the rows already requested land first
     if (lane == 0)
@@ -585,11 +594,20 @@ __global__ void __launch_bounds__(NW * 32, 1) k_union_rows(const UnionParams prm
 
   const uint32_t hs_addr = smem_addr(hs);
   unsigned long long best0 = 0ull, best1 = 0ull;  // queries lane and lane + 32
+  // Sampling: the row's Gumbel terms are drawn before its dot products, lane l for queries l and
+  // l + 32 of the cluster's mask, all lanes at once (rather than one lane per (row, query) after the
+  // sum), so the draws overlap the products.
+  float g0 = 0.0f, g1 = 0.0f;
+  auto draw = [&](unsigned long long mk, uint32_t tok) {
+    if (mk >> lane & 1ull)
+      g0 = gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)lane, 1u, tok));
+    if (mk >> (lane + 32) & 1ull)
+      g1 = gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)(lane + 32), 1u, tok));
+  };
   auto fold = [&](int q, float z, uint32_t tok) {
     if (lane == (q & 31)) {
       float val = z;
-      if (prm.sample)
-        val = z / prm.tau + gumbel_from_u32(philox_word(prm.seed, prm.step, (uint32_t)q, 1u, tok));
+      if (prm.sample) val = z / prm.tau + (q < 32 ? g0 : g1);
       const unsigned long long pk = pack_best(val, tok);
       if (q < 32) best0 = pk > best0 ? pk : best0;
       else best1 = pk > best1 ? pk : best1;
@@ -614,6 +632,7 @@ __global__ void __launch_bounds__(NW * 32, 1) k_union_rows(const UnionParams prm
     const uint32_t row_s = smem_addr(ring_w + (size_t)slot * row_bytes);
     const uint32_t tok = (uint32_t)tok_s[i - lo];
     unsigned long long mk = msk_s[i / b - c_lo];
+    if (prm.sample) draw(mk, tok);
     if constexpr (RCH > 0) {
       // the row into registers, its slot refilled at once, then the cluster's queries two at a time
       uint4 ra[RCH];
@@ -919,6 +938,26 @@ static cudaError_t set_smem(Kern kern, size_t bytes) {
   return set_smem_attr(reinterpret_cast<const void*>(kern), bytes);
 }
 
+// Launch `kern` with programmatic stream serialisation when `overlap` is set: its blocks may be
+// scheduled once every block of the preceding kernel has signalled launch_dependents, and the kernel
+// waits (pdl_wait_prior) before it reads anything that kernel wrote.  Only for launches that follow
+// another kernel of the same call on the stream.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_k(bool overlap, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = overlap ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 cudaError_t set_smem_attr(const void* kernel, size_t bytes) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -1007,12 +1046,13 @@ cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int
                           void* zero, size_t zero_bytes) {
   uint32_t* z = static_cast<uint32_t*>(zero);
   const int zw = zero ? (int)(zero_bytes / 4) : 0;  // a few hundred KB at most
-  if (c <= 512 * 4) k_select<512, 4><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
-  else if (c <= 512 * 8) k_select<512, 8><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
-  else if (c <= 512 * 16) k_select<512, 16><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
-  else if (c <= 512 * 32) k_select<512, 32><<<B, 512, 0, st>>>(keys, sel, c, p, z, zw);
-  else k_select<1024, 32><<<B, 1024, 0, st>>>(keys, sel, c, p, z, zw);
-  return cudaGetLastError();
+  // a selection that clears the masks is the batched head's, right after its Stage-1 kernel
+  const bool ov = zero != nullptr;
+  if (c <= 512 * 4) return launch_k(ov, k_select<512, 4>, B, 512, 0, st, keys, sel, c, p, z, zw);
+  if (c <= 512 * 8) return launch_k(ov, k_select<512, 8>, B, 512, 0, st, keys, sel, c, p, z, zw);
+  if (c <= 512 * 16) return launch_k(ov, k_select<512, 16>, B, 512, 0, st, keys, sel, c, p, z, zw);
+  if (c <= 512 * 32) return launch_k(ov, k_select<512, 32>, B, 512, 0, st, keys, sel, c, p, z, zw);
+  return launch_k(ov, k_select<1024, 32>, B, 1024, 0, st, keys, sel, c, p, z, zw);
 }
 
 // List slots for the lanes that claim one: one returning add per converged group of lanes (rather
@@ -1038,11 +1078,13 @@ __device__ __forceinline__ int32_t claim_slot(int32_t* count, bool need) {
 __global__ void k_build_qmask(const int32_t* __restrict__ sel, int B, int p, unsigned long long* qmask,
                               int32_t* list, int32_t* count, uint32_t* tile_flags, int64_t b,
                               int64_t rows, int tile_rows) {
+  pdl_launch_dependents();
+  pdl_wait_prior();  // the probe sets and the cleared masks
   const int64_t n = (int64_t)B * p;
   // a cluster of b rows overlaps at most this many tiles
   const int64_t span = tile_flags ? (b - 1 + tile_rows - 1) / tile_rows + 1 : 1;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int32_t k = sel[i];
+    const int32_t k = __ldcg(sel + i);
     const unsigned long long old = atomicOr(qmask + k, 1ull << (uint32_t)(i / p));
     if (!list) continue;
     const bool first = old == 0ull;
@@ -1063,11 +1105,11 @@ __global__ void k_build_qmask(const int32_t* __restrict__ sel, int B, int p, uns
 
 cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
                                cudaStream_t st, int32_t* list, int32_t* count, uint32_t* tile_flags,
-                               int64_t b, int64_t rows, int tile_rows) {
+                               int64_t b, int64_t rows, int tile_rows, bool overlap) {
   const int64_t n = (int64_t)B * p;
   const int blocks = (int)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024);
-  k_build_qmask<<<blocks, 256, 0, st>>>(sel, B, p, qmask, list, count, tile_flags, b, rows, tile_rows);
-  return cudaGetLastError();
+  return launch_k(overlap, k_build_qmask, blocks, 256, 0, st, sel, B, p, qmask, list, count, tile_flags, b,
+                  rows, tile_rows);
 }
 
 int stage2_blocks(int64_t rows, int B, int num_sms) {
@@ -1145,10 +1187,10 @@ cudaError_t launch_union_rows(const UnionParams& prm, int elem, int num_sms, cud
   // rows of up to 256 16-byte chunks (4 KB) are held in registers, 8 chunks a lane
   const bool cached = row_bytes <= 256u * 16u;
   cudaError_t e;
-#define FH_UN(EL, W, R)                                                             \
-  do {                                                                              \
-    if ((e = set_smem(k_union_rows<EL, W, R>, smem)) != cudaSuccess) return e;      \
-    k_union_rows<EL, W, R><<<G, W * 32, smem, st>>>(prm, K, rows_max, cl_max);      \
+#define FH_UN(EL, W, R)                                                                      \
+  do {                                                                                       \
+    if ((e = set_smem(k_union_rows<EL, W, R>, smem)) != cudaSuccess) return e;               \
+    e = launch_k(true, k_union_rows<EL, W, R>, G, W * 32, smem, st, prm, K, rows_max, cl_max); \
   } while (0)
 #define FH_UN_W(EL, R)                 \
   do {                                 \
@@ -1163,7 +1205,7 @@ cudaError_t launch_union_rows(const UnionParams& prm, int elem, int num_sms, cud
   }
 #undef FH_UN_W
 #undef FH_UN
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_dense(const DenseParams& prm, int elem, int num_sms, cudaStream_t st) {

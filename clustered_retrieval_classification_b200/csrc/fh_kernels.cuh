@@ -143,7 +143,7 @@ cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms
 cudaError_t launch_build_qmask(const int32_t* sel, int B, int p, unsigned long long* qmask,
                                cudaStream_t st, int32_t* list = nullptr, int32_t* count = nullptr,
                                uint32_t* tile_flags = nullptr, int64_t b = 0, int64_t rows = 0,
-                               int tile_rows = 128);
+                               int tile_rows = 128, bool overlap = false);
 bool tc_int4_supported(int64_t d, int B, const void* scales);
 // INT4 Stage-1 keys on the tensor cores: out_keys[q][k] = Σ_j q4[k][j]·scale[k][j/32]·h_q[j] (or the
 // Gumbel key when sample != 0), dequantised to fp16 in shared memory (fh_tc.cu).
@@ -196,7 +196,8 @@ cudaError_t launch_stage1(const Stage1Params& prm, int elem, int int4, int num_s
 cudaError_t launch_gumbel_keys(const float* s, float* keys, int B, int64_t c, float tau,
                                uint64_t seed, uint64_t step, uint32_t rng_stream,
                                cudaStream_t st);
-// zero / zero_bytes (optional, a multiple of 4): a region cleared on the way, for the next kernel.
+// zero / zero_bytes (optional, a multiple of 4): a region cleared on the way, for the next kernel; a
+// call that passes one follows the Stage-1 kernel of the same head call and may overlap its tail.
 cudaError_t launch_select(const float* keys, int32_t* sel, int B, int64_t c, int p,
                           cudaStream_t st, void* zero = nullptr, size_t zero_bytes = 0);
 cudaError_t launch_stage2(const Stage2Params& prm, int elem, int num_sms, cudaStream_t st);

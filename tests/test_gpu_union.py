@@ -97,3 +97,22 @@ def test_union_reuses_one_workspace(fh, mid, mid_index):
     for _ in range(3):
         assert np.array_equal(fh.head_greedy(mid_index, Hd, idx.cfg.p, ws=ws).cpu().numpy(), ref)
     fh.ws_status(ws)
+
+
+@pytest.mark.parametrize("dtype,d,B,sample", [
+    ("bf16", 3072, 16, False),   # 6 KB rows: read from the ring in place, 8 warps (16 x 6 KB of queries)
+    ("bf16", 3072, 16, True),
+    ("bf16", 3072, 5, False),    # 12 warps with two slots each beside five query vectors
+    ("f32", 1536, 16, False),    # fp32 rows over 4 KB, 8 warps
+    ("f32", 768, 12, False),     # fp32 rows held in registers, 16 warps x 3 slots
+])
+def test_union_row_sizes_and_warp_splits(fh, orc, dtype, d, B, sample):
+    """The union kernel's other forms: rows too long to hold in registers (over 4 KB) and the warp
+    counts left when the query vectors crowd the ring, in BF16 and fp32 (the pair-wise dot products
+    and the early slot refill of register-held rows in fp32 too)."""
+    cfg = synth.dataclasses.replace(synth.scaled(synth.CONFIGS["llama"], v=8000, c=500, d=d, p=40,
+                                                 name=f"union-{dtype}-d{d}"), dtype=dtype)
+    idx = synth.make_index(cfg)
+    H = synth.make_queries(cfg, B)
+    check_head(fh, orc, idx, H, cfg.p, sample=sample, tau=0.8, seed=synth.SAMPLE_SEED, step=B,
+               batch=B, debug="sel")

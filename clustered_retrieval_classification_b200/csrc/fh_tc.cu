@@ -814,10 +814,13 @@ cudaError_t launch_tc_head(const void* A, const void* H, TcParams p, int num_sms
   // listed tiles (the kernel reads their count on the device): filled by the query-mask builder
   if (p.tile_list && (!p.qmask || !p.tile_count)) return cudaErrorInvalidValue;
   CUtensorMap mE, mH;
-  // copies of the queries where the epilogue bounds the kernel: the head modes, sampled keys, and
-  // keys of more than 32 queries (measured at the Llama-3.2-1B shape; below that the plain keys'
-  // epilogue is light, and copies multiply the query bytes each stage brings in)
-  tc_query_layout(p.B, !p.out_keys || p.sample || p.B > 32, p.qrows, p.copies);
+  // copies of the queries where the epilogue bounds the kernel: the head modes, sampled keys of 16
+  // queries or more, and keys of more than 32 queries (measured at the Llama-3.2-1B shape; below
+  // that the keys' epilogue is light enough, and copies multiply the query bytes each stage brings
+  // in: 64 KB of query rows beside 32 KB of centroid rows a stage.  Sampled head at 2 / 4 / 6 / 12
+  // queries without copies 52.5 / 64.7 / 73.3 / 103.4 µs against 55.0 / 67.0 / 75.3 / 104.7 with
+  // them; at 16, 120.9 against 119.5)
+  tc_query_layout(p.B, !p.out_keys || (p.sample && p.B >= 16) || p.B > 32, p.qrows, p.copies);
   // K-blocks per stage: the keys' small tiles fetch a row's consecutive K-blocks together
   p.kbs = p.out_keys ? FH_TC_KEYS_KBS : FH_TC_HEAD_KBS;
   if (!make_map(&mE, A, p.d, p.rows, box) || !make_map(&mH, H, p.d, p.B, (uint32_t)p.qrows))

@@ -95,6 +95,17 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+def tensor_peak():
+    """Dense BF16 tensor-core peak in TFLOP/s for a kernel timed inside long back-to-back runs: the
+    measured sustained cuBLAS figure, else this pool's earlier burst measurement."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 # ----------------------------------------------------------------------------- clocks
 
 
@@ -381,7 +392,14 @@ def sweep(F, T, R, cfg, idx, Hd, Hh, args, peak):
     for B in (1, 64):
         t, n, _ = T.b2b(dense_step(F, R, Hd, B), min(K, 32), W, repeats=3)
         t = statistics.median(t)
-        rec(f"dense_b{B}", t, n, B, costmodel.dense_bytes(cfg.v, cfg.d, B, 2))
+        extra = None
+        if B > 1:  # tensor cores: every MMA has 128 rows (the batch padded to 32 or 64 and copied)
+            tp, kind = tensor_peak()
+            issued, useful = 2.0 * 128 * cfg.v * cfg.d, 2.0 * B * cfg.v * cfg.d
+            tf = issued / (1e-3 * t / n) / 1e12
+            extra = {"mma": {"issued_tflop_per_call": issued / 1e12, "useful_tflop_per_call": useful / 1e12,
+                             "issued_tflops": tf, "peak_tflops": tp, "peak_kind": kind, "frac": tf / tp}}
+        rec(f"dense_b{B}", t, n, B, costmodel.dense_bytes(cfg.v, cfg.d, B, 2), extra)
     for B in (1, 4, 16, 64):
         t, n, _ = T.b2b(head_step(F, R, Hd, B, cfg.p, mode="sample"), K, W, repeats=3)
         t = statistics.median(t)

@@ -821,7 +821,8 @@ def main():
     achieved = bytes_call / (us_call * 1e-6) / 1e9
     iso = T.isolated(step, min(args.steps, 200), args.warmup)
 
-    # end to end through the public API with pinned host buffers (eager, back to back)
+    # end to end through the public API with pinned host buffers (eager, back to back): one
+    # fh_head_greedy_host call a step queues the query copy, the head and the token copy
     h_host = torch.from_numpy(Hh.view(np.int16)).view(torch.bfloat16).pin_memory()
     tok_host = torch.empty((len(R.handles), B), dtype=torch.int32).pin_memory()
     h_dev = torch.empty((B, cfg.d), dtype=torch.bfloat16, device="cuda")
@@ -832,9 +833,7 @@ def main():
     def e2e_step(k):
         r = k % len(R.handles)
         off = (k * B) % (1024 - B + 1)
-        h_dev.copy_(h_host[off:off + B], non_blocking=True)
-        F.head_greedy(R[r], h_dev, cfg.p, out=tok_dev, ws=e2e_ws[r])
-        tok_host[r].copy_(tok_dev, non_blocking=True)
+        F.head_greedy_host(R[r], h_host[off:off + B], cfg.p, tok_host[r], h_dev, tok_dev, ws=e2e_ws[r])
     for k in range(args.warmup):
         e2e_step(k)
     T.barrier()

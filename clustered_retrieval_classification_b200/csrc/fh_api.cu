@@ -536,6 +536,24 @@ fh_status fh_head_greedy(const fh_index* idx, const void* H, int B, int p, int32
                   static_cast<cudaStream_t>(stream), dbg);
 }
 
+fh_status fh_head_greedy_host(const fh_index* idx, const void* H_host, int B, int p, int32_t* tok_host,
+                              void* h_dev, int32_t* tok_dev, void* ws, size_t ws_bytes, fh_stream stream) {
+  FH_NVTX_RANGE("fh_head_greedy_host");
+  fh_status s = check_batch(idx, h_dev, B);
+  if (s != FH_OK) return s;
+  if (!H_host || !tok_host || !tok_dev) return fail(FH_ERR_ARG, "H_host, tok_host or tok_dev is NULL");
+  if (p < 1 || p > idx->desc.c) return fail(FH_ERR_ARG, "p=%d outside [1, c=%lld]", p, (long long)idx->desc.c);
+  if ((s = check_ws(ws, ws_bytes, layout_for(idx, FH_OP_GREEDY, B, p, 0, 0).total)) != FH_OK) return s;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t h_bytes = (size_t)B * (size_t)idx->desc.d * (idx->desc.dtype == FH_BF16 ? 2u : 4u);
+  cudaError_t e = cudaMemcpyAsync(h_dev, H_host, h_bytes, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "query copy");
+  if ((s = run_head(idx, h_dev, B, p, 0, 1.0f, 0, 0, tok_dev, ws, ws_bytes, st, nullptr)) != FH_OK) return s;
+  if ((e = cudaMemcpyAsync(tok_host, tok_dev, (size_t)B * 4u, cudaMemcpyDeviceToHost, st)) != cudaSuccess)
+    return cuda_fail(e, "token copy");
+  return FH_OK;
+}
+
 fh_status fh_head_sample(const fh_index* idx, const void* H, int B, int p, float tau, uint64_t seed,
                          uint64_t step, int32_t* out_tok, void* ws, size_t ws_bytes,
                          fh_stream stream, const fh_debug_out* dbg) {

@@ -71,6 +71,7 @@ SIGNATURES = {
     "fh_ws_status": (_i, [_p, _p]),
     "fh_last_error": (ct.c_char_p, []),
     "fh_head_greedy": (_i, [_p, _p, _i, _i, _p, _p, _sz, _p, _p]),
+    "fh_head_greedy_host": (_i, [_p, _p, _i, _i, _p, _p, _p, _p, _sz, _p]),
     "fh_head_sample": (_i, [_p, _p, _i, _i, _f, _u64, _u64, _p, _p, _sz, _p, _p]),
     "fh_mc_token_prob": (_i, [_p, _p, _i, _p, _i, _i, _f, _i64, _u64, _p, _p, _p, _sz, _p]),
     "fh_mc_token_prob_range": (_i, [_p, _p, _i, _p, _i, _i, _f, _i64, _i64, _u64, _p, _p, _p, _sz, _p]),
@@ -218,6 +219,23 @@ def head_greedy(index: Index, H, p, out=None, ws=None, stream=None, debug=None):
     _check(load().fh_head_greedy(index.handle, _ptr(H), B, p, _ptr(out), _ptr(ws), ws.numel(),
                                  _stream(stream), _debug(debug)))
     return out
+
+
+def head_greedy_host(index: Index, H_host, p, tok_host, h_dev, tok_dev, ws=None, stream=None):
+    """head_greedy with host buffers: H_host (CPU, [B, d], pinned for an asynchronous copy) is copied
+    to h_dev, the head runs into tok_dev, and the tokens are copied to tok_host (CPU int32 [B]), all
+    queued on the stream in one library call; tok_host is valid once the stream has synchronised."""
+    _need(h_dev, "h_dev")
+    _need(tok_dev, "tok_dev")
+    if H_host.is_cuda or tok_host.is_cuda or not H_host.is_contiguous() or not tok_host.is_contiguous():
+        raise ValueError("H_host and tok_host must be contiguous host tensors")
+    B = H_host.shape[0]
+    if h_dev.shape != H_host.shape or h_dev.dtype != H_host.dtype or tok_dev.numel() < B or tok_host.numel() < B:
+        raise ValueError("staging buffers do not match the queries")
+    ws = ws if ws is not None else index.workspace(FH_OP_GREEDY, B, p)
+    _check(load().fh_head_greedy_host(index.handle, _ptr(H_host), B, p, _ptr(tok_host), _ptr(h_dev),
+                                      _ptr(tok_dev), _ptr(ws), ws.numel(), _stream(stream)))
+    return tok_host
 
 
 def head_sample(index: Index, H, p, tau, seed, step, out=None, ws=None, stream=None, debug=None):

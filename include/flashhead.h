@@ -158,14 +158,24 @@ const char* fh_last_error(void);
    For each query q: S_q = the p clusters with the largest s_q = C·h_q; candidates = the p·b tokens of
    S_q through C2T; out_tok[q] = argmax of their exact logits z_t = E[t]·h_q (fp32 accumulation).
    out_tok: device, B int32.  dbg: optional intermediate outputs, or NULL.
-   Execution (all paths compute the same thing): B = 1 runs one persistent kernel; BF16 batches of 12
-   or more run Stage 1 and Stage 2 on the tensor cores, reading each needed E row once for the whole
-   batch (dbg->cand_tok or dbg->cand_logit force the per-query Stage 2 instead; dbg->sel alone does
-   not); other batches run per-query CUDA-core
-   kernels.  The paths sum the fp32 logits in different orders, so their tokens can differ only where
-   two candidates' logits are within that rounding (~1e-6 relative); each path is deterministic. */
+   Execution (all paths compute the same thing): B = 1 runs one persistent kernel; batches of 2 to 16
+   stream the union of their probe sets once on the CUDA cores (Stage 1 on the tensor cores in BF16),
+   and BF16 batches above 16 run both stages on the tensor cores, each needed E row read once for the
+   whole batch (dbg->cand_tok or dbg->cand_logit force the per-query CUDA-core Stage 2 instead;
+   dbg->sel alone does not).  The paths sum the fp32 logits in different orders, so their tokens can
+   differ only where two candidates' logits are within that rounding (~1e-6 relative); each path is
+   deterministic. */
 fh_status fh_head_greedy(const fh_index* idx, const void* H, int B, int p, int32_t* out_tok,
                          void* ws, size_t ws_bytes, fh_stream stream, const fh_debug_out* dbg);
+
+/* fh_head_greedy with host buffers, the call a host-side decode loop makes: copies H_host (host,
+   B x d of the index's dtype; pinned memory keeps the copy asynchronous) to h_dev (device, the same
+   size, 16-byte aligned), runs fh_head_greedy into tok_dev (device, B int32) and copies the tokens
+   to tok_host (host, B int32).  All three steps are queued on `stream`; tok_host holds the tokens
+   once the stream has synchronised.  The staging buffers h_dev and tok_dev belong to the caller and
+   are overwritten; arguments are checked before anything is queued, with fh_head_greedy's codes. */
+fh_status fh_head_greedy_host(const fh_index* idx, const void* H_host, int B, int p, int32_t* tok_host,
+                              void* h_dev, int32_t* tok_dev, void* ws, size_t ws_bytes, fh_stream stream);
 
 /* Sampling FlashHead head (FlashHead notes, Module 2 sampling mode and Eq. 3; FlashHead summary,
    Abstract item (3)).  Stage 1 draws p clusters without replacement from softmax(s_q/τ) as the top p of

@@ -66,6 +66,7 @@ def test_host_side_argument_checks(lib):
     assert L.fh_index_load_ws_bytes(ct.byref(desc)) >= 1024 + 16
     # calls on a NULL handle
     assert L.fh_head_greedy(None, None, 1, 1, None, None, 0, None, None) == 1
+    assert L.fh_head_greedy_host(None, None, 1, 1, None, None, None, None, 0, None) == 1
     assert L.fh_workspace_bytes(None, 0, 1, 1, 1, 1) == 0
     assert L.fh_select_topp(None, 1, 8, 2, None, None) == 1
     assert L.fh_philox_u32(0, 0, 0, 0, 0, None, None) == 1

@@ -312,6 +312,26 @@ def test_batch1_without_debug_outputs_on_one_workspace(fh, orc, mid):
     assert checked >= 2
 
 
+@pytest.mark.parametrize("B", [1, 5])
+def test_head_greedy_host_buffers(fh, mid, B):
+    """fh_head_greedy_host (host query and token buffers, both copies queued by the library) gives
+    the tokens of fh_head_greedy on the same queries, call after call on one workspace."""
+    idx, H = mid
+    cfg = idx.cfg
+    I = load(fh, idx)
+    ws = I.workspace(fh.FH_OP_GREEDY, B, cfg.p)
+    h_dev = torch.empty((B, cfg.d), dtype=dev(H[:1], cfg.dtype).dtype, device=DEV)
+    tok_dev = torch.empty(B, dtype=torch.int32, device=DEV)
+    tok_host = torch.empty(B, dtype=torch.int32).pin_memory()
+    for k in range(3):
+        Hd = dev(H[k:k + B], cfg.dtype)
+        ref = fh.head_greedy(I, Hd, cfg.p).cpu().numpy()
+        fh.head_greedy_host(I, Hd.cpu().pin_memory(), cfg.p, tok_host, h_dev, tok_dev, ws=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(tok_host.numpy(), ref), k
+    fh.ws_status(ws)
+
+
 def test_bounded_wait_times_out_and_workspace_recovers(fh, mid):
     """Failure detection without a fault: one histogram bin of the workspace is pre-set so that the
     batch-1 kernel's grid barrier (a bounded poll of the histogram until its counts reach c) can never
